@@ -1,0 +1,405 @@
+#!/usr/bin/env python
+"""Benchmark of the fully-integer attention forward on B200.
+
+One step = one IntAttention forward (int8 Q.K^T -> IndexSoftmax -> u8 x s8
+P.V -> int8) over one batch of the workload, through the C ABI.  Default
+workload: BERT-base batch, B=8 H=12 L=512 d=64, non-causal.
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME]
+  python bench.py --impl reference ...   # the CPU oracle, timed on host cores
+
+Rank 0 prints one JSON line.  Timing: CUDA events on the launching stream,
+max over ranks; inputs rotate over enough copies to exceed the 126 MB L2.
+"""
+from __future__ import annotations
+
+import argparse
+import datetime
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+METRIC = "IntAttention fwd effective int8 TOPS & % of INT8 tensor roofline; decode GB/s"
+L2_BYTES = 126 * 1024 * 1024
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+INT8_OVER_BF16 = 2.0  # nominal dense ratio: 4.5 POPS int8 / 2.25 PFLOP/s bf16
+
+
+def parse_args(argv=None):
+    p = argparse.ArgumentParser()
+    p.add_argument("--gpus", type=int, default=1)
+    p.add_argument("--steps", type=int, default=200)
+    p.add_argument("--warmup", type=int, default=10)
+    p.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    p.add_argument("--workload", default="bert_base_b8_l512")
+    p.add_argument("--decode-workload", default="llama7b_decode_b64_lk4096")
+    p.add_argument("--no-decode", action="store_true")
+    p.add_argument("--no-cpu-baseline", action="store_true")
+    p.add_argument("--cpu-seconds", type=float, default=12.0)
+    return p.parse_args(argv)
+
+
+# ------------------------------------------------------------ distributed
+def dist_env():
+    return (int(os.environ.get("RANK", "0")), int(os.environ.get("LOCAL_RANK", "0")),
+            int(os.environ.get("WORLD_SIZE", "1")))
+
+
+def init_dist(world: int, backend: str):
+    import torch.distributed as dist
+    if world > 1 and not dist.is_initialized():
+        dist.init_process_group(backend=backend, timeout=datetime.timedelta(seconds=120))
+    return dist
+
+
+def max_over_ranks(x: float, world: int, device=None) -> float:
+    """Largest value of x over all ranks (the slowest rank sets the time)."""
+    if world <= 1:
+        return float(x)
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([float(x)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def barrier(world: int, device=None):
+    if world > 1:
+        import torch.distributed as dist
+        if device is not None and device.type == "cuda":
+            dist.barrier(device_ids=[device.index])
+        else:
+            dist.barrier()
+
+
+def aggregate_value(per_rank_units: float, world: int, seconds: float) -> float:
+    """Whole-job throughput: units every rank processed / the max-over-ranks time."""
+    return per_rank_units * world / seconds
+
+
+# ------------------------------------------------------------------ peaks
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            d = json.load(f)
+        return d, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+def kernel_traffic(kernel: str, workload: str):
+    """DRAM bytes per launch from a committed ncu summary, only while the
+    kernel source still has the hash the counters were taken with."""
+    import hashlib
+    path = os.path.join(ROOT, "profiles", "traffic.json")
+    if not os.path.exists(path):
+        return None
+    with open(path) as f:
+        table = json.load(f)
+    ent = table.get(kernel, {}).get(workload)
+    if not ent:
+        return None
+    h = hashlib.sha256()
+    for rel in ent.get("sources", []):
+        with open(os.path.join(ROOT, rel), "rb") as f:
+            h.update(f.read())
+    if h.hexdigest()[:16] != ent.get("source_hash"):
+        return None
+    return ent.get("bytes_per_launch")
+
+
+# ----------------------------------------------------------------- clocks
+class ClockSampler:
+    """nvidia-smi clocks and throttle reasons sampled every 200 ms."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.path = None
+
+    def start(self):
+        try:
+            fd, self.path = tempfile.mkstemp(suffix=".csv")
+            os.close(fd)
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "200", "-f", self.path],
+                stdout=subprocess.DEVNULL, stderr=subprocess.DEVNULL)
+        except (OSError, FileNotFoundError):
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        time.sleep(0.25)
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        rows = []
+        with open(self.path) as f:
+            for line in f:
+                parts = [p.strip() for p in line.split(",")]
+                if len(parts) >= 9:
+                    rows.append(parts)
+        os.unlink(self.path)
+        if not rows:
+            return None
+        sm = [float(r[1]) for r in rows if r[1].replace(".", "").isdigit()]
+        smax = [float(r[2]) for r in rows if r[2].replace(".", "").isdigit()]
+        pw = [float(r[3]) for r in rows if r[3].replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({n for r in rows for n, v in zip(names, r[5:9]) if v.strip().lower() == "active"})
+        loaded = [s for s, p in zip(sm, pw) if p >= 0.5 * max(pw)] if pw else sm
+        return {"sm_mhz": statistics.median(loaded or sm) if sm else None,
+                "sm_max_mhz": max(smax) if smax else None,
+                "power_w_max": max(pw) if pw else None,
+                "samples": len(rows), "reasons": reasons}
+
+
+# ------------------------------------------------------------- our arm
+def _int8_peak(peaks, sustained: bool):
+    key = "bf16_tflops_sustained" if sustained and "bf16_tflops_sustained" in peaks else "bf16_tflops"
+    return peaks[key] * INT8_OVER_BF16, key
+
+
+def run_ours(args):
+    import numpy as np
+    import torch
+
+    import integer_only_quantized_b200 as ia
+    from integer_only_quantized_b200 import workloads as wl
+
+    rank, local_rank, world = dist_env()
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    init_dist(world, "nccl")
+    w = wl.WORKLOADS[args.workload]
+    assert not w.decode, "the headline workload is a prefill workload"
+    x = wl.make_inputs(w)
+    sc = ia.Scales(x.s_q, x.s_k, x.s_v, x.s_o, per_head=w.per_head)
+    set_bytes = x.q.nbytes + x.k.nbytes + x.v.nbytes + x.q.nbytes
+    nsets = max(2, min(64, math.ceil(2 * L2_BYTES / set_bytes)))
+    q0, k0, v0 = (torch.from_numpy(a).to(dev) for a in (x.q, x.k, x.v))
+    sets = [(q0.clone(), k0.clone(), v0.clone(), torch.empty_like(q0)) for _ in range(nsets)]
+    stream = torch.cuda.current_stream(dev)
+
+    def step(i):
+        q, k, v, o = sets[i % nsets]
+        ia.forward(q, k, v, sc, w.causal, w.clip_c, out=o, stream=stream)
+
+    for i in range(args.warmup):
+        step(i)
+    torch.cuda.synchronize(dev)
+    if ia.device_error(stream) != ia.OK:
+        raise RuntimeError("a kernel wait timed out during warm-up")
+    clocks = ClockSampler(local_rank)
+    barrier(world, dev)
+    torch.cuda.synchronize(dev)
+    clocks.start()
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    t0.record(stream)
+    for i in range(args.steps):
+        step(i)
+    t1.record(stream)
+    torch.cuda.synchronize(dev)
+    barrier(world, dev)
+    clk = clocks.stop()
+    ms = t0.elapsed_time(t1) / args.steps
+    ms = max_over_ranks(ms, world, dev)
+    if ia.device_error(stream) != ia.OK:
+        raise RuntimeError("a kernel wait timed out during the timed steps")
+    ops = w.effective_ops
+    value = aggregate_value(ops, world, ms * 1e-3) / 1e12
+
+    # end to end through the public API with pinned HOST buffers
+    hq, hk, hv = (torch.from_numpy(a).pin_memory() for a in (x.q, x.k, x.v))
+    ho = torch.empty(x.q.shape, dtype=torch.int8).pin_memory()
+
+    def e2e_step(i):
+        q, k, v, o = sets[i % nsets]
+        q.copy_(hq, non_blocking=True)
+        k.copy_(hk, non_blocking=True)
+        v.copy_(hv, non_blocking=True)
+        ia.forward(q, k, v, sc, w.causal, w.clip_c, out=o, stream=stream)
+        ho.copy_(o, non_blocking=True)
+
+    for i in range(args.warmup):
+        e2e_step(i)
+    torch.cuda.synchronize(dev)
+    barrier(world, dev)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for i in range(args.steps):
+        e2e_step(i)
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    barrier(world, dev)
+    e2e_ms = max_over_ranks(e0.elapsed_time(e1) / args.steps, world, dev)
+    e2e_val = aggregate_value(ops, world, e2e_ms * 1e-3) / 1e12
+
+    peaks, peak_src = load_peaks()
+    peak_int8, peak_key = _int8_peak(peaks, sustained=False)
+    achieved = ops / (ms * 1e-3) / 1e12  # one launch per step: per-launch duration = ms
+    traffic = kernel_traffic("prefill_kernel", w.name)
+    line = {
+        "metric": METRIC, "value": round(value, 3), "unit": "TOPS", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms, 5),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "int8", "data": "synthetic",
+        "config": {"workload": w.name, "B": w.B, "H": w.H, "Lq": w.Lq, "Lk": w.Lk, "d": w.d,
+                   "causal": w.causal, "clip_c": w.clip_c,
+                   "quant": "per_head" if w.per_head else "per_tensor",
+                   "l2": f"inputs rotate over {nsets} copies ({nsets * set_bytes / 2**20:.0f} MiB > 126 MiB L2)",
+                   "parallelism": f"dp{world} (independent problems)"},
+        "roofline": {"bound": "tensor", "kernel": "prefill_kernel", "achieved": round(achieved, 3),
+                     "peak": round(peak_int8, 1), "unit": "TOPS", "frac": round(achieved / peak_int8, 4),
+                     "peak_source": f"{peak_src} {peak_key} x {INT8_OVER_BF16} (dense int8/bf16)",
+                     "traffic": traffic},
+        "e2e": {"value": round(e2e_val, 3), "unit": "TOPS",
+                "h2d_bytes_per_step": int(x.q.nbytes + x.k.nbytes + x.v.nbytes),
+                "d2h_bytes_per_step": int(x.q.nbytes), "ms_per_step": round(e2e_ms, 5)},
+        "gpu_launches": args.steps,
+        "clocks": clk,
+    }
+
+    if not args.no_decode:
+        line["decode"] = run_decode(args, dev, stream, world, peaks, peak_src)
+    if not args.no_cpu_baseline and rank == 0 and world == 1:
+        line["cpu_baseline"] = cpu_baseline(w, x, args.cpu_seconds)
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+
+
+def run_decode(args, dev, stream, world, peaks, peak_src):
+    """Decode over the int8 KV cache: GB/s of K/V cache rows + q + out."""
+    import torch
+
+    import integer_only_quantized_b200 as ia
+    from integer_only_quantized_b200 import workloads as wl
+    w = wl.WORKLOADS[args.decode_workload]
+    x = wl.make_inputs_torch(w, dev)
+    sc = ia.Scales(x.s_q, x.s_k, x.s_v, x.s_o, per_head=w.per_head)
+    ws = torch.empty(ia.decode_workspace_size(w.B, w.H, w.Lk, w.d), dtype=torch.uint8, device=dev)
+    out = torch.empty_like(x.q)
+    steps = max(10, min(args.steps, 100))
+    for _ in range(max(3, args.warmup)):
+        ia.decode(x.q, x.k, x.v, sc, w.Lk, w.clip_c, out=out, workspace=ws, stream=stream)
+    torch.cuda.synchronize(dev)
+    barrier(world, dev)
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    t0.record(stream)
+    for _ in range(steps):
+        ia.decode(x.q, x.k, x.v, sc, w.Lk, w.clip_c, out=out, workspace=ws, stream=stream)
+    t1.record(stream)
+    torch.cuda.synchronize(dev)
+    barrier(world, dev)
+    ms = max_over_ranks(t0.elapsed_time(t1) / steps, world, dev)
+    if ia.device_error(stream) != ia.OK:
+        raise RuntimeError("a kernel wait timed out in decode")
+    gbs = w.decode_bytes / (ms * 1e-3) / 1e9
+    return {"workload": w.name, "value": round(aggregate_value(w.decode_bytes, world, ms * 1e-3) / 1e9, 1),
+            "unit": "GB/s", "ms_per_call": round(ms, 5), "launches_per_call": 2,
+            "bytes_per_call": int(w.decode_bytes),
+            "roofline": {"bound": "hbm", "achieved": round(gbs, 1), "peak": peaks["hbm_gbs"],
+                         "unit": "GB/s", "frac": round(gbs / peaks["hbm_gbs"], 4),
+                         "peak_source": f"{peak_src} hbm_gbs", "traffic": None},
+            "l2": "K/V caches 2 GiB > 126 MiB L2"}
+
+
+# ------------------------------------------------------- CPU oracle legs
+def _oracle_sample(w, x, seconds: float):
+    """Time the oracle on whole (b, h) slices until about `seconds` of work."""
+    import oracle
+    threads = os.cpu_count() or 1
+    oracle.build()
+    heads = [(b, h) for b in range(w.B) for h in range(w.H)]
+
+    def run(n):
+        sel = heads[:n]
+        done = 0.0
+        t = time.perf_counter()
+        for b in sorted({b for b, _ in sel}):
+            hs = [h for bb, h in sel if bb == b]
+            sl = slice(hs[0], hs[-1] + 1)
+            hsc = (lambda s: s[sl] if w.per_head else s)
+            oracle.forward(x.q[b:b + 1, sl], x.k[b:b + 1, sl], x.v[b:b + 1, sl], w.per_head,
+                           hsc(x.s_q), hsc(x.s_k), hsc(x.s_v), hsc(x.s_o), w.causal, w.clip_c,
+                           nthreads=threads)
+            done += len(hs)
+        return time.perf_counter() - t, done
+
+    dt, n = run(1)
+    per_head = max(dt, 1e-6)
+    want = int(min(len(heads), max(1, seconds / per_head)))
+    if want > 1:
+        dt, n = run(want)
+    ops = w.effective_ops / (w.B * w.H) * n
+    return ops, dt, threads, f"{int(n)} of {w.B * w.H} (b, h) slices of {w.name}, all their rows"
+
+
+def cpu_baseline(w, x, seconds):
+    ops, dt, threads, sample = _oracle_sample(w, x, seconds)
+    return {"value": round(ops / dt / 1e12, 6), "unit": "TOPS", "cores": threads, "kind": "oracle",
+            "sample": sample, "seconds": round(dt, 2)}
+
+
+def run_reference(args):
+    from integer_only_quantized_b200 import workloads as wl
+    rank, _, world = dist_env()
+    if rank != 0:
+        return  # only rank 0 times the oracle; the other ranks do no work
+    w = wl.WORKLOADS[args.workload]
+    x = wl.make_inputs(w)
+    per_step = max(0.5, 120.0 / max(1, args.steps + args.warmup))
+    for _ in range(args.warmup):
+        _oracle_sample(w, x, per_step)
+    total_ops, total_t = 0.0, 0.0
+    sample = threads = None
+    for _ in range(args.steps):
+        ops, dt, threads, sample = _oracle_sample(w, x, per_step)
+        total_ops += ops
+        total_t += dt
+    value = total_ops / total_t / 1e12
+    line = {"metric": METRIC, "value": round(value, 6), "unit": "TOPS", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": round(1e3 * total_t / args.steps, 3), "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "int8", "data": "synthetic",
+            "impl": "reference",
+            "config": {"workload": w.name, "B": w.B, "H": w.H, "Lq": w.Lq, "Lk": w.Lk, "d": w.d,
+                       "causal": w.causal, "clip_c": w.clip_c,
+                       "quant": "per_head" if w.per_head else "per_tensor"},
+            "cpu_baseline": {"value": round(value, 6), "unit": "TOPS", "cores": threads,
+                             "kind": "oracle", "sample": f"each step: {sample}"},
+            "e2e": {"value": round(value, 6), "unit": "TOPS", "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+def main(argv=None):
+    args = parse_args(argv)
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_ours(args)
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,128 @@
+/*
+ * intattn.h -- C ABI of the B200 (sm_100a) fully-integer attention forward.
+ *
+ * Method: IntAttention (arXiv 2511.21513), as summarised on the euno.news
+ * pages "IntAttention: a fully-integer attention pipeline for efficient edge
+ * inference" (Chinese and Korean editions), section "Methodology":
+ *   item 2  IndexSoftmax -- the int32 attention scores are clipped by a
+ *           sparsity-aware threshold, looked up in a 32-entry exp table, the
+ *           looked-up pseudo-exponentials are summed in int32 and scaled by a
+ *           reciprocal with an integer multiply and a right shift;
+ *   item 3  Q.K^T and V.softmax stay in the integer domain (end-to-end INT8).
+ * The pages fix no constant, rounding rule or width.  The exact definition
+ * this library computes (identical, bit for bit, to the CPU oracle that the
+ * tests compare it with) is:
+ *
+ *   per head h:  alpha = s_q s_k / sqrt(d);  r = alpha * 31 / c
+ *                s = 26, lowered while llround(r 2^s) > 2^24;  M = llround(r 2^s)
+ *                D = ceil(61 2^(s-1) / M)   (smallest gap with index 31)
+ *                LUT[i] = llround(2^15 exp(-i c / 31)), i < 31;  LUT[31] = 0
+ *                s_v / (255 s_o) = f 2^e, f in [0.5,1):  Mo = llround(f 2^31),
+ *                so = 31 - e  (Mo == 2^31 -> Mo = 2^30, so - 1)
+ *   per row i:   S_j = sum_t Q[i,t] K[j,t] over valid keys j (causal: j <= i + Lk - Lq)
+ *                m = max_j S_j;  idx_j = (min(m - S_j, D) M + 2^(s-1)) >> s
+ *                E_j = LUT[idx_j];  Z = sum_j E_j  (int32)
+ *                R = floor((255 2^32 + floor(Z/2)) / Z)
+ *                P_j = (E_j R + 2^31) >> 32        (u8, sums to about 255)
+ *                acc_t = sum_j P_j V[j,t]          (int32)
+ *                out_t = clamp((acc_t Mo + 2^(so-1)) >> so, -127, 127)  (floor shift)
+ *
+ * Conventions for every entry point:
+ *   - Tensor pointers are DEVICE pointers, 16-byte aligned, row-major and
+ *     contiguous with the innermost dimension d.  The caller owns them.
+ *   - The library allocates and frees nothing, never synchronises the stream
+ *     (except intattn_device_error), and launches only on the given stream.
+ *     Calls are asynchronous: a 0 return means the work was enqueued.
+ *   - Scale arrays are HOST pointers, read during the call only.
+ *   - d must be 64 or 128; 1 <= Lk <= 65535 (keeps Z < 2^31).
+ *   - Return codes are the INTATTN_* values below; on any non-zero return
+ *     nothing was launched (INTATTN_ERR_CUDA: a launch was refused).
+ */
+#ifndef INTATTN_H
+#define INTATTN_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* cudaStream_t without requiring the CUDA headers (same underlying type). */
+typedef struct CUstream_st *intattn_stream_t;
+
+enum {
+    INTATTN_OK = 0,
+    INTATTN_ERR_INVALID_ARG = 1,  /* null pointer, negative size, causal with Lq > Lk, Lk out of range */
+    INTATTN_ERR_UNSUPPORTED = 2,  /* d not 64/128, misaligned pointer, too many heads */
+    INTATTN_ERR_PARAM_RANGE = 3,  /* scale or clip not finite / not > 0; M or so out of range */
+    INTATTN_ERR_CUDA = 4,         /* a CUDA launch or driver call failed */
+    INTATTN_ERR_WORKSPACE = 5,    /* decode workspace missing or too small */
+    INTATTN_ERR_TIMEOUT = 6       /* a kernel wait ran out (reported by intattn_device_error) */
+};
+
+/* Largest H for per-head scales (the per-head parameters travel as kernel
+ * arguments). */
+#define INTATTN_MAX_HEADS 128
+
+/* Quantisation scales (real value = scale * int8 code).  per_head = 0: each
+ * array holds one entry shared by all heads; per_head = 1: H entries. */
+typedef struct intattn_scales {
+    int32_t per_head;
+    const float *s_q;
+    const float *s_k;
+    const float *s_v;
+    const float *s_o;
+} intattn_scales_t;
+
+/* Derived integer parameters of one head (see the definition above). */
+typedef struct intattn_head_params {
+    int32_t M;   /* index multiplier            */
+    int32_t s;   /* index shift, 1..26          */
+    int32_t D;   /* gap clip                    */
+    int32_t Mo;  /* requantisation multiplier   */
+    int32_t so;  /* requantisation shift, 1..62 */
+} intattn_head_params_t;
+
+/* Host-only: derive the LUT and the per-head parameters exactly as the
+ * kernels use them.  lut: 32 entries; out: H entries.  No GPU needed. */
+int intattn_derive_params(const intattn_scales_t *scales, int H, int d, float clip_c,
+                          int32_t lut[32], intattn_head_params_t *out);
+
+/* Prefill / full forward (IntAttention "Methodology" items 2-3).
+ *   q   [B, H, Lq, d] int8      k, v [B, H, Lk, d] int8      out [B, H, Lq, d] int8
+ *   causal != 0: key j is visible to query i iff j <= i + (Lk - Lq) (requires Lq <= Lk).
+ *   clip_c: the sparsity-aware clip threshold, in logit units (> 0).
+ * B*H*Lq == 0 returns INTATTN_OK without a launch. */
+int intattn_forward(const int8_t *q, const int8_t *k, const int8_t *v,
+                    const intattn_scales_t *scales, int B, int H, int Lq, int Lk, int d,
+                    int causal, float clip_c, int8_t *out, intattn_stream_t stream);
+
+/* Bytes of device workspace intattn_decode needs for these sizes. */
+size_t intattn_decode_workspace_size(int B, int H, int Lk, int d);
+
+/* Decode: one query per (b, h) against the first Lk rows of an int8 KV cache
+ * of capacity Lmax rows (same definition with Lq = 1, no mask).
+ *   q [B, H, 1, d]   k_cache, v_cache [B, H, Lmax, d]   out [B, H, 1, d]
+ *   workspace: caller-owned device buffer of at least
+ *   intattn_decode_workspace_size(B, H, Lk, d) bytes, 256-byte aligned; its
+ *   contents need no initialisation and are overwritten.  Calls that share a
+ *   workspace must be ordered on one stream. */
+int intattn_decode(const int8_t *q, const int8_t *k_cache, const int8_t *v_cache,
+                   const intattn_scales_t *scales, int B, int H, int Lk, int Lmax, int d,
+                   float clip_c, int8_t *out, void *workspace, size_t workspace_bytes,
+                   intattn_stream_t stream);
+
+/* Synchronises `stream`, then returns and clears the device error word that a
+ * kernel sets when one of its bounded waits runs out (INTATTN_ERR_TIMEOUT), or
+ * INTATTN_OK.  INTATTN_ERR_CUDA if the synchronisation itself fails. */
+int intattn_device_error(intattn_stream_t stream);
+
+/* Static description of a return code. */
+const char *intattn_strerror(int code);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* INTATTN_H */

@@ -1,0 +1,188 @@
+"""Fully-integer attention forward (IntAttention, arXiv 2511.21513) on B200.
+
+Python binding of the C ABI in ``include/intattn.h``: argument marshalling
+only.  Every step of the computation runs in the CUDA kernels of
+``libintattn.so``; torch supplies device memory and streams.  There is no CPU
+fallback: if the library is missing, every call raises.
+"""
+from __future__ import annotations
+
+import ctypes
+import dataclasses
+import os
+from typing import Optional, Sequence, Union
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libintattn.so")
+
+OK, ERR_INVALID_ARG, ERR_UNSUPPORTED, ERR_PARAM_RANGE, ERR_CUDA, ERR_WORKSPACE, ERR_TIMEOUT = range(7)
+MAX_HEADS = 128
+
+# every function declared in include/intattn.h
+EXPORTED = ("intattn_derive_params", "intattn_forward", "intattn_decode_workspace_size",
+            "intattn_decode", "intattn_device_error", "intattn_strerror")
+
+
+class IntAttnError(RuntimeError):
+    def __init__(self, code: int, what: str):
+        self.code = code
+        super().__init__(f"{what}: {strerror(code) if _lib is not None else code} (code {code})")
+
+
+class _Scales(ctypes.Structure):
+    _fields_ = [("per_head", ctypes.c_int32),
+                ("s_q", ctypes.POINTER(ctypes.c_float)),
+                ("s_k", ctypes.POINTER(ctypes.c_float)),
+                ("s_v", ctypes.POINTER(ctypes.c_float)),
+                ("s_o", ctypes.POINTER(ctypes.c_float))]
+
+
+class _HeadParams(ctypes.Structure):
+    _fields_ = [("M", ctypes.c_int32), ("s", ctypes.c_int32), ("D", ctypes.c_int32),
+                ("Mo", ctypes.c_int32), ("so", ctypes.c_int32)]
+
+
+FloatArg = Union[float, Sequence[float], np.ndarray]
+
+
+@dataclasses.dataclass
+class Scales:
+    """Quantisation scales (real = scale * code).  per_head: arrays of H."""
+    s_q: FloatArg
+    s_k: FloatArg
+    s_v: FloatArg
+    s_o: FloatArg
+    per_head: bool = False
+
+    def _c(self):
+        arrs = [np.ascontiguousarray(np.atleast_1d(np.asarray(x, dtype=np.float32)))
+                for x in (self.s_q, self.s_k, self.s_v, self.s_o)]
+        fp = ctypes.POINTER(ctypes.c_float)
+        s = _Scales(int(bool(self.per_head)), *[a.ctypes.data_as(fp) for a in arrs])
+        return s, arrs  # keep the arrays alive for the duration of the call
+
+
+_lib = None
+
+
+def lib() -> ctypes.CDLL:
+    """The loaded C library.  Raises if it has not been built."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise ImportError(f"{LIB_PATH} is missing: build it with "
+                              "`python -m integer_only_quantized_b200.build` (nvcc, sm_100a)")
+        L = ctypes.CDLL(LIB_PATH)
+        vp, i32, f32 = ctypes.c_void_p, ctypes.c_int, ctypes.c_float
+        L.intattn_derive_params.argtypes = [ctypes.POINTER(_Scales), i32, i32, f32,
+                                            ctypes.POINTER(ctypes.c_int32), ctypes.POINTER(_HeadParams)]
+        L.intattn_forward.argtypes = [vp, vp, vp, ctypes.POINTER(_Scales), i32, i32, i32, i32, i32,
+                                      i32, f32, vp, vp]
+        L.intattn_decode_workspace_size.argtypes = [i32, i32, i32, i32]
+        L.intattn_decode_workspace_size.restype = ctypes.c_size_t
+        L.intattn_decode.argtypes = [vp, vp, vp, ctypes.POINTER(_Scales), i32, i32, i32, i32, i32,
+                                     f32, vp, vp, ctypes.c_size_t, vp]
+        L.intattn_device_error.argtypes = [vp]
+        L.intattn_strerror.argtypes = [i32]
+        L.intattn_strerror.restype = ctypes.c_char_p
+        _lib = L
+    return _lib
+
+
+def strerror(code: int) -> str:
+    return lib().intattn_strerror(int(code)).decode()
+
+
+def _check(rc: int, what: str):
+    if rc != OK:
+        raise IntAttnError(rc, what)
+
+
+def derive_params(scales: Scales, H: int, d: int, clip_c: float):
+    """(lut[32] int32, [H, 5] int32 of M, s, D, Mo, so) as the kernels use them."""
+    sc, keep = scales._c()
+    lut = np.zeros(32, dtype=np.int32)
+    hp = (_HeadParams * H)()
+    rc = lib().intattn_derive_params(ctypes.byref(sc), int(H), int(d), float(clip_c),
+                                     lut.ctypes.data_as(ctypes.POINTER(ctypes.c_int32)), hp)
+    _check(rc, "intattn_derive_params")
+    del keep
+    return lut, np.array([[p.M, p.s, p.D, p.Mo, p.so] for p in hp], dtype=np.int32)
+
+
+def _stream_handle(stream, device) -> int:
+    import torch
+    if stream is None:
+        stream = torch.cuda.current_stream(device)
+    return int(stream.cuda_stream) if hasattr(stream, "cuda_stream") else int(stream)
+
+
+def _check_tensor(t, name: str):
+    import torch
+    if not isinstance(t, torch.Tensor) or t.dtype != torch.int8 or not t.is_cuda:
+        raise TypeError(f"{name} must be a CUDA int8 tensor")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+
+
+def forward(q, k, v, scales: Scales, causal: bool, clip_c: float, out=None, stream=None):
+    """out[B,H,Lq,d] int8 = IntAttention forward of int8 q[B,H,Lq,d], k/v[B,H,Lk,d]."""
+    import torch
+    for t, n in ((q, "q"), (k, "k"), (v, "v")):
+        _check_tensor(t, n)
+    B, H, Lq, d = q.shape
+    Lk = k.shape[2]
+    if k.shape != (B, H, Lk, d) or v.shape != k.shape:
+        raise ValueError("k and v must be [B, H, Lk, d] matching q")
+    if out is None:
+        out = torch.empty_like(q)
+    _check_tensor(out, "out")
+    if out.shape != q.shape:
+        raise ValueError("out must match q")
+    sc, keep = scales._c()
+    rc = lib().intattn_forward(q.data_ptr(), k.data_ptr(), v.data_ptr(), ctypes.byref(sc), B, H, Lq, Lk,
+                               d, int(bool(causal)), float(clip_c), out.data_ptr(),
+                               _stream_handle(stream, q.device))
+    del keep
+    _check(rc, "intattn_forward")
+    return out
+
+
+def decode_workspace_size(B: int, H: int, Lk: int, d: int) -> int:
+    return int(lib().intattn_decode_workspace_size(int(B), int(H), int(Lk), int(d)))
+
+
+def decode(q, k_cache, v_cache, scales: Scales, Lk: int, clip_c: float, out=None, workspace=None,
+           stream=None):
+    """out[B,H,1,d] int8: one query per (b, h) over the first Lk rows of the caches."""
+    import torch
+    for t, n in ((q, "q"), (k_cache, "k_cache"), (v_cache, "v_cache")):
+        _check_tensor(t, n)
+    B, H, one, d = q.shape
+    if one != 1:
+        raise ValueError("decode takes one query per (b, h): q is [B, H, 1, d]")
+    Lmax = k_cache.shape[2]
+    if k_cache.shape != (B, H, Lmax, d) or v_cache.shape != k_cache.shape:
+        raise ValueError("caches must be [B, H, Lmax, d]")
+    if out is None:
+        out = torch.empty_like(q)
+    _check_tensor(out, "out")
+    need = decode_workspace_size(B, H, Lk, d)
+    if workspace is None:
+        workspace = torch.empty(max(need, 1), dtype=torch.uint8, device=q.device)
+    sc, keep = scales._c()
+    rc = lib().intattn_decode(q.data_ptr(), k_cache.data_ptr(), v_cache.data_ptr(), ctypes.byref(sc), B,
+                              H, int(Lk), Lmax, d, float(clip_c), out.data_ptr(), workspace.data_ptr(),
+                              workspace.numel() * workspace.element_size(),
+                              _stream_handle(stream, q.device))
+    del keep
+    _check(rc, "intattn_decode")
+    return out
+
+
+def device_error(stream=None) -> int:
+    """Synchronise and return/clear the device error word (OK or ERR_TIMEOUT)."""
+    import torch
+    return int(lib().intattn_device_error(_stream_handle(stream, torch.device("cuda"))))

@@ -1,0 +1,300 @@
+// Decode kernels: one query per (batch, head) against an int8 KV cache.
+//
+// Same integer definition as the prefill path with Lq = 1 and no mask.  The
+// work is an HBM stream of the K and V rows (2*Lk*d bytes per (b, h)), so it
+// is split over key chunks to fill every SM, in two launches:
+//   decode_qk  per (b, h, chunk): S_j = q.K_j with 16-byte vector loads and
+//              dp4a; S to the workspace, chunk max to the workspace.
+//   decode_pv  per (b, h, chunk): m = max of the chunk maxima; Z over all Lk
+//              scores of the row (16 KB from L2 per (b, h)); R and the u8
+//              probabilities of this chunk; V chunk streamed with 16-byte
+//              loads, P.V by dp4a after a 4x4 byte transpose; int32 partial
+//              sums to the workspace.  The last CTA of a (b, h) (atomic
+//              ticket) adds the partials and requantises.  Integer addition
+//              is associative, so the result does not depend on the order.
+#pragma once
+#include <climits>
+#include <cstdint>
+
+#include "common.cuh"
+#include "sm100.cuh"
+
+namespace intattn {
+
+struct DecodeArgs {
+  const int8_t* q;   // [BH, d]
+  const int8_t* k;   // [BH, Lmax, d]
+  const int8_t* v;   // [BH, Lmax, d]
+  int8_t* out;       // [BH, d]
+  int32_t* ws_s;     // [BH, Lk]          scores
+  int32_t* ws_max;   // [BH, nsplit]      chunk maxima
+  int32_t* ws_part;  // [BH, nsplit, d]   partial P.V sums
+  uint32_t* ws_cnt;  // [BH]              arrival tickets
+  int32_t BH, H, Lk, Lmax, nsplit, chunk, per_head;
+  uint32_t lut[32];
+  HeadParamsDev hp[INTATTN_MAX_HEADS];
+};
+
+namespace decode {
+
+constexpr int kThreads = 256;
+constexpr int kChunk = 512;  // keys per CTA (multiple of the rows one step covers)
+
+__device__ __forceinline__ uint4 ld_stream(const void* p) {
+  uint4 r;
+  asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0, %1, %2, %3}, [%4];"
+               : "=r"(r.x), "=r"(r.y), "=r"(r.z), "=r"(r.w)
+               : "l"(p));
+  return r;
+}
+
+__device__ __forceinline__ int32_t dp4a_ss(uint32_t a, uint32_t b, int32_t c) {
+  int32_t d;
+  asm("dp4a.s32.s32 %0, %1, %2, %3;" : "=r"(d) : "r"(a), "r"(b), "r"(c));
+  return d;
+}
+// signed bytes of a times unsigned bytes of b
+__device__ __forceinline__ int32_t dp4a_su(uint32_t a, uint32_t b, int32_t c) {
+  int32_t d;
+  asm("dp4a.s32.u32 %0, %1, %2, %3;" : "=r"(d) : "r"(a), "r"(b), "r"(c));
+  return d;
+}
+
+__device__ __forceinline__ int32_t imax32(int32_t a, int32_t b) { return a > b ? a : b; }
+
+// Thread layout shared by both kernels: CPR = D/16 threads cover one row in
+// 16-byte pieces; a thread handles 4 rows (a "quad") per step.
+template <int D>
+struct Layout {
+  static constexpr int kCPR = D / 16;                  // 16-byte pieces per row
+  static constexpr int kGroups = kThreads / kCPR;      // row quads per step
+  static constexpr int kRowsPerStep = 4 * kGroups;     // 128 (d=128) or 256 (d=64)
+  static_assert(kChunk % kRowsPerStep == 0, "chunk must be whole steps");
+};
+
+template <int D>
+__global__ void __launch_bounds__(kThreads) decode_qk_kernel(const __grid_constant__ DecodeArgs a) {
+  using Lt = Layout<D>;
+  const int bh = blockIdx.y;
+  const int sp = blockIdx.x;
+  const int j0 = sp * a.chunk;
+  const int j1 = min(a.Lk, j0 + a.chunk);
+  const int tid = threadIdx.x;
+  const int piece = tid % Lt::kCPR;
+  const int grp = tid / Lt::kCPR;
+  const int lane = tid & 31;
+
+  if (sp == 0 && tid == 0) a.ws_cnt[bh] = 0u;  // ticket for decode_pv
+
+  const uint4 qv = *reinterpret_cast<const uint4*>(a.q + static_cast<size_t>(bh) * D + piece * 16);
+  const int8_t* kbase = a.k + static_cast<size_t>(bh) * a.Lmax * D + piece * 16;
+  int32_t* srow = a.ws_s + static_cast<size_t>(bh) * a.Lk;
+  int32_t mx = INT_MIN;
+
+  for (int base = j0; base < j1; base += Lt::kRowsPerStep) {
+    const int r0 = base + 4 * grp;
+    uint4 kv[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const int j = r0 + i;
+      kv[i] = (j < j1) ? ld_stream(kbase + static_cast<size_t>(j) * D) : make_uint4(0, 0, 0, 0);
+    }
+    int32_t s[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      int32_t acc = 0;
+      acc = dp4a_ss(kv[i].x, qv.x, acc);
+      acc = dp4a_ss(kv[i].y, qv.y, acc);
+      acc = dp4a_ss(kv[i].z, qv.z, acc);
+      acc = dp4a_ss(kv[i].w, qv.w, acc);
+      s[i] = acc;
+    }
+    // reduce the CPR partial sums of each of the 4 rows (transpose-reduce)
+    int32_t t0, t1;
+    if (Lt::kCPR == 8) {
+      const bool hi = lane & 4;
+      const int32_t send0 = hi ? s[0] : s[2], send1 = hi ? s[1] : s[3];
+      const int32_t keep0 = hi ? s[2] : s[0], keep1 = hi ? s[3] : s[1];
+      t0 = keep0 + __shfl_xor_sync(0xffffffffu, send0, 4);
+      t1 = keep1 + __shfl_xor_sync(0xffffffffu, send1, 4);
+    } else {
+      t0 = s[0];  // with CPR = 4 the pair (0,1)/(2,3) split happens below
+      t1 = s[1];
+    }
+    int32_t row_val;
+    int row_idx;
+    if (Lt::kCPR == 8) {
+      const bool b1 = lane & 2;
+      const int32_t send = b1 ? t0 : t1, keep = b1 ? t1 : t0;
+      int32_t u = keep + __shfl_xor_sync(0xffffffffu, send, 2);
+      u += __shfl_xor_sync(0xffffffffu, u, 1);
+      row_val = u;
+      row_idx = ((lane & 4) ? 2 : 0) + ((lane & 2) ? 1 : 0);
+    } else {
+      const bool b1 = lane & 2;
+      const int32_t send0 = b1 ? s[0] : s[2], send1 = b1 ? s[1] : s[3];
+      const int32_t keep0 = b1 ? s[2] : s[0], keep1 = b1 ? s[3] : s[1];
+      const int32_t u0 = keep0 + __shfl_xor_sync(0xffffffffu, send0, 2);
+      const int32_t u1 = keep1 + __shfl_xor_sync(0xffffffffu, send1, 2);
+      const bool b0 = lane & 1;
+      const int32_t send = b0 ? u0 : u1, keep = b0 ? u1 : u0;
+      row_val = keep + __shfl_xor_sync(0xffffffffu, send, 1);
+      row_idx = (b1 ? 2 : 0) + (b0 ? 1 : 0);
+      (void)t0;
+      (void)t1;
+    }
+    const int j = r0 + row_idx;
+    const bool writer = (Lt::kCPR == 8) ? ((lane & 1) == 0) : true;
+    if (writer && j < j1) {
+      srow[j] = row_val;
+      mx = imax32(mx, row_val);
+    }
+  }
+  // chunk max
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) mx = imax32(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+  __shared__ int32_t red[kThreads / 32];
+  if (lane == 0) red[tid >> 5] = mx;
+  __syncthreads();
+  if (tid == 0) {
+    int32_t r = red[0];
+    for (int w = 1; w < kThreads / 32; ++w) r = imax32(r, red[w]);
+    a.ws_max[static_cast<size_t>(bh) * a.nsplit + sp] = r;
+  }
+}
+
+template <int D>
+__global__ void __launch_bounds__(kThreads) decode_pv_kernel(const __grid_constant__ DecodeArgs a) {
+  using Lt = Layout<D>;
+  const int bh = blockIdx.y;
+  const int sp = blockIdx.x;
+  const int j0 = sp * a.chunk;
+  const int j1 = min(a.Lk, j0 + a.chunk);
+  const int tid = threadIdx.x;
+  const int lane = tid & 31;
+  const int h = bh % a.H;
+  const HeadParamsDev hp = a.hp[a.per_head ? h : 0];
+
+  __shared__ uint32_t lut_s[32];
+  __shared__ uint32_t ptab_s[32];
+  __shared__ int32_t red[kThreads / 32];
+  __shared__ uint32_t pk[kChunk / 4];              // u8 probabilities of this chunk
+  __shared__ int32_t part[kThreads * 16];          // per-thread partial sums
+  __shared__ int last_flag;
+
+  if (tid < 32) lut_s[tid] = a.lut[tid];
+
+  // row max from the chunk maxima
+  int32_t m = INT_MIN;
+  for (int i = 0; i < a.nsplit; ++i) m = imax32(m, __ldcg(a.ws_max + static_cast<size_t>(bh) * a.nsplit + i));
+  const long long lo64 = static_cast<long long>(m) - hp.D;
+  const int32_t lo = lo64 < INT_MIN ? INT_MIN : static_cast<int32_t>(lo64);
+  const uint32_t Mu = static_cast<uint32_t>(hp.M);
+  const uint32_t sh = static_cast<uint32_t>(hp.s);
+  const uint32_t Cm = static_cast<uint32_t>(m) * Mu + (1u << (sh - 1));
+  __syncthreads();
+
+  // Z over the whole row
+  const int32_t* srow = a.ws_s + static_cast<size_t>(bh) * a.Lk;
+  int32_t z = 0;
+  for (int j = tid; j < a.Lk; j += kThreads) {
+    const int32_t t = imax32(__ldcg(srow + j), lo);
+    z += static_cast<int32_t>(lut_s[(Cm - static_cast<uint32_t>(t) * Mu) >> sh]);
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) z += __shfl_xor_sync(0xffffffffu, z, o);
+  if (lane == 0) red[tid >> 5] = z;
+  __syncthreads();
+  if (tid < 32) {
+    int32_t Z = 0;
+    for (int w = 0; w < kThreads / 32; ++w) Z += red[w];
+    const unsigned long long R =
+        ((255ull << 32) + static_cast<unsigned long long>(Z >> 1)) / static_cast<unsigned long long>(Z);
+    ptab_s[tid] = static_cast<uint32_t>((static_cast<unsigned long long>(lut_s[tid]) * R + (1ull << 31)) >> 32);
+  }
+  __syncthreads();
+
+  // u8 probabilities of this chunk, 4 per word (rows past j1 get 0)
+  for (int w = tid; w < a.chunk / 4; w += kThreads) {
+    uint32_t word = 0;
+#pragma unroll
+    for (int b = 0; b < 4; ++b) {
+      const int j = j0 + 4 * w + b;
+      if (j < j1) {
+        const int32_t t = imax32(__ldcg(srow + j), lo);
+        word |= ptab_s[(Cm - static_cast<uint32_t>(t) * Mu) >> sh] << (8 * b);
+      }
+    }
+    pk[w] = word;
+  }
+  __syncthreads();
+
+  // stream V: acc[c] over this thread's 16 columns
+  const int piece = tid % Lt::kCPR;
+  const int grp = tid / Lt::kCPR;
+  const int8_t* vbase = a.v + static_cast<size_t>(bh) * a.Lmax * D + piece * 16;
+  int32_t acc[16];
+#pragma unroll
+  for (int c = 0; c < 16; ++c) acc[c] = 0;
+  for (int base = j0; base < j1; base += Lt::kRowsPerStep) {
+    const int r0 = base + 4 * grp;
+    uint4 vv[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const int j = r0 + i;
+      vv[i] = (j < j1) ? ld_stream(vbase + static_cast<size_t>(j) * D) : make_uint4(0, 0, 0, 0);
+    }
+    const uint32_t p4 = pk[(r0 - j0) >> 2];  // P of rows r0..r0+3, one byte each
+    const uint32_t* w0 = reinterpret_cast<const uint32_t*>(&vv[0]);
+    const uint32_t* w1 = reinterpret_cast<const uint32_t*>(&vv[1]);
+    const uint32_t* w2 = reinterpret_cast<const uint32_t*>(&vv[2]);
+    const uint32_t* w3 = reinterpret_cast<const uint32_t*>(&vv[3]);
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      // bytes (row i, column 4q+c) -> word c holds the 4 rows of column 4q+c
+      const uint32_t ab_lo = __byte_perm(w0[q], w1[q], 0x5140);
+      const uint32_t ab_hi = __byte_perm(w0[q], w1[q], 0x7362);
+      const uint32_t cd_lo = __byte_perm(w2[q], w3[q], 0x5140);
+      const uint32_t cd_hi = __byte_perm(w2[q], w3[q], 0x7362);
+      acc[4 * q + 0] = dp4a_su(__byte_perm(ab_lo, cd_lo, 0x5410), p4, acc[4 * q + 0]);
+      acc[4 * q + 1] = dp4a_su(__byte_perm(ab_lo, cd_lo, 0x7632), p4, acc[4 * q + 1]);
+      acc[4 * q + 2] = dp4a_su(__byte_perm(ab_hi, cd_hi, 0x5410), p4, acc[4 * q + 2]);
+      acc[4 * q + 3] = dp4a_su(__byte_perm(ab_hi, cd_hi, 0x7632), p4, acc[4 * q + 3]);
+    }
+  }
+  // reduce over the row groups: column piece*16 + c
+#pragma unroll
+  for (int c = 0; c < 16; ++c) part[tid * 16 + c] = acc[c];
+  __syncthreads();
+  int32_t* gpart = a.ws_part + (static_cast<size_t>(bh) * a.nsplit + sp) * D;
+  if (tid < D) {
+    const int pc = tid / 16, c = tid % 16;
+    int32_t sum = 0;
+    for (int g = 0; g < Lt::kGroups; ++g) sum += part[(g * Lt::kCPR + pc) * 16 + c];
+    gpart[tid] = sum;
+  }
+  // the last CTA of this (b, h) adds the partials and requantises
+  __threadfence();
+  __syncthreads();
+  if (tid == 0) {
+    const unsigned prev = atomicAdd(a.ws_cnt + bh, 1u);
+    last_flag = (prev == static_cast<unsigned>(a.nsplit - 1));
+  }
+  __syncthreads();
+  if (last_flag) {
+    __threadfence();
+    if (tid < D) {
+      int32_t tot = 0;
+      const int32_t* p0 = a.ws_part + static_cast<size_t>(bh) * a.nsplit * D + tid;
+      for (int i = 0; i < a.nsplit; ++i) tot += __ldcg(p0 + static_cast<size_t>(i) * D);
+      const long long t = static_cast<long long>(tot) * hp.Mo + (1ll << (hp.so - 1));
+      long long y = t >> hp.so;
+      y = y > 127 ? 127 : (y < -127 ? -127 : y);
+      a.out[static_cast<size_t>(bh) * D + tid] = static_cast<int8_t>(y);
+    }
+    if (tid == 0) a.ws_cnt[bh] = 0u;
+  }
+}
+
+}  // namespace decode
+}  // namespace intattn

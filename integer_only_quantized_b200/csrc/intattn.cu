@@ -1,0 +1,300 @@
+// C ABI of the fully-integer attention forward (see include/intattn.h).
+//
+// Host side: argument checks, the integer parameters of every head (IEEE
+// double, the order of operations fixed by the definition in intattn.h),
+// TMA descriptors, and launches on the caller's stream.  Device side: the
+// kernels in prefill_kernel.cuh and decode_kernel.cuh, compiled into this
+// single translation unit for sm_100a.
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <cmath>
+#include <cstdint>
+#include <cstring>
+#include <mutex>
+
+#include "intattn.h"
+
+#include "decode_kernel.cuh"
+#include "prefill_kernel.cuh"
+
+using intattn::DecodeArgs;
+using intattn::HeadParamsDev;
+using intattn::PrefillArgs;
+
+namespace {
+
+// ----------------------------------------------------------------- params
+// Index multiplier/shift/clip of one head: M / 2^s approximates
+// alpha * 31 / c with alpha = s_q s_k / sqrt(d); D is the first gap whose
+// rounded index is 31.
+int index_params(double s_q, double s_k, int d, double c, HeadParamsDev* hp) {
+  if (!std::isfinite(s_q) || !std::isfinite(s_k) || !std::isfinite(c)) return INTATTN_ERR_PARAM_RANGE;
+  if (!(s_q > 0.0) || !(s_k > 0.0) || !(c > 0.0)) return INTATTN_ERR_PARAM_RANGE;
+  const double alpha = (s_q * s_k) / std::sqrt(static_cast<double>(d));
+  const double steps_per_unit = (alpha * 31.0) / c;
+  int shift = 26;
+  long long mult = std::llround(std::ldexp(steps_per_unit, shift));
+  while (shift > 1 && mult > (1ll << 24)) {
+    --shift;
+    mult = std::llround(std::ldexp(steps_per_unit, shift));
+  }
+  if (mult < 1 || mult > (1ll << 24) || mult > (1ll << shift)) return INTATTN_ERR_PARAM_RANGE;
+  const long long half_steps = 61ll << (shift - 1);  // 30.5 index steps, in units of 2^-s
+  hp->M = static_cast<int32_t>(mult);
+  hp->s = shift;
+  hp->D = static_cast<int32_t>((half_steps + mult - 1) / mult);
+  return INTATTN_OK;
+}
+
+// Requantisation multiplier/shift: acc * s_v / (255 s_o) ~= acc * Mo / 2^so.
+int requant_params(double s_v, double s_o, HeadParamsDev* hp) {
+  if (!std::isfinite(s_v) || !std::isfinite(s_o) || !(s_v > 0.0) || !(s_o > 0.0))
+    return INTATTN_ERR_PARAM_RANGE;
+  int e = 0;
+  const double f = std::frexp(s_v / (255.0 * s_o), &e);  // f in [0.5, 1)
+  long long mo = std::llround(f * 2147483648.0);
+  if (mo == (1ll << 31)) {
+    mo = 1ll << 30;
+    ++e;
+  }
+  const int so = 31 - e;
+  if (so < 1 || so > 62) return INTATTN_ERR_PARAM_RANGE;
+  hp->Mo = static_cast<int32_t>(mo);
+  hp->so = so;
+  return INTATTN_OK;
+}
+
+int make_lut(double c, uint32_t lut[32]) {
+  if (!std::isfinite(c) || !(c > 0.0)) return INTATTN_ERR_PARAM_RANGE;
+  for (int i = 0; i < 31; ++i)
+    lut[i] = static_cast<uint32_t>(std::llround(32768.0 * std::exp(-(static_cast<double>(i) * c) / 31.0)));
+  lut[31] = 0u;  // a clipped gap contributes nothing
+  return INTATTN_OK;
+}
+
+// LUT and head parameters; per-tensor scales fill hp[0] only.
+int derive(const intattn_scales_t* sc, int H, int d, float clip_c, uint32_t lut[32],
+           HeadParamsDev* hp, int max_heads) {
+  if (!sc || !sc->s_q || !sc->s_k || !sc->s_v || !sc->s_o) return INTATTN_ERR_INVALID_ARG;
+  if (H <= 0) return INTATTN_ERR_INVALID_ARG;
+  const int n = sc->per_head ? H : 1;
+  if (n > max_heads) return INTATTN_ERR_UNSUPPORTED;
+  int rc = make_lut(static_cast<double>(clip_c), lut);
+  if (rc) return rc;
+  for (int i = 0; i < n; ++i) {
+    rc = index_params(sc->s_q[i], sc->s_k[i], d, static_cast<double>(clip_c), &hp[i]);
+    if (rc) return rc;
+    rc = requant_params(sc->s_v[i], sc->s_o[i], &hp[i]);
+    if (rc) return rc;
+  }
+  return INTATTN_OK;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+// ------------------------------------------------------------------- TMA
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                   const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                   CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static std::once_flag once;
+  static EncodeTiledFn fn = nullptr;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  });
+  return fn;
+}
+
+// [planes, rows, d] int8 tensor, box {d, box_rows, 1}, swizzle = d bytes.
+bool encode_3d(CUtensorMap* m, const void* base, int d, long long rows, long long planes, int box_rows) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return false;
+  const cuuint64_t dims[3] = {static_cast<cuuint64_t>(d), static_cast<cuuint64_t>(rows),
+                              static_cast<cuuint64_t>(planes)};
+  const cuuint64_t strides[2] = {static_cast<cuuint64_t>(d), static_cast<cuuint64_t>(rows) * d};
+  const cuuint32_t box[3] = {static_cast<cuuint32_t>(d), static_cast<cuuint32_t>(box_rows), 1u};
+  const cuuint32_t estr[3] = {1u, 1u, 1u};
+  const CUtensorMapSwizzle sw = (d == 128) ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B;
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, const_cast<void*>(base), dims, strides, box, estr,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, sw, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// ------------------------------------------------------- kernel attributes
+template <int D>
+int prefill_launch(const PrefillArgs& args, int grid, cudaStream_t stream) {
+  using C = intattn::prefill::Cfg<D>;
+  static bool attr_set[64] = {};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return INTATTN_ERR_CUDA;
+  if (dev < 0 || dev >= 64) return INTATTN_ERR_CUDA;
+  if (!attr_set[dev]) {
+    if (cudaFuncSetAttribute(intattn::prefill::prefill_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             static_cast<int>(C::kSmemBytes)) != cudaSuccess)
+      return INTATTN_ERR_CUDA;
+    attr_set[dev] = true;
+  }
+  intattn::prefill::prefill_kernel<D><<<grid, intattn::prefill::kThreads, C::kSmemBytes, stream>>>(args);
+  return cudaGetLastError() == cudaSuccess ? INTATTN_OK : INTATTN_ERR_CUDA;
+}
+
+struct DecodeLayout {
+  int nsplit;
+  size_t off_s, off_max, off_part, off_cnt, total;
+};
+
+size_t round256(size_t x) { return (x + 255) & ~size_t(255); }
+
+DecodeLayout decode_layout(long long BH, int Lk, int d) {
+  DecodeLayout L{};
+  L.nsplit = (Lk + intattn::decode::kChunk - 1) / intattn::decode::kChunk;
+  L.off_s = 0;
+  L.off_max = L.off_s + round256(static_cast<size_t>(BH) * Lk * 4);
+  L.off_part = L.off_max + round256(static_cast<size_t>(BH) * L.nsplit * 4);
+  L.off_cnt = L.off_part + round256(static_cast<size_t>(BH) * L.nsplit * d * 4);
+  L.total = L.off_cnt + round256(static_cast<size_t>(BH) * 4);
+  return L;
+}
+
+template <int D>
+int decode_launch(const DecodeArgs& a, cudaStream_t stream) {
+  const dim3 grid(a.nsplit, a.BH);
+  intattn::decode::decode_qk_kernel<D><<<grid, intattn::decode::kThreads, 0, stream>>>(a);
+  if (cudaGetLastError() != cudaSuccess) return INTATTN_ERR_CUDA;
+  intattn::decode::decode_pv_kernel<D><<<grid, intattn::decode::kThreads, 0, stream>>>(a);
+  return cudaGetLastError() == cudaSuccess ? INTATTN_OK : INTATTN_ERR_CUDA;
+}
+
+}  // namespace
+
+extern "C" {
+
+int intattn_derive_params(const intattn_scales_t* scales, int H, int d, float clip_c, int32_t lut[32],
+                          intattn_head_params_t* out) {
+  if (!lut || !out) return INTATTN_ERR_INVALID_ARG;
+  if (d != 64 && d != 128) return INTATTN_ERR_UNSUPPORTED;
+  uint32_t l[32];
+  HeadParamsDev hp[INTATTN_MAX_HEADS];
+  if (scales && !scales->per_head && H > 0) {
+    // per-tensor: every head shares entry 0; any H is accepted
+    const int rc = derive(scales, 1, d, clip_c, l, hp, INTATTN_MAX_HEADS);
+    if (rc) return rc;
+    for (int h = 0; h < H; ++h) out[h] = {hp[0].M, hp[0].s, hp[0].D, hp[0].Mo, hp[0].so};
+  } else {
+    const int rc = derive(scales, H, d, clip_c, l, hp, INTATTN_MAX_HEADS);
+    if (rc) return rc;
+    for (int h = 0; h < H; ++h) out[h] = {hp[h].M, hp[h].s, hp[h].D, hp[h].Mo, hp[h].so};
+  }
+  for (int i = 0; i < 32; ++i) lut[i] = static_cast<int32_t>(l[i]);
+  return INTATTN_OK;
+}
+
+int intattn_forward(const int8_t* q, const int8_t* k, const int8_t* v, const intattn_scales_t* scales, int B,
+                    int H, int Lq, int Lk, int d, int causal, float clip_c, int8_t* out,
+                    intattn_stream_t stream) {
+  if (B < 0 || H <= 0 || Lq < 0 || Lk < 1 || Lk > 65535) return INTATTN_ERR_INVALID_ARG;
+  if (causal && Lq > Lk) return INTATTN_ERR_INVALID_ARG;
+  if (d != 64 && d != 128) return INTATTN_ERR_UNSUPPORTED;
+  if (!scales) return INTATTN_ERR_INVALID_ARG;
+  static_assert(sizeof(PrefillArgs) <= 4096, "kernel argument block too large");
+  PrefillArgs args;
+  std::memset(&args, 0, sizeof(args));
+  int rc = derive(scales, H, d, clip_c, args.lut, args.hp, INTATTN_MAX_HEADS);
+  if (rc) return rc;
+  const long long BH = static_cast<long long>(B) * H;
+  if (BH == 0 || Lq == 0) return INTATTN_OK;
+  if (!q || !k || !v || !out) return INTATTN_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out)) return INTATTN_ERR_UNSUPPORTED;
+  const int n_qtiles = (Lq + intattn::prefill::kBM - 1) / intattn::prefill::kBM;
+  if (BH * n_qtiles > 0x7fffffffll || BH > 0x7fffffffll) return INTATTN_ERR_UNSUPPORTED;
+  if (!encode_3d(&args.tm_q, q, d, Lq, BH, intattn::prefill::kBM) ||
+      !encode_3d(&args.tm_k, k, d, Lk, BH, intattn::prefill::kBN) ||
+      !encode_3d(&args.tm_v, v, d, Lk, BH, intattn::prefill::kBN))
+    return INTATTN_ERR_CUDA;
+  args.out = out;
+  args.BH = static_cast<int32_t>(BH);
+  args.H = H;
+  args.Lq = Lq;
+  args.Lk = Lk;
+  args.causal = causal ? 1 : 0;
+  args.n_qtiles = n_qtiles;
+  args.per_head = scales->per_head ? 1 : 0;
+  const int grid = static_cast<int>(BH * n_qtiles);
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  return d == 64 ? prefill_launch<64>(args, grid, st) : prefill_launch<128>(args, grid, st);
+}
+
+size_t intattn_decode_workspace_size(int B, int H, int Lk, int d) {
+  if (B < 0 || H <= 0 || Lk < 1 || (d != 64 && d != 128)) return 0;
+  return decode_layout(static_cast<long long>(B) * H, Lk, d).total;
+}
+
+int intattn_decode(const int8_t* q, const int8_t* k_cache, const int8_t* v_cache, const intattn_scales_t* scales,
+                   int B, int H, int Lk, int Lmax, int d, float clip_c, int8_t* out, void* workspace,
+                   size_t workspace_bytes, intattn_stream_t stream) {
+  if (B < 0 || H <= 0 || Lk < 1 || Lk > 65535 || Lmax < Lk) return INTATTN_ERR_INVALID_ARG;
+  if (d != 64 && d != 128) return INTATTN_ERR_UNSUPPORTED;
+  if (!scales) return INTATTN_ERR_INVALID_ARG;
+  static_assert(sizeof(DecodeArgs) <= 4096, "kernel argument block too large");
+  DecodeArgs a;
+  std::memset(&a, 0, sizeof(a));
+  int rc = derive(scales, H, d, clip_c, a.lut, a.hp, INTATTN_MAX_HEADS);
+  if (rc) return rc;
+  const long long BH = static_cast<long long>(B) * H;
+  if (BH == 0) return INTATTN_OK;
+  if (BH > 65535) return INTATTN_ERR_UNSUPPORTED;  // grid y limit
+  if (!q || !k_cache || !v_cache || !out) return INTATTN_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k_cache) || !aligned16(v_cache)) return INTATTN_ERR_UNSUPPORTED;
+  const DecodeLayout L = decode_layout(BH, Lk, d);
+  if (!workspace || workspace_bytes < L.total || (reinterpret_cast<uintptr_t>(workspace) & 255u))
+    return INTATTN_ERR_WORKSPACE;
+  char* ws = static_cast<char*>(workspace);
+  a.q = q;
+  a.k = k_cache;
+  a.v = v_cache;
+  a.out = out;
+  a.ws_s = reinterpret_cast<int32_t*>(ws + L.off_s);
+  a.ws_max = reinterpret_cast<int32_t*>(ws + L.off_max);
+  a.ws_part = reinterpret_cast<int32_t*>(ws + L.off_part);
+  a.ws_cnt = reinterpret_cast<uint32_t*>(ws + L.off_cnt);
+  a.BH = static_cast<int32_t>(BH);
+  a.H = H;
+  a.Lk = Lk;
+  a.Lmax = Lmax;
+  a.nsplit = L.nsplit;
+  a.chunk = intattn::decode::kChunk;
+  a.per_head = scales->per_head ? 1 : 0;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  return d == 64 ? decode_launch<64>(a, st) : decode_launch<128>(a, st);
+}
+
+int intattn_device_error(intattn_stream_t stream) {
+  if (cudaStreamSynchronize(reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess) return INTATTN_ERR_CUDA;
+  unsigned int v = 0;
+  if (cudaMemcpyFromSymbol(&v, intattn::g_device_error, sizeof(v)) != cudaSuccess) return INTATTN_ERR_CUDA;
+  if (v == 0) return INTATTN_OK;
+  const unsigned int zero = 0;
+  if (cudaMemcpyToSymbol(intattn::g_device_error, &zero, sizeof(zero)) != cudaSuccess) return INTATTN_ERR_CUDA;
+  return INTATTN_ERR_TIMEOUT;
+}
+
+const char* intattn_strerror(int code) {
+  switch (code) {
+    case INTATTN_OK: return "ok";
+    case INTATTN_ERR_INVALID_ARG: return "invalid argument";
+    case INTATTN_ERR_UNSUPPORTED: return "unsupported shape, alignment or head count";
+    case INTATTN_ERR_PARAM_RANGE: return "scale or clip out of range";
+    case INTATTN_ERR_CUDA: return "CUDA launch or driver call failed";
+    case INTATTN_ERR_WORKSPACE: return "decode workspace missing, misaligned or too small";
+    case INTATTN_ERR_TIMEOUT: return "a kernel wait timed out";
+    default: return "unknown error";
+  }
+}
+
+}  // extern "C"

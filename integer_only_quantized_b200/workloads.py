@@ -204,3 +204,73 @@ def make_inputs(w: Workload, nthreads: int = 8) -> Inputs:
     v, s_v = _quantise(w, "v", Lkv, nthreads)
     s_o = _output_scale(w, q, k, v, s_q, s_k, s_v)
     return Inputs(w, q, k, v, s_q, s_k, s_v, s_o)
+
+
+@dataclasses.dataclass
+class DeviceInputs:
+    w: Workload
+    q: "object"            # torch int8 tensors on the device
+    k: "object"
+    v: "object"
+    s_q: np.ndarray
+    s_k: np.ndarray
+    s_v: np.ndarray
+    s_o: np.ndarray
+
+
+def make_inputs_torch(w: Workload, device) -> DeviceInputs:
+    """Same recipe drawn with torch's generator on the device (for benchmark
+    inputs too large to draw quickly with numpy; a different random stream
+    from make_inputs, and never compared with the oracle)."""
+    import torch
+
+    g = torch.Generator(device=device)
+    g.manual_seed(w.seed)
+    Lkv = w.Lmax if w.decode else w.Lk
+
+    def one(which, L):
+        x = torch.randn((w.B, w.H, L, w.d), generator=g, device=device, dtype=torch.float32)
+        if w.dist == "student_t4":
+            chi = torch.randn((4, w.B, w.H, L, w.d), generator=g, device=device).pow(2).sum(0)
+            x = x / torch.sqrt(chi / 4.0)
+        if which in w.outlier_tensors and w.outlier_frac > 0:
+            n = int(round(w.outlier_frac * w.H * w.d))
+            flat = torch.randperm(w.H * w.d, generator=g, device=device)[:n]
+            for f in flat.tolist():
+                x[:, f // w.d, :, f % w.d] *= w.outlier_scale
+        amax = x.abs().amax(dim=(0, 2, 3)).double()
+        if not w.per_head:
+            amax = amax.max().reshape(1)
+        scale = (amax / 127.0).float()
+        scale[scale == 0] = 1.0
+        sh = scale.double() if w.per_head else scale.double().expand(w.H)
+        q = torch.clamp(torch.round(x.double() / sh.view(1, -1, 1, 1)), -127, 127).to(torch.int8)
+        return q, scale.cpu().numpy().astype(np.float32)
+
+    q, s_q = one("q", w.Lq)
+    k, s_k = one("k", Lkv)
+    v, s_v = one("v", Lkv)
+    # output scale from an fp64 row sample, as in make_inputs
+    rows = torch.as_tensor(_sample_rows(w.Lq), device=device)
+    sq = torch.as_tensor(np.broadcast_to(s_q, (w.H,)) if w.per_head else np.full(w.H, s_q[0]),
+                         device=device, dtype=torch.float64)
+    sk = torch.as_tensor(np.broadcast_to(s_k, (w.H,)) if w.per_head else np.full(w.H, s_k[0]),
+                         device=device, dtype=torch.float64)
+    sv = torch.as_tensor(np.broadcast_to(s_v, (w.H,)) if w.per_head else np.full(w.H, s_v[0]),
+                         device=device, dtype=torch.float64)
+    amax = torch.zeros(w.H, dtype=torch.float64, device=device)
+    for b in range(w.B):
+        qf = q[b][:, rows].double() * sq.view(-1, 1, 1)
+        kf = k[b][:, :w.Lk].double() * sk.view(-1, 1, 1)
+        vf = v[b][:, :w.Lk].double() * sv.view(-1, 1, 1)
+        logits = torch.einsum("hid,hjd->hij", qf, kf) / math.sqrt(w.d)
+        if w.causal:
+            mask = torch.arange(w.Lk, device=device)[None, :] > (rows[:, None] + (w.Lk - w.Lq))
+            logits = logits.masked_fill(mask[None], float("-inf"))
+        o = torch.einsum("hij,hjd->hid", torch.softmax(logits, dim=-1), vf)
+        amax = torch.maximum(amax, o.abs().amax(dim=(1, 2)))
+    if not w.per_head:
+        amax = amax.max().reshape(1)
+    s_o = (amax / 127.0).float().cpu().numpy().astype(np.float32)
+    s_o[s_o == 0] = np.float32(1.0)
+    return DeviceInputs(w, q.contiguous(), k.contiguous(), v.contiguous(), s_q, s_k, s_v, s_o)

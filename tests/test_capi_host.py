@@ -1,0 +1,155 @@
+"""Host-side checks of the C ABI (no GPU): the library loads, exports every
+function declared in include/intattn.h, derives exactly the oracle's
+parameters, and rejects bad arguments before touching the device."""
+import ctypes
+import os
+import re
+
+import numpy as np
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def ia():
+    from integer_only_quantized_b200 import build
+    build.build()
+    import integer_only_quantized_b200 as mod
+    mod.lib()
+    return mod
+
+
+def _declared_functions():
+    src = open(os.path.join(ROOT, "include", "intattn.h")).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"\b(intattn_[a-z_]+)\s*\(", src)))
+
+
+def test_library_exports_every_declared_function(ia):
+    declared = _declared_functions()
+    assert declared == sorted(ia.EXPORTED)
+    L = ia.lib()
+    for name in declared:
+        assert hasattr(L, name), name
+    # and the symbols are real dynamic exports of the shared object
+    import subprocess
+    out = subprocess.run(["nm", "-D", "--defined-only", ia.LIB_PATH], capture_output=True,
+                         text=True, check=True).stdout
+    for name in declared:
+        assert re.search(rf"\bT {name}$", out, re.M), name
+
+
+@pytest.mark.parametrize("seed", range(6))
+def test_derived_params_equal_oracle(ia, oracle_mod, seed):
+    rng = np.random.default_rng(seed)
+    H = int(rng.integers(1, 40))
+    d = int(rng.choice([64, 128]))
+    per_head = bool(seed % 2)
+    n = H if per_head else 1
+    s_q = (10 ** rng.uniform(-3, -0.3, n)).astype(np.float32)
+    s_k = (10 ** rng.uniform(-3, -0.3, n)).astype(np.float32)
+    s_v = (10 ** rng.uniform(-3, 0, n)).astype(np.float32)
+    s_o = (10 ** rng.uniform(-4, -1, n)).astype(np.float32)
+    c = float(np.float32(rng.uniform(2, 14)))
+    lut, hp = ia.derive_params(ia.Scales(s_q, s_k, s_v, s_o, per_head), H, d, c)
+    olut, ohp = oracle_mod.params(per_head, s_q, s_k, s_v, s_o, H, d, c)
+    assert np.array_equal(lut, olut)
+    assert np.array_equal(hp, ohp)
+
+
+def test_derive_params_for_the_workloads(ia, oracle_mod):
+    from integer_only_quantized_b200 import workloads as wl
+    for w in wl.WORKLOADS.values():
+        if w.B * w.H * w.Lk * w.d > 2 ** 22:
+            continue  # large inputs are covered on the GPU
+        x = wl.make_inputs(w)
+        sc = ia.Scales(x.s_q, x.s_k, x.s_v, x.s_o, w.per_head)
+        lut, hp = ia.derive_params(sc, w.H, w.d, w.clip_c)
+        olut, ohp = oracle_mod.params(w.per_head, x.s_q, x.s_k, x.s_v, x.s_o, w.H, w.d, w.clip_c)
+        assert np.array_equal(lut, olut) and np.array_equal(hp, ohp), w.name
+
+
+def _fwd(ia, q=1, k=1, v=1, scales=None, B=1, H=2, Lq=4, Lk=4, d=64, causal=0, c=8.0, out=1):
+    sc = scales or ia.Scales(0.1, 0.1, 0.1, 0.1)
+    s, keep = sc._c()
+    ptr = lambda x: None if x is None else 16 * x  # aligned fake pointers, never dereferenced
+    return ia.lib().intattn_forward(ptr(q), ptr(k), ptr(v), ctypes.byref(s), B, H, Lq, Lk, d, causal,
+                                    c, ptr(out), None)
+
+
+def test_forward_argument_errors_need_no_device(ia):
+    assert _fwd(ia, d=96) == ia.ERR_UNSUPPORTED
+    assert _fwd(ia, Lk=0) == ia.ERR_INVALID_ARG
+    assert _fwd(ia, Lk=65536) == ia.ERR_INVALID_ARG
+    assert _fwd(ia, causal=1, Lq=5, Lk=4) == ia.ERR_INVALID_ARG
+    assert _fwd(ia, B=-1) == ia.ERR_INVALID_ARG
+    assert _fwd(ia, H=0) == ia.ERR_INVALID_ARG
+    assert _fwd(ia, c=0.0) == ia.ERR_PARAM_RANGE
+    assert _fwd(ia, c=float("inf")) == ia.ERR_PARAM_RANGE
+    assert _fwd(ia, scales=ia.Scales(0.0, 0.1, 0.1, 0.1)) == ia.ERR_PARAM_RANGE
+    assert _fwd(ia, scales=ia.Scales(0.1, 0.1, float("nan"), 0.1)) == ia.ERR_PARAM_RANGE
+    assert _fwd(ia, scales=ia.Scales(40.0, 40.0, 0.1, 0.1)) == ia.ERR_PARAM_RANGE
+    assert _fwd(ia, q=None) == ia.ERR_INVALID_ARG
+    assert _fwd(ia, out=None) == ia.ERR_INVALID_ARG
+    too_many = ia.Scales([0.1] * 129, [0.1] * 129, [0.1] * 129, [0.1] * 129, per_head=True)
+    assert _fwd(ia, H=129, scales=too_many) == ia.ERR_UNSUPPORTED
+    # nothing to do: success without a launch, even with null tensors
+    assert _fwd(ia, B=0, q=None, k=None, v=None, out=None) == ia.OK
+    assert _fwd(ia, Lq=0, q=None, out=None) == ia.OK
+    # a scale-less call
+    L = ia.lib()
+    assert L.intattn_forward(16, 16, 16, None, 1, 1, 4, 4, 64, 0, 8.0, 16, None) == ia.ERR_INVALID_ARG
+
+
+def test_misaligned_pointer_is_rejected(ia):
+    sc = ia.Scales(0.1, 0.1, 0.1, 0.1)
+    s, keep = sc._c()
+    L = ia.lib()
+    assert L.intattn_forward(16 * 5 + 8, 16, 16, ctypes.byref(s), 1, 1, 4, 4, 64, 0, 8.0, 16,
+                             None) == ia.ERR_UNSUPPORTED
+
+
+def test_decode_argument_errors_need_no_device(ia):
+    sc = ia.Scales(0.1, 0.1, 0.1, 0.1)
+    s, keep = sc._c()
+    L = ia.lib()
+    ws = ia.decode_workspace_size(2, 3, 700, 128)
+    assert ws > 2 * 3 * 700 * 4
+    assert ia.decode_workspace_size(2, 3, 0, 128) == 0
+    assert ia.decode_workspace_size(2, 3, 700, 96) == 0
+    args = lambda **kw: dict(dict(q=16, k=16, v=16, B=2, H=3, Lk=700, Lmax=768, d=128, c=8.0, out=16,
+                                  ws=256, wsb=ws), **kw)
+
+    def call(**kw):
+        a = args(**kw)
+        return L.intattn_decode(a["q"], a["k"], a["v"], ctypes.byref(s), a["B"], a["H"], a["Lk"],
+                                a["Lmax"], a["d"], a["c"], a["out"], a["ws"], a["wsb"], None)
+    assert call(Lmax=600) == ia.ERR_INVALID_ARG
+    assert call(d=32) == ia.ERR_UNSUPPORTED
+    assert call(wsb=ws - 1) == ia.ERR_WORKSPACE
+    assert call(ws=None) == ia.ERR_WORKSPACE
+    assert call(ws=256 + 16) == ia.ERR_WORKSPACE
+    assert call(k=None) == ia.ERR_INVALID_ARG
+    assert call(B=0, q=None) == ia.OK
+
+
+def test_strerror(ia):
+    for code in range(7):
+        assert ia.strerror(code)
+    assert "unknown" in ia.strerror(99)
+
+
+def test_binding_rejects_cpu_tensors(ia):
+    import torch
+    x = torch.zeros(1, 1, 4, 64, dtype=torch.int8)
+    with pytest.raises(TypeError):
+        ia.forward(x, x, x, ia.Scales(0.1, 0.1, 0.1, 0.1), False, 8.0)
+
+
+def test_binding_fails_loudly_without_library(tmp_path, monkeypatch, ia):
+    import integer_only_quantized_b200 as mod
+    monkeypatch.setattr(mod, "_lib", None)
+    monkeypatch.setattr(mod, "LIB_PATH", str(tmp_path / "missing.so"))
+    with pytest.raises(ImportError):
+        mod.lib()

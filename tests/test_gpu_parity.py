@@ -1,0 +1,202 @@
+"""GPU parity: the sm_100a kernels, called through the C ABI, against the CPU
+oracle on the same seeded inputs.  int8 outputs must be identical byte for
+byte (the whole path is integer arithmetic)."""
+import numpy as np
+import pytest
+
+from integer_only_quantized_b200 import workloads as wl
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def ia():
+    import torch
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    from integer_only_quantized_b200 import build
+    build.build()
+    import integer_only_quantized_b200 as mod
+    mod.lib()
+    return mod
+
+
+def _dev(x):
+    import torch
+    return torch.from_numpy(np.ascontiguousarray(x)).cuda()
+
+
+def _gpu_forward(ia, x, w, guard=0):
+    """Run the C-ABI forward; with guard > 0 the output sits between canary bands."""
+    import torch
+    sc = ia.Scales(x.s_q, x.s_k, x.s_v, x.s_o, per_head=w.per_head)
+    q, k, v = _dev(x.q), _dev(x.k), _dev(x.v)
+    n = x.q.size
+    buf = torch.full((n + 2 * guard,), 0x5A, dtype=torch.int8, device="cuda")
+    out = buf[guard:guard + n].view(x.q.shape)
+    ia.forward(q, k, v, sc, w.causal, w.clip_c, out=out)
+    assert ia.device_error() == ia.OK
+    if guard:
+        b = buf.cpu().numpy()
+        assert np.all(b[:guard] == 0x5A) and np.all(b[guard + n:] == 0x5A), "write outside out"
+    return out.cpu().numpy()
+
+
+def _oracle_forward(oracle_mod, x, w):
+    return oracle_mod.forward(x.q, x.k, x.v, w.per_head, x.s_q, x.s_k, x.s_v, x.s_o, w.causal, w.clip_c)
+
+
+def _assert_equal(got, want, what):
+    if not np.array_equal(got, want):
+        bad = np.argwhere(got != want)
+        raise AssertionError(f"{what}: {len(bad)} of {got.size} bytes differ; first at {bad[:5].tolist()} "
+                             f"got {got[tuple(bad[0])]} want {want[tuple(bad[0])]}")
+
+
+# ----------------------------------------------------- benchmark workloads
+
+@pytest.mark.parametrize("name", ["bert_base_l128", "bert_base_b8_l512", "vit_b16_l197"])
+def test_workload_full_parity(ia, oracle_mod, name):
+    w = wl.WORKLOADS[name]
+    x = wl.make_inputs(w)
+    got = _gpu_forward(ia, x, w, guard=4096)
+    _assert_equal(got, _oracle_forward(oracle_mod, x, w), name)
+
+
+def _sample_rows(w, rng, n_random=256):
+    rows = set()
+    Lq = w.Lq
+    special = sorted({i for i in (0, 1, 126, 127, 128, 129, 255, 256, Lq // 2, Lq - 129, Lq - 128,
+                                  Lq - 2, Lq - 1) if 0 <= i < Lq})
+    for b in {0, w.B - 1}:
+        for h in {0, w.H - 1}:
+            for i in special:
+                rows.add((b, h, i))
+    for _ in range(n_random):
+        rows.add((int(rng.integers(w.B)), int(rng.integers(w.H)), int(rng.integers(Lq))))
+    return np.array(sorted(rows), dtype=np.int32)
+
+
+@pytest.mark.parametrize("name", ["gpt2_small_causal_l2048", "llama7b_causal_l8192"])
+def test_workload_sampled_parity(ia, oracle_mod, name):
+    """Full-size causal workloads, launched exactly as the benchmark does;
+    the oracle recomputes a sample of rows one by one."""
+    w = wl.WORKLOADS[name]
+    x = wl.make_inputs(w)
+    got = _gpu_forward(ia, x, w, guard=4096)
+    rows = _sample_rows(w, np.random.default_rng(w.seed))
+    want = oracle_mod.forward_rows(x.q, x.k, x.v, w.per_head, x.s_q, x.s_k, x.s_v, x.s_o, w.causal,
+                                   w.clip_c, rows)
+    _assert_equal(got[rows[:, 0], rows[:, 1], rows[:, 2]], want, name)
+    # a property that holds at any size: the same call twice gives the same bytes
+    again = _gpu_forward(ia, x, w)
+    _assert_equal(again, got, name + " (determinism)")
+
+
+def test_decode_workload_full_parity(ia, oracle_mod):
+    w = wl.WORKLOADS["llama7b_decode_b64_lk4096"]
+    x = wl.make_inputs(w)
+    sc = ia.Scales(x.s_q, x.s_k, x.s_v, x.s_o, per_head=w.per_head)
+    out = ia.decode(_dev(x.q), _dev(x.k), _dev(x.v), sc, w.Lk, w.clip_c)
+    assert ia.device_error() == ia.OK
+    want = oracle_mod.decode(x.q, x.k, x.v, w.per_head, x.s_q, x.s_k, x.s_v, x.s_o, w.Lk, w.clip_c)
+    _assert_equal(out.cpu().numpy(), want, w.name)
+
+
+# ----------------------------------------------------------- shape sweep
+
+SWEEP = [
+    # (B, H, Lq, Lk, d, causal, per_head, dist)
+    (1, 1, 1, 1, 64, False, False, "normal"),
+    (1, 2, 1, 1, 128, True, True, "normal"),
+    (2, 3, 31, 31, 64, True, False, "normal"),
+    (1, 2, 127, 127, 128, False, True, "student_t4"),
+    (1, 2, 128, 128, 64, True, False, "normal"),
+    (1, 2, 129, 129, 128, True, True, "normal"),
+    (2, 2, 197, 197, 64, False, True, "student_t4"),
+    (1, 3, 255, 255, 128, False, False, "normal"),
+    (1, 2, 256, 256, 64, True, True, "normal"),
+    (1, 2, 511, 511, 64, False, False, "normal"),
+    (1, 2, 513, 513, 128, True, False, "normal"),
+    (1, 1, 1000, 1000, 128, True, True, "normal"),
+    (1, 2, 64, 300, 64, True, False, "normal"),     # Lq < Lk, bottom-right causal
+    (1, 2, 130, 700, 128, False, True, "normal"),   # cross attention, ragged
+    (1, 2, 1, 777, 64, True, False, "normal"),      # one query row sees every key
+    (3, 1, 200, 200, 128, False, False, "student_t4"),
+]
+
+
+@pytest.mark.parametrize("case", SWEEP, ids=lambda c: "B{}H{}Lq{}Lk{}d{}{}{}".format(
+    c[0], c[1], c[2], c[3], c[4], "c" if c[5] else "", "h" if c[6] else ""))
+def test_shape_sweep(ia, oracle_mod, case):
+    B, H, Lq, Lk, d, causal, per_head, dist = case
+    w = wl.custom_workload("sweep", B, H, Lq, Lk, d, causal, per_head=per_head, dist=dist,
+                           clip_c=8.0 if d == 64 else 10.0, index=300 + Lq + Lk + d)
+    x = wl.make_inputs(w)
+    got = _gpu_forward(ia, x, w, guard=1024)
+    _assert_equal(got, _oracle_forward(oracle_mod, x, w), str(case))
+
+
+@pytest.mark.parametrize("d", [64, 128])
+def test_extreme_codes(ia, oracle_mod, d):
+    """-128 codes everywhere (largest |S| = 128^2 d), and rows of equal scores."""
+    import dataclasses
+    w = wl.custom_workload("extreme", 1, 2, 200, 200, d, True, index=700 + d)
+    x = wl.make_inputs(w)
+    x = dataclasses.replace(x, q=np.full_like(x.q, -128), k=np.full_like(x.k, -128))
+    _assert_equal(_gpu_forward(ia, x, w), _oracle_forward(oracle_mod, x, w), "all -128")
+    rng = np.random.default_rng(d)
+    k = np.where(rng.random(x.k.shape) < 0.5, -128, 127).astype(np.int8)
+    v = np.where(rng.random(x.v.shape) < 0.5, -128, 127).astype(np.int8)
+    x2 = dataclasses.replace(x, q=np.full_like(x.q, 127), k=k, v=v)
+    _assert_equal(_gpu_forward(ia, x2, w), _oracle_forward(oracle_mod, x2, w), "+-extremes")
+    x3 = dataclasses.replace(x, q=np.zeros_like(x.q))  # every score 0: uniform rows
+    _assert_equal(_gpu_forward(ia, x3, w), _oracle_forward(oracle_mod, x3, w), "uniform rows")
+
+
+@pytest.mark.parametrize("clip_c", [0.5, 3.0, 30.0])
+def test_clip_extremes(ia, oracle_mod, clip_c):
+    """Tiny clip (most keys clipped to index 31) and huge clip (none)."""
+    w = wl.custom_workload("clip", 2, 2, 300, 300, 64, False, clip_c=clip_c, index=800)
+    x = wl.make_inputs(w)
+    _assert_equal(_gpu_forward(ia, x, w), _oracle_forward(oracle_mod, x, w), f"c={clip_c}")
+
+
+# ---------------------------------------------------------------- decode
+
+DECODE_SWEEP = [
+    (1, 1, 1, 1, 64), (2, 3, 100, 160, 128), (1, 2, 511, 511, 64), (1, 2, 512, 512, 128),
+    (2, 2, 513, 600, 64), (3, 2, 1500, 2048, 128), (1, 4, 4096, 4100, 64), (2, 1, 9000, 9000, 128),
+]
+
+
+@pytest.mark.parametrize("case", DECODE_SWEEP, ids=lambda c: "B{}H{}Lk{}Lmax{}d{}".format(*c))
+def test_decode_sweep(ia, oracle_mod, case):
+    import torch
+    B, H, Lk, Lmax, d = case
+    w = wl.custom_workload("dec", B, H, 1, Lk, d, False, per_head=True, clip_c=10.0,
+                           index=500 + Lk + d, decode=True, Lmax=Lmax)
+    x = wl.make_inputs(w)
+    sc = ia.Scales(x.s_q, x.s_k, x.s_v, x.s_o, per_head=True)
+    # a workspace full of garbage: the kernels must not depend on its contents
+    ws = torch.randint(0, 255, (ia.decode_workspace_size(B, H, Lk, d),), dtype=torch.uint8, device="cuda")
+    out = ia.decode(_dev(x.q), _dev(x.k), _dev(x.v), sc, Lk, w.clip_c, workspace=ws)
+    assert ia.device_error() == ia.OK
+    want = oracle_mod.decode(x.q, x.k, x.v, True, x.s_q, x.s_k, x.s_v, x.s_o, Lk, w.clip_c)
+    _assert_equal(out.cpu().numpy(), want, str(case))
+    # second call on the same workspace
+    out2 = ia.decode(_dev(x.q), _dev(x.k), _dev(x.v), sc, Lk, w.clip_c, workspace=ws)
+    _assert_equal(out2.cpu().numpy(), want, str(case) + " (reused workspace)")
+
+
+def test_decode_matches_prefill_last_row(ia):
+    """Decode of query row i over the first Lk cache rows == row i of the
+    causal prefill (same definition, independent kernels)."""
+    w = wl.custom_workload("dec_vs_prefill", 2, 3, 700, 700, 128, True, per_head=True, clip_c=10.0,
+                           index=950)
+    x = wl.make_inputs(w)
+    pre = _gpu_forward(ia, x, w)
+    sc = ia.Scales(x.s_q, x.s_k, x.s_v, x.s_o, per_head=True)
+    for i in (0, 350, 699):
+        out = ia.decode(_dev(x.q[:, :, i:i + 1]), _dev(x.k), _dev(x.v), sc, i + 1, w.clip_c)
+        _assert_equal(out.cpu().numpy()[:, :, 0], pre[:, :, i], f"row {i}")
