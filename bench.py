@@ -119,56 +119,68 @@ def kernel_traffic(kernel: str, workload: str):
 
 # ----------------------------------------------------------------- clocks
 class ClockSampler:
-    """nvidia-smi clocks and throttle reasons sampled every 200 ms."""
+    """SM clock, power and throttle reasons of one GPU, polled through NVML
+    from a background thread every millisecond while the timed region runs
+    (nvidia-smi's 200 ms period would miss a region of a few milliseconds)."""
 
-    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
-              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
-              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    REASONS = {"hw_slowdown": 0x8, "hw_thermal_slowdown": 0x40, "sw_thermal_slowdown": 0x20,
+               "sw_power_cap": 0x4}
 
     def __init__(self, gpu_index: int):
         self.gpu = gpu_index
-        self.proc = None
-        self.path = None
+        self.samples = []
+        self._stop = None
+        self._thread = None
+
+    def _handle(self, pynvml):
+        """NVML handle of the CUDA device (matched by PCI bus id, since NVML
+        indices ignore CUDA_VISIBLE_DEVICES)."""
+        try:
+            import torch
+            p = torch.cuda.get_device_properties(self.gpu)
+            bus = f"{p.pci_domain_id:08x}:{p.pci_bus_id:02x}:{p.pci_device_id:02x}.0"
+            return pynvml.nvmlDeviceGetHandleByPciBusId(bus)
+        except Exception:  # noqa: BLE001
+            return pynvml.nvmlDeviceGetHandleByIndex(self.gpu)
 
     def start(self):
+        import threading
         try:
-            fd, self.path = tempfile.mkstemp(suffix=".csv")
-            os.close(fd)
-            self.proc = subprocess.Popen(
-                ["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.FIELDS}",
-                 "--format=csv,noheader,nounits", "-lms", "200", "-f", self.path],
-                stdout=subprocess.DEVNULL, stderr=subprocess.DEVNULL)
-        except (OSError, FileNotFoundError):
-            self.proc = None
+            import pynvml
+            pynvml.nvmlInit()
+            handle = self._handle(pynvml)
+            self.sm_max = pynvml.nvmlDeviceGetMaxClockInfo(handle, pynvml.NVML_CLOCK_SM)
+        except Exception:  # noqa: BLE001 - no NVML: report no clocks
+            return
+        self._stop = threading.Event()
+
+        def poll():
+            while not self._stop.is_set():
+                try:
+                    sm = pynvml.nvmlDeviceGetClockInfo(handle, pynvml.NVML_CLOCK_SM)
+                    pw = pynvml.nvmlDeviceGetPowerUsage(handle) / 1000.0
+                    rs = pynvml.nvmlDeviceGetCurrentClocksEventReasons(handle)
+                    self.samples.append((sm, pw, rs))
+                except Exception:  # noqa: BLE001
+                    pass
+                time.sleep(0.001)
+
+        self._thread = threading.Thread(target=poll, daemon=True)
+        self._thread.start()
 
     def stop(self):
-        if self.proc is None:
+        if self._thread is None:
             return None
-        time.sleep(0.25)
-        self.proc.terminate()
-        try:
-            self.proc.wait(timeout=5)
-        except subprocess.TimeoutExpired:
-            self.proc.kill()
-        rows = []
-        with open(self.path) as f:
-            for line in f:
-                parts = [p.strip() for p in line.split(",")]
-                if len(parts) >= 9:
-                    rows.append(parts)
-        os.unlink(self.path)
-        if not rows:
+        self._stop.set()
+        self._thread.join(timeout=5)
+        if not self.samples:
             return None
-        sm = [float(r[1]) for r in rows if r[1].replace(".", "").isdigit()]
-        smax = [float(r[2]) for r in rows if r[2].replace(".", "").isdigit()]
-        pw = [float(r[3]) for r in rows if r[3].replace(".", "").isdigit()]
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        reasons = sorted({n for r in rows for n, v in zip(names, r[5:9]) if v.strip().lower() == "active"})
-        loaded = [s for s, p in zip(sm, pw) if p >= 0.5 * max(pw)] if pw else sm
-        return {"sm_mhz": statistics.median(loaded or sm) if sm else None,
-                "sm_max_mhz": max(smax) if smax else None,
-                "power_w_max": max(pw) if pw else None,
-                "samples": len(rows), "reasons": reasons}
+        sm = [s[0] for s in self.samples]
+        pw = [s[1] for s in self.samples]
+        reasons = sorted({n for s in self.samples for n, bit in self.REASONS.items() if s[2] & bit})
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": self.sm_max,
+                "power_w_max": round(max(pw), 1), "samples": len(sm), "reasons": reasons,
+                "source": "NVML, 1 ms polling during the timed region"}
 
 
 # ------------------------------------------------------------- our arm
@@ -200,21 +212,27 @@ def run_ours(args):
 
     def step(i):
         q, k, v, o = sets[i % nsets]
-        ia.forward(q, k, v, sc, w.causal, w.clip_c, out=o, stream=stream)
+        ia.forward(q, k, v, sc, w.causal, w.clip_c, out=o, stream=torch.cuda.current_stream(dev))
 
     for i in range(args.warmup):
         step(i)
     torch.cuda.synchronize(dev)
     if ia.device_error(stream) != ia.OK:
         raise RuntimeError("a kernel wait timed out during warm-up")
+    # the K timed steps are captured once as a CUDA graph and replayed: the
+    # device time then excludes the host's per-call launch latency
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph):
+        for i in range(args.steps):
+            step(i)
+    torch.cuda.synchronize(dev)
     clocks = ClockSampler(local_rank)
     barrier(world, dev)
     torch.cuda.synchronize(dev)
     clocks.start()
     t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     t0.record(stream)
-    for i in range(args.steps):
-        step(i)
+    graph.replay()
     t1.record(stream)
     torch.cuda.synchronize(dev)
     barrier(world, dev)
@@ -223,6 +241,7 @@ def run_ours(args):
     ms = max_over_ranks(ms, world, dev)
     if ia.device_error(stream) != ia.OK:
         raise RuntimeError("a kernel wait timed out during the timed steps")
+    del graph
     ops = w.effective_ops
     value = aggregate_value(ops, world, ms * 1e-3) / 1e12
 
@@ -265,6 +284,7 @@ def run_ours(args):
                    "causal": w.causal, "clip_c": w.clip_c,
                    "quant": "per_head" if w.per_head else "per_tensor",
                    "l2": f"inputs rotate over {nsets} copies ({nsets * set_bytes / 2**20:.0f} MiB > 126 MiB L2)",
+                   "timing": "K steps captured as one CUDA graph, replayed once between CUDA events",
                    "parallelism": f"dp{world} (independent problems)"},
         "roofline": {"bound": "tensor", "kernel": "prefill_kernel", "achieved": round(achieved, 3),
                      "peak": round(peak_int8, 1), "unit": "TOPS", "frac": round(achieved / peak_int8, 4),
@@ -326,33 +346,28 @@ def run_decode(args, dev, stream, world, peaks, peak_src):
 
 # ------------------------------------------------------- CPU oracle legs
 def _oracle_sample(w, x, seconds: float):
-    """Time the oracle on whole (b, h) slices until about `seconds` of work."""
+    """Time the oracle on whole (b, h) slices, in order and wrapping around,
+    until about `seconds` of work (at least one slice)."""
     import oracle
     threads = os.cpu_count() or 1
     oracle.build()
     heads = [(b, h) for b in range(w.B) for h in range(w.H)]
-
-    def run(n):
-        sel = heads[:n]
-        done = 0.0
-        t = time.perf_counter()
-        for b in sorted({b for b, _ in sel}):
-            hs = [h for bb, h in sel if bb == b]
-            sl = slice(hs[0], hs[-1] + 1)
-            hsc = (lambda s: s[sl] if w.per_head else s)
-            oracle.forward(x.q[b:b + 1, sl], x.k[b:b + 1, sl], x.v[b:b + 1, sl], w.per_head,
-                           hsc(x.s_q), hsc(x.s_k), hsc(x.s_v), hsc(x.s_o), w.causal, w.clip_c,
-                           nthreads=threads)
-            done += len(hs)
-        return time.perf_counter() - t, done
-
-    dt, n = run(1)
-    per_head = max(dt, 1e-6)
-    want = int(min(len(heads), max(1, seconds / per_head)))
-    if want > 1:
-        dt, n = run(want)
-    ops = w.effective_ops / (w.B * w.H) * n
-    return ops, dt, threads, f"{int(n)} of {w.B * w.H} (b, h) slices of {w.name}, all their rows"
+    done = 0
+    t0 = time.perf_counter()
+    while True:
+        b, h = heads[done % len(heads)]
+        sl = slice(h, h + 1)
+        hsc = (lambda s: s[sl] if w.per_head else s)
+        oracle.forward(x.q[b:b + 1, sl], x.k[b:b + 1, sl], x.v[b:b + 1, sl], w.per_head,
+                       hsc(x.s_q), hsc(x.s_k), hsc(x.s_v), hsc(x.s_o), w.causal, w.clip_c,
+                       nthreads=threads)
+        done += 1
+        dt = time.perf_counter() - t0
+        if dt >= seconds:
+            break
+    ops = w.effective_ops / (w.B * w.H) * done
+    return ops, dt, threads, (f"{done} (b, h) slices of {w.name} (all rows of each; "
+                              f"{done / (w.B * w.H):.2f} passes over the workload)")
 
 
 def cpu_baseline(w, x, seconds):

@@ -126,6 +126,31 @@ bool encode_3d(CUtensorMap* m, const void* base, int d, long long rows, long lon
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// Multiprocessor count of the current device (cached per device).
+int sm_count(int* out) {
+  static int cache[64] = {};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return INTATTN_ERR_CUDA;
+  if (cache[dev] == 0) {
+    int v = 0;
+    if (cudaDeviceGetAttribute(&v, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || v <= 0)
+      return INTATTN_ERR_CUDA;
+    cache[dev] = v;
+  }
+  *out = cache[dev];
+  return INTATTN_OK;
+}
+
+// Text of the last CUDA error a launch reported (this thread), for
+// intattn_strerror(INTATTN_ERR_CUDA).
+thread_local const char* g_last_cuda_error = nullptr;
+
+int note_launch(cudaError_t e) {
+  if (e == cudaSuccess) return INTATTN_OK;
+  g_last_cuda_error = cudaGetErrorString(e);
+  return INTATTN_ERR_CUDA;
+}
+
 // ------------------------------------------------------- kernel attributes
 template <int D>
 int prefill_launch(const PrefillArgs& args, int grid, cudaStream_t stream) {
@@ -141,7 +166,7 @@ int prefill_launch(const PrefillArgs& args, int grid, cudaStream_t stream) {
     attr_set[dev] = true;
   }
   intattn::prefill::prefill_kernel<D><<<grid, intattn::prefill::kThreads, C::kSmemBytes, stream>>>(args);
-  return cudaGetLastError() == cudaSuccess ? INTATTN_OK : INTATTN_ERR_CUDA;
+  return note_launch(cudaGetLastError());
 }
 
 struct DecodeLayout {
@@ -166,9 +191,10 @@ template <int D>
 int decode_launch(const DecodeArgs& a, cudaStream_t stream) {
   const dim3 grid(a.nsplit, a.BH);
   intattn::decode::decode_qk_kernel<D><<<grid, intattn::decode::kThreads, 0, stream>>>(a);
-  if (cudaGetLastError() != cudaSuccess) return INTATTN_ERR_CUDA;
+  const int rc = note_launch(cudaGetLastError());
+  if (rc != INTATTN_OK) return rc;
   intattn::decode::decode_pv_kernel<D><<<grid, intattn::decode::kThreads, 0, stream>>>(a);
-  return cudaGetLastError() == cudaSuccess ? INTATTN_OK : INTATTN_ERR_CUDA;
+  return note_launch(cudaGetLastError());
 }
 
 }  // namespace
@@ -225,7 +251,11 @@ int intattn_forward(const int8_t* q, const int8_t* k, const int8_t* v, const int
   args.causal = causal ? 1 : 0;
   args.n_qtiles = n_qtiles;
   args.per_head = scales->per_head ? 1 : 0;
-  const int grid = static_cast<int>(BH * n_qtiles);
+  args.n_tiles = static_cast<int32_t>(BH * n_qtiles);
+  int sms = 0;
+  if (sm_count(&sms) != INTATTN_OK) return INTATTN_ERR_CUDA;
+  // persistent kernel: one CTA per SM (each holds all 512 TMEM columns)
+  const int grid = args.n_tiles < sms ? args.n_tiles : sms;
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   return d == 64 ? prefill_launch<64>(args, grid, st) : prefill_launch<128>(args, grid, st);
 }
@@ -290,7 +320,8 @@ const char* intattn_strerror(int code) {
     case INTATTN_ERR_INVALID_ARG: return "invalid argument";
     case INTATTN_ERR_UNSUPPORTED: return "unsupported shape, alignment or head count";
     case INTATTN_ERR_PARAM_RANGE: return "scale or clip out of range";
-    case INTATTN_ERR_CUDA: return "CUDA launch or driver call failed";
+    case INTATTN_ERR_CUDA:
+      return g_last_cuda_error ? g_last_cuda_error : "CUDA launch or driver call failed";
     case INTATTN_ERR_WORKSPACE: return "decode workspace missing, misaligned or too small";
     case INTATTN_ERR_TIMEOUT: return "a kernel wait timed out";
     default: return "unknown error";

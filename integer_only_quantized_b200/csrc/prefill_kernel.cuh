@@ -5,24 +5,38 @@
 // sum, reciprocal multiply-shift) gives u8 probabilities; u8 x s8 P.V
 // accumulates in int32 and is requantised to int8.
 //
-// One CTA owns one (batch, head, 128-query tile).  Warp roles:
-//   warps 0-3  IndexSoftmax + epilogue; thread t owns query row t, which is
-//              TMEM lane t of every accumulator (tcgen05.ld/st 32x32b).
-//   warp 4     TMA producer (one thread): Q once, then K/V tiles through a
-//              ring of shared-memory slots.
-//   warp 5     TMEM allocator and MMA issuer (one thread): tcgen05.mma
-//              kind::i8 for S = Q.K^T (both operands in shared memory) and
-//              O += P.V (P from TMEM, V from shared memory, N-major).
+// Work unit: one (batch, head, 128-query tile).  The kernel is persistent:
+// one CTA per SM takes a tile in each round, in snake order over the tiles
+// sorted longest first (causal), so the loads and MMAs of a tile overlap the
+// reductions and the epilogue of the previous one.  Warp roles:
+//   warps 0-15  IndexSoftmax + epilogue, in two teams of eight.  Team t
+//               (warps 8t .. 8t+7) takes the S tiles whose running index is
+//               t mod 2, so one team computes while the other waits for its
+//               next tile.  Warp w reads TMEM lane quadrant w % 4 (query rows
+//               32(w%4) .. +31, one row per thread) and key half (w / 4) % 2
+//               (64 of the 128 keys of an S tile).  Row max and row sum
+//               combine the four partial results of a row (two teams x two
+//               halves) through shared memory.
+//   warp 16     TMA producer (one thread): Q (double-buffered), then K/V
+//               tiles through a ring of shared-memory slots.
+//   warp 17     TMEM allocator and MMA issuer (one thread): tcgen05.mma
+//               kind::i8 for S = Q.K^T (both operands in shared memory) and
+//               O += P.V (P from TMEM, V from shared memory, N-major).
 //
 // The LUT index of a score depends on the final row max and P depends on
 // the final row sum Z, so a bit-exact result needs three sweeps over the
 // keys of a row (online rescaling would round differently):
-//   pass A  S tiles -> running row max m
+//   pass A  S tiles -> row max m
 //   pass B  S tiles -> Z = sum LUT[idx]; then R and the per-row table
 //           Ptab[i] = (LUT[i] R + 2^31) >> 32
 //   pass C  S tiles -> P = Ptab[idx] packed 4 per TMEM column -> O += P.V
 // S is recomputed by the tensor cores in each pass; K streams three times
 // (from L2 after the first), V once.
+//
+// Every mbarrier wait is bounded (polls with a time limit).  In each softmax
+// team one leader warp polls and the other warps sleep in a named barrier
+// that ANDs the leader's verdict (bar.red.and), so all warps of a team leave
+// together, also on a timeout, and no warp can be left waiting.
 #pragma once
 #include <cuda.h>
 #include <climits>
@@ -38,22 +52,48 @@ struct PrefillArgs {
   CUtensorMap tm_k;  // [B*H, Lk, d]
   CUtensorMap tm_v;  // [B*H, Lk, d]
   int8_t* out;       // [B, H, Lq, d]
-  int32_t BH, H, Lq, Lk, causal, n_qtiles, per_head;
+  int32_t BH, H, Lq, Lk, causal, n_qtiles, per_head, n_tiles;
   uint32_t lut[32];
   HeadParamsDev hp[INTATTN_MAX_HEADS];
 };
 
 namespace prefill {
 
-constexpr int kBM = 128;       // query rows per CTA (MMA M)
-constexpr int kBN = 128;       // keys per S tile (QK MMA N)
-constexpr int kThreads = 192;  // 4 softmax warps + producer warp + MMA warp
+constexpr int kBM = 128;                  // query rows per tile (MMA M)
+constexpr int kBN = 128;                  // keys per S tile (QK MMA N)
+constexpr int kGroups = 4;                // partial results per query row (team x half)
+constexpr int kCols = kBN / 2;            // S columns per thread and tile (a key half)
+constexpr int kSoftWarps = 16;            // two teams of eight
+constexpr int kTeamWarps = 8;
+constexpr int kProducerWarp = kSoftWarps;
+constexpr int kMmaWarp = kSoftWarps + 1;
+constexpr int kThreads = 32 * (kSoftWarps + 2);  // 576
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kColS = 0;    // two S buffers: [0,128) and [128,256)
 constexpr uint32_t kColO = 256;  // O accumulator: d columns
-constexpr uint32_t kColP = 384;  // two P buffers of 32 columns (128 u8 keys)
+constexpr uint32_t kColP = 384;  // four P buffers of 32 columns (128 u8 keys each)
+constexpr int kPBufs = 4;
+// named barriers (id 0 is __syncthreads)
+constexpr uint32_t kNbAll = 1;   // all softmax warps
+constexpr uint32_t kNbTeam = 2;  // + team: the warps of one team
+
+static_assert(kCols == 64, "two 32-column TMEM loads per thread and tile");
 
 enum Role : unsigned { kRoleSoftmax = 1, kRoleProducer = 2, kRoleMma = 3 };
+
+// Shared-memory barriers, by index.
+enum Bar : int {
+  kBarQFull = 0,        // [2]  Q tile landed
+  kBarQEmpty = 2,       // [2]  every MMA reading that Q buffer is done
+  kBarSFull = 4,        // [2]  S tile ready in TMEM
+  kBarSEmpty = 6,       // [2]  S tile loaded by all softmax warps
+  kBarPFull = 8,        // [4]  P tile written to TMEM
+  kBarPEmpty = 12,      // [4]  P.V MMA that read it is done
+  kBarOFull = 16,       //      all P.V MMAs of a tile done
+  kBarOEmpty = 17,      //      epilogue has read O
+  kBarDrain = 18,       //      final MMA drain
+  kBarKvFull = 19,      // [stages], then kv_empty[stages]
+};
 
 template <int D>
 struct Cfg {
@@ -62,13 +102,12 @@ struct Cfg {
   static constexpr uint32_t kQBytes = kBM * D;
   static constexpr uint32_t kSwizzle = (D == 128) ? 2u : 4u;  // 128B / 64B swizzle
   static constexpr uint32_t kSBO = 8 * D;  // 8 rows of D bytes
-  // barriers: q_full, kv_full[S], kv_empty[S], s_full[2], s_empty[2],
-  // p_full[2], p_empty[2], o_full, drain
-  static constexpr int kNumBars = 1 + 2 * kStages + 8 + 2;
-  static constexpr uint32_t kOffQ = 0;
-  static constexpr uint32_t kOffKV = kOffQ + kQBytes;
-  static constexpr uint32_t kOffPtab = kOffKV + kStages * kTileBytes;
-  static constexpr uint32_t kOffLut = kOffPtab + 32 * kBM * 4;
+  static constexpr int kNumBars = kBarKvFull + 2 * kStages;
+  static constexpr uint32_t kOffQ = 0;                                  // [2] Q tiles
+  static constexpr uint32_t kOffKV = kOffQ + 2 * kQBytes;
+  static constexpr uint32_t kOffPtab = kOffKV + kStages * kTileBytes;    // [32][kBM] u32
+  static constexpr uint32_t kOffRed = kOffPtab + 32 * kBM * 4;          // [2][kGroups][kBM] int32
+  static constexpr uint32_t kOffLut = kOffRed + 2 * kGroups * kBM * 4;
   static constexpr uint32_t kOffBars = kOffLut + 32 * 4;
   static constexpr uint32_t kOffTmem = kOffBars + kNumBars * 8;
   static constexpr uint32_t kUsed = kOffTmem + 16;
@@ -87,64 +126,82 @@ __device__ __forceinline__ uint32_t requant_byte(int32_t acc, int32_t Mo, int32_
   return static_cast<uint32_t>(static_cast<uint8_t>(static_cast<int8_t>(y)));
 }
 
+// Four u8 values (each < 256 in a 32-bit register) into one word, byte k = p_k.
+__device__ __forceinline__ uint32_t pack4(uint32_t p0, uint32_t p1, uint32_t p2, uint32_t p3) {
+  return __byte_perm(__byte_perm(p0, p1, 0x3340), __byte_perm(p2, p3, 0x3340), 0x5410);
+}
+
+// Geometry of one work unit.
+struct Tile {
+  int bh, h, q0, nkt;
+};
+
+// Tile of round `round` for CTA `cta`: rounds alternate direction over the
+// tiles (sorted longest first for causal), which evens out the work per CTA.
+__device__ __forceinline__ int tile_index(int round, int cta, int ctas) {
+  return round * ctas + ((round & 1) ? (ctas - 1 - cta) : cta);
+}
+
+__device__ __forceinline__ Tile tile_of(const PrefillArgs& a, int L) {
+  Tile t;
+  const int rank = L / a.BH;
+  t.bh = L - rank * a.BH;
+  const int qt = a.causal ? (a.n_qtiles - 1 - rank) : rank;
+  t.q0 = qt * kBM;
+  t.h = t.bh % a.H;
+  const int off = a.Lk - a.Lq;
+  const int q_last = min(t.q0 + kBM, a.Lq) - 1;
+  const int kend = a.causal ? min(a.Lk, q_last + off + 1) : a.Lk;
+  t.nkt = (kend + kBN - 1) / kBN;
+  return t;
+}
+
 template <int D>
 __global__ void __launch_bounds__(kThreads, 1) prefill_kernel(const __grid_constant__ PrefillArgs args) {
   using C = Cfg<D>;
-  extern __shared__ uint8_t smem_raw[];
-  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  // 1024-byte aligned base (swizzled TMA tiles); offsetting the __shared__
+  // array keeps the compiler aware of the address space.
+  uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
   const uint32_t s_base = smem_u32(smem);
-  const uint32_t sQ = s_base + C::kOffQ;
   const uint32_t sKV = s_base + C::kOffKV;
   uint32_t* ptab = reinterpret_cast<uint32_t*>(smem + C::kOffPtab);
+  int32_t* red = reinterpret_cast<int32_t*>(smem + C::kOffRed);
   uint32_t* lut_s = reinterpret_cast<uint32_t*>(smem + C::kOffLut);
   const uint32_t bars = s_base + C::kOffBars;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::kOffTmem);
-
-  const uint32_t bar_q_full = bars;
-  auto bar_kv_full = [&](int i) { return bars + 8u * (1 + i); };
-  auto bar_kv_empty = [&](int i) { return bars + 8u * (1 + C::kStages + i); };
-  auto bar_s_full = [&](int i) { return bars + 8u * (1 + 2 * C::kStages + i); };
-  auto bar_s_empty = [&](int i) { return bars + 8u * (3 + 2 * C::kStages + i); };
-  auto bar_p_full = [&](int i) { return bars + 8u * (5 + 2 * C::kStages + i); };
-  auto bar_p_empty = [&](int i) { return bars + 8u * (7 + 2 * C::kStages + i); };
-  const uint32_t bar_o_full = bars + 8u * (9 + 2 * C::kStages);
-  const uint32_t bar_drain = bars + 8u * (10 + 2 * C::kStages);
+  auto bar = [&](int i) { return bars + 8u * static_cast<uint32_t>(i); };
+  auto bar_kv_full = [&](int i) { return bar(kBarKvFull + i); };
+  auto bar_kv_empty = [&](int i) { return bar(kBarKvFull + C::kStages + i); };
+  auto sQ = [&](uint32_t i) { return s_base + C::kOffQ + i * C::kQBytes; };
 
   const int tid = threadIdx.x;
   const int warp = tid >> 5;
   const int lane = tid & 31;
 
-  // ---- tile of this CTA (causal: the longest key ranges launch first) ----
-  const int rank = blockIdx.x / args.BH;
-  const int bh = blockIdx.x - rank * args.BH;
-  const int qt = args.causal ? (args.n_qtiles - 1 - rank) : rank;
-  const int q0 = qt * kBM;
-  const int h = bh % args.H;
-  const HeadParamsDev hp = args.hp[args.per_head ? h : 0];
-  const int off = args.Lk - args.Lq;
-  const int q_last = min(q0 + kBM, args.Lq) - 1;
-  const int kend = args.causal ? min(args.Lk, q_last + off + 1) : args.Lk;
-  const int nkt = (kend + kBN - 1) / kBN;
-
-  // ---- set-up: barriers, LUT, TMEM ----
+  // ---- set-up: barriers, LUT, TMEM (once per CTA) ----
   if (tid == 0) {
-    mbar_init(bar_q_full, 1);
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(bar(kBarQFull + i), 1);
+      mbar_init(bar(kBarQEmpty + i), 1);
+      mbar_init(bar(kBarSFull + i), 1);
+      mbar_init(bar(kBarSEmpty + i), kTeamWarps);
+    }
+    for (int i = 0; i < kPBufs; ++i) {
+      mbar_init(bar(kBarPFull + i), kTeamWarps);
+      mbar_init(bar(kBarPEmpty + i), 1);
+    }
+    mbar_init(bar(kBarOFull), 1);
+    mbar_init(bar(kBarOEmpty), kSoftWarps);
+    mbar_init(bar(kBarDrain), 1);
     for (int i = 0; i < C::kStages; ++i) {
       mbar_init(bar_kv_full(i), 1);
       mbar_init(bar_kv_empty(i), 1);
     }
-    for (int i = 0; i < 2; ++i) {
-      mbar_init(bar_s_full(i), 1);
-      mbar_init(bar_s_empty(i), kBM);
-      mbar_init(bar_p_full(i), kBM);
-      mbar_init(bar_p_empty(i), 1);
-    }
-    mbar_init(bar_o_full, 1);
-    mbar_init(bar_drain, 1);
     mbar_fence_init();
   }
   if (tid < 32) lut_s[tid] = args.lut[tid];
-  if (warp == 5) {
+  if (warp == kMmaWarp) {
     tmem_alloc(smem_u32(tmem_slot), kTmemCols);
     tmem_relinquish();
   }
@@ -153,179 +210,240 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_kernel(const __grid_const
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
 
-  if (warp < 4) {
+  if (warp < kSoftWarps) {
     // ======================= IndexSoftmax warps =======================
-    const int r = tid;  // query row within the tile == TMEM lane
-    const uint32_t trow = tmem + (static_cast<uint32_t>(warp * 32) << 16);
-    const int row_limit = q0 + r + off;  // causal: last visible key of this row
-    auto tile_full = [&](int j) {
-      const int last = (j + 1) * kBN - 1;
-      return last < args.Lk && (!args.causal || last <= q0 + off);
-    };
-    auto valid = [&](int key) { return key < args.Lk && (!args.causal || key <= row_limit); };
+    const int quad = warp & 3;
+    const int half = (warp >> 2) & 1;
+    const int team = warp >> 3;
+    const int grp = team * 2 + half;  // slot of this thread's partial results
+    const int r = quad * 32 + lane;   // query row within the tile == TMEM lane
+    const uint32_t tlane = tmem + (static_cast<uint32_t>(quad * 32) << 16);
+    const uint32_t trow = tlane + half * kCols;
+    const uint32_t prow = smem_u32(ptab) + 4u * r;  // Ptab[i][r] at prow + 512 i
+    // lane i holds LUT[i] as a float; a shuffle whose source lane is the low
+    // 5 bits of the index bits looks it up.  Per tile a thread sums 32 values
+    // below 2^15, so the float partial sums are exact.
+    const int32_t lut_lane = __float_as_int(__int2float_rn(static_cast<int32_t>(lut_s[lane])));
     bool ok = true;
-    uint32_t sc = 0;  // S tiles consumed (all passes)
-    auto wait_s = [&](uint32_t& buf) {
-      buf = sc & 1;
-      const bool got = mbar_wait(bar_s_full(buf), (sc >> 1) & 1, kRoleSoftmax);
-      return __all_sync(0xffffffffu, got);
+    uint32_t sc = 0;  // S tiles of the CTA so far (both teams, all passes and tiles)
+    uint32_t pc = 0;  // P tiles of the CTA so far
+    const bool leader = (warp & (kTeamWarps - 1)) == 0;  // warps 0 and 8 poll for their team
+    // wait for a barrier phase: the team leader polls, the team sleeps in a
+    // named barrier that hands everyone the leader's verdict
+    auto team_wait = [&](uint32_t b, uint32_t parity) {
+      const bool got = leader ? mbar_wait(b, parity, kRoleSoftmax) : true;
+      return bar_red_and(kNbTeam + team, 32 * kTeamWarps, got);
     };
-
-    // ---- pass A: row max over valid keys ----
-    int32_t m = INT_MIN;
-    for (int j = 0; j < nkt; ++j, ++sc) {
-      uint32_t buf;
-      if (!wait_s(buf)) { ok = false; break; }
+    // all sixteen softmax warps: every warp's `ok`, and (warp 0 polling) a phase
+    auto all_sync = [&](bool mine) { return bar_red_and(kNbAll, 32 * kSoftWarps, mine); };
+    auto arrive_warp = [&](uint32_t b) {  // one arrival per warp
+      __syncwarp();
+      if (lane == 0) mbar_arrive(b);
+    };
+    // S tile `idx` (running index; this team's tiles have idx % 2 == team,
+    // which is also the buffer) -> registers; released as soon as it is loaded
+    auto load_s = [&](uint32_t idx, uint32_t (&v)[64]) {
+      const uint32_t buf = idx & 1;
+      if (!team_wait(bar(kBarSFull + buf), (idx >> 1) & 1)) return false;
       tc_fence_after();
-      const bool full = tile_full(j);
-#pragma unroll 1
-      for (int c = 0; c < kBN / 32; ++c) {
-        uint32_t v[32];
-        tmem_ld32(trow + kColS + buf * kBN + c * 32, v);
-        tmem_wait_ld();
-        if (full) {
-#pragma unroll
-          for (int k = 0; k < 32; ++k) m = imax(m, static_cast<int32_t>(v[k]));
-        } else {
-          const int key0 = j * kBN + c * 32;
-#pragma unroll
-          for (int k = 0; k < 32; ++k)
-            if (valid(key0 + k)) m = imax(m, static_cast<int32_t>(v[k]));
-        }
-      }
+      uint32_t (&v0)[32] = *reinterpret_cast<uint32_t(*)[32]>(&v[0]);
+      uint32_t (&v1)[32] = *reinterpret_cast<uint32_t(*)[32]>(&v[32]);
+      tmem_ld32(trow + kColS + buf * kBN, v0);
+      tmem_ld32(trow + kColS + buf * kBN + 32, v1);
+      tmem_wait_ld();
       tc_fence_before();
-      mbar_arrive(bar_s_empty(buf));
-    }
+      arrive_warp(bar(kBarSEmpty + buf));
+      return true;
+    };
+    // first tile of a pass of nkt tiles that belongs to this team
+    auto first_j = [&](uint32_t s0) { return static_cast<int>((static_cast<uint32_t>(team) - s0) & 1u); };
 
-    // index of a score: (min(m - S, D) M + 2^(s-1)) >> s, evaluated as
-    // (C - max(S, m - D) M) >> s in wrapping 32-bit arithmetic; the true value
-    // lies in [0, 2^31) so the wrap is exact.
-    const long long lo64 = static_cast<long long>(m) - hp.D;
-    const int32_t lo = lo64 < INT_MIN ? INT_MIN : static_cast<int32_t>(lo64);
-    const uint32_t Mu = static_cast<uint32_t>(hp.M);
-    const uint32_t sh = static_cast<uint32_t>(hp.s);
-    const uint32_t Cm = static_cast<uint32_t>(m) * Mu + (1u << (sh - 1));
+    for (int it = 0; ok; ++it) {
+      const int L = tile_index(it, blockIdx.x, gridDim.x);
+      if (L >= args.n_tiles) break;
+      const Tile T = tile_of(args, L);
+      const HeadParamsDev hp = args.hp[args.per_head ? T.h : 0];
+      const int off = args.Lk - args.Lq;
+      const int row_limit = T.q0 + r + off;  // causal: last visible key of this row
+      auto tile_full = [&](int j) {
+        const int last = (j + 1) * kBN - 1;
+        return last < args.Lk && (!args.causal || last <= T.q0 + off);
+      };
+      // keys of this thread's 64-key segment of tile j that are visible: a prefix
+      const int key_lim = args.causal ? min(args.Lk, row_limit + 1) : args.Lk;
+      auto nvalid = [&](int j) { return min(max(key_lim - (j * kBN + half * kCols), 0), kCols); };
 
-    // ---- pass B: Z = sum of pseudo-exponentials ----
-    int32_t Z = 0;
-    for (int j = 0; ok && j < nkt; ++j, ++sc) {
-      uint32_t buf;
-      if (!wait_s(buf)) { ok = false; break; }
-      tc_fence_after();
-      const bool full = tile_full(j);
-#pragma unroll 1
-      for (int c = 0; c < kBN / 32; ++c) {
-        uint32_t v[32];
-        tmem_ld32(trow + kColS + buf * kBN + c * 32, v);
-        tmem_wait_ld();
-        if (full) {
+      // ---- pass A: row max over valid keys ----
+      int32_t m = INT_MIN;
+      for (int j = first_j(sc); j < T.nkt; j += 2) {
+        uint32_t v[64];
+        if (!load_s(sc + j, v)) { ok = false; break; }
+        int32_t m4[4] = {INT_MIN, INT_MIN, INT_MIN, INT_MIN};
+        if (tile_full(j)) {
 #pragma unroll
-          for (int k = 0; k < 32; ++k) {
-            const int32_t t = imax(static_cast<int32_t>(v[k]), lo);
-            Z += static_cast<int32_t>(lut_s[(Cm - static_cast<uint32_t>(t) * Mu) >> sh]);
+          for (int k = 0; k < 64; k += 8) {
+            m4[0] = __vimax3_s32(m4[0], static_cast<int32_t>(v[k + 0]), static_cast<int32_t>(v[k + 1]));
+            m4[1] = __vimax3_s32(m4[1], static_cast<int32_t>(v[k + 2]), static_cast<int32_t>(v[k + 3]));
+            m4[2] = __vimax3_s32(m4[2], static_cast<int32_t>(v[k + 4]), static_cast<int32_t>(v[k + 5]));
+            m4[3] = __vimax3_s32(m4[3], static_cast<int32_t>(v[k + 6]), static_cast<int32_t>(v[k + 7]));
           }
         } else {
-          // a masked key takes the clip value lo: index 31, LUT[31] = 0
-          const int key0 = j * kBN + c * 32;
+          const int nv = nvalid(j);
 #pragma unroll
-          for (int k = 0; k < 32; ++k) {
-            const int32_t t = valid(key0 + k) ? imax(static_cast<int32_t>(v[k]), lo) : lo;
-            Z += static_cast<int32_t>(lut_s[(Cm - static_cast<uint32_t>(t) * Mu) >> sh]);
+          for (int k = 0; k < 64; ++k) m4[k & 3] = imax(m4[k & 3], k < nv ? static_cast<int32_t>(v[k]) : INT_MIN);
+        }
+        m = imax(m, imax(imax(m4[0], m4[1]), imax(m4[2], m4[3])));
+      }
+      sc += T.nkt;
+      red[grp * kBM + r] = m;
+      if (!all_sync(ok)) { ok = false; break; }
+      m = imax(imax(red[r], red[kBM + r]), imax(red[2 * kBM + r], red[3 * kBM + r]));
+
+      // LUT index of a score, idx = floor((min(m - S, D) M + 2^(s-1)) / 2^s),
+      // evaluated exactly on the FP32 pipe (the integer pipe is the scarcer one):
+      //  * (0x4B000000 + m) - S, read as a float, is 2^23 + (m - S) exactly
+      //    (0 <= m - S <= 2^22);
+      //  * fminf clips the gap at D' = min(D, 2^22 + 1) (D' = D whenever a gap
+      //    can reach D);
+      //  * every valid parameter set has s in {24, 25, 26}, so Ms = M 2^-s and
+      //    c0 = 1/2 - 2^23 Ms are exact floats, and one fused multiply-add
+      //    rounded toward zero gives RZ(gap M / 2^s + 1/2), whose floor is idx;
+      //  * adding 2^23 rounded toward zero leaves 0x4B000000 + idx in the bits:
+      //    the low 5 bits are idx, and (bits * 512) mod 2^32 is idx * 512.
+      // A masked key uses the bits 0x4B00001F: index 31, LUT[31] = 0, Ptab[31] = 0.
+      const uint32_t Cx = 0x4B000000u + static_cast<uint32_t>(m);
+      const int32_t Dp = hp.D < (1 << 22) + 1 ? hp.D : (1 << 22) + 1;
+      const float Xclip = __uint_as_float(0x4B000000u + static_cast<uint32_t>(Dp));
+      const float Mf = __int2float_rn(hp.M);                                                     // exact: M <= 2^24
+      const float Ms = Mf * __uint_as_float(static_cast<uint32_t>(127 - hp.s) << 23);           // M 2^-s
+      const float c0 = 0.5f - Mf * __uint_as_float(static_cast<uint32_t>(127 + 23 - hp.s) << 23);  // exact
+      auto idx_bits = [&](uint32_t sv) {
+        const float X = fminf(__uint_as_float(Cx - sv), Xclip);
+        return __float_as_uint(__fadd_rz(__fmaf_rz(X, Ms, c0), 8388608.0f));
+      };
+      constexpr uint32_t kMaskedBits = 0x4B00001Fu;
+
+      // ---- pass B: Z = sum of pseudo-exponentials ----
+      int32_t Z = 0;
+      for (int j = first_j(sc); j < T.nkt; j += 2) {
+        uint32_t v[64];
+        if (!load_s(sc + j, v)) { ok = false; break; }
+        float z4[4] = {0.f, 0.f, 0.f, 0.f};
+        if (tile_full(j)) {
+#pragma unroll
+          for (int k = 0; k < 64; ++k)
+            z4[k & 3] += __int_as_float(__shfl_sync(0xffffffffu, lut_lane, static_cast<int>(idx_bits(v[k]))));
+        } else {
+          const int nv = nvalid(j);
+#pragma unroll
+          for (int k = 0; k < 64; ++k) {
+            const uint32_t ib = k < nv ? idx_bits(v[k]) : kMaskedBits;
+            z4[k & 3] += __int_as_float(__shfl_sync(0xffffffffu, lut_lane, static_cast<int>(ib)));
           }
         }
+        Z += __float2int_rn((z4[0] + z4[1]) + (z4[2] + z4[3]));
       }
-      tc_fence_before();
-      mbar_arrive(bar_s_empty(buf));
-    }
+      sc += T.nkt;
+      red[(kGroups + grp) * kBM + r] = Z;
+      if (!all_sync(ok)) { ok = false; break; }
+      Z = (red[kGroups * kBM + r] + red[(kGroups + 1) * kBM + r]) +
+          (red[(kGroups + 2) * kBM + r] + red[(kGroups + 3) * kBM + r]);
 
-    // reciprocal and this row's probability table
-    if (ok) {
-      const unsigned long long R =
-          ((255ull << 32) + static_cast<unsigned long long>(Z >> 1)) / static_cast<unsigned long long>(Z);
-#pragma unroll
-      for (int i = 0; i < 32; ++i)
-        ptab[i * kBM + r] = static_cast<uint32_t>((static_cast<unsigned long long>(lut_s[i]) * R + (1ull << 31)) >> 32);
-    }
-
-    // ---- pass C: P tiles into TMEM for the P.V MMAs ----
-    for (int j = 0; ok && j < nkt; ++j, ++sc) {
-      uint32_t buf;
-      if (!wait_s(buf)) { ok = false; break; }
-      const uint32_t pb = j & 1;
+      // reciprocal and this row's probability table (each of the four threads
+      // of a row writes 8 of the 32 entries)
       {
-        const bool got = mbar_wait(bar_p_empty(pb), ((j >> 1) & 1) ^ 1, kRoleSoftmax);
-        if (!__all_sync(0xffffffffu, got)) { ok = false; break; }
-      }
-      tc_fence_after();
-      const bool full = tile_full(j);
-#pragma unroll 1
-      for (int c = 0; c < kBN / 32; ++c) {
-        uint32_t v[32];
-        tmem_ld32(trow + kColS + buf * kBN + c * 32, v);
-        tmem_wait_ld();
-        uint32_t pw[8];
-        const int key0 = j * kBN + c * 32;
+        // R = floor(N / Z), N = 255 2^32 + floor(Z/2) < 2^40: the double
+        // quotient is within one unit of R, and one integer step makes it exact.
+        const unsigned long long N = (255ull << 32) + static_cast<unsigned long long>(Z >> 1);
+        const unsigned long long Zu = static_cast<unsigned long long>(Z);
+        unsigned long long R =
+            static_cast<unsigned long long>(__ddiv_rn(static_cast<double>(N), static_cast<double>(Z)));
+        if (R * Zu > N) --R;
+        else if ((R + 1) * Zu <= N) ++R;
 #pragma unroll
-        for (int q = 0; q < 8; ++q) {
-          uint32_t word = 0;
-#pragma unroll
-          for (int b = 0; b < 4; ++b) {
-            const int k = q * 4 + b;
-            // masked key: index 31, Ptab[31] = 0
-            const int32_t t = (full || valid(key0 + k)) ? imax(static_cast<int32_t>(v[k]), lo) : lo;
-            const uint32_t p = ptab[((Cm - static_cast<uint32_t>(t) * Mu) >> sh) * kBM + r];
-            word |= p << (8 * b);
-          }
-          pw[q] = word;
-        }
-        tmem_st8(trow + kColP + pb * 32 + c * 8, pw);
+        for (int i = grp * 8; i < grp * 8 + 8; ++i)
+          ptab[i * kBM + r] = static_cast<uint32_t>((static_cast<unsigned long long>(lut_s[i]) * R + (1ull << 31)) >> 32);
       }
-      tmem_wait_st();
-      tc_fence_before();
-      mbar_arrive(bar_s_empty(buf));
-      mbar_arrive(bar_p_full(pb));
-    }
+      all_sync(true);  // the table is complete
 
-    // ---- epilogue: O (int32, TMEM) -> requantised int8 rows ----
-    if (ok) {
-      const bool got = mbar_wait(bar_o_full, 0, kRoleSoftmax);
-      ok = __all_sync(0xffffffffu, got);
-    }
-    if (ok) {
-      tc_fence_after();
-      const int row = q0 + r;
-      int8_t* dst = args.out + (static_cast<size_t>(bh) * args.Lq + row) * D;
-#pragma unroll 1
-      for (int c = 0; c < D / 32; ++c) {
-        uint32_t v[32];
-        tmem_ld32(trow + kColO + c * 32, v);
-        tmem_wait_ld();
-        uint32_t w[8];
+      // ---- pass C: P tiles into TMEM for the P.V MMAs ----
+      for (int j = first_j(sc); j < T.nkt; j += 2) {
+        const uint32_t pi = pc + j;  // running P index of this tile
+        const uint32_t pb = pi & (kPBufs - 1);
+        if (!team_wait(bar(kBarPEmpty + pb), ((pi / kPBufs) & 1) ^ 1)) { ok = false; break; }
+        uint32_t v[64];
+        if (!load_s(sc + j, v)) { ok = false; break; }
+        uint32_t pw[16];
+        if (tile_full(j)) {
 #pragma unroll
-        for (int q = 0; q < 8; ++q) {
-          w[q] = requant_byte(static_cast<int32_t>(v[4 * q + 0]), hp.Mo, hp.so) |
-                 (requant_byte(static_cast<int32_t>(v[4 * q + 1]), hp.Mo, hp.so) << 8) |
-                 (requant_byte(static_cast<int32_t>(v[4 * q + 2]), hp.Mo, hp.so) << 16) |
-                 (requant_byte(static_cast<int32_t>(v[4 * q + 3]), hp.Mo, hp.so) << 24);
+          for (int q = 0; q < 16; ++q) {
+            uint32_t p[4];
+#pragma unroll
+            for (int b = 0; b < 4; ++b) p[b] = lds_u32(idx_bits(v[q * 4 + b]) * 512u + prow);
+            pw[q] = pack4(p[0], p[1], p[2], p[3]);
+          }
+        } else {
+          const int nv = nvalid(j);
+#pragma unroll
+          for (int q = 0; q < 16; ++q) {
+            uint32_t p[4];
+#pragma unroll
+            for (int b = 0; b < 4; ++b) {
+              const int k = q * 4 + b;
+              const uint32_t ib = k < nv ? idx_bits(v[k]) : kMaskedBits;
+              p[b] = lds_u32(ib * 512u + prow);
+            }
+            pw[q] = pack4(p[0], p[1], p[2], p[3]);
+          }
         }
-        if (row < args.Lq) {
-          uint4* o = reinterpret_cast<uint4*>(dst + c * 32);
-          o[0] = make_uint4(w[0], w[1], w[2], w[3]);
-          o[1] = make_uint4(w[4], w[5], w[6], w[7]);
-        }
+        tmem_st16(tlane + kColP + pb * 32 + half * 16, pw);
+        tmem_wait_st();
+        tc_fence_before();
+        arrive_warp(bar(kBarPFull + pb));
+      }
+      sc += T.nkt;
+      pc += T.nkt;
+
+      // ---- epilogue: O (int32, TMEM) -> requantised int8 rows ----
+      {
+        const bool got = (ok && warp == 0) ? mbar_wait(bar(kBarOFull), it & 1, kRoleSoftmax) : ok;
+        if (!all_sync(got)) { ok = false; break; }
+      }
+      tc_fence_after();
+      constexpr int kOC = D / kGroups;  // output columns per thread: 16 or 32
+      uint32_t v[32];
+      if constexpr (kOC == 32) {
+        tmem_ld32(tlane + kColO + grp * kOC, v);
+      } else {
+        tmem_ld16(tlane + kColO + grp * kOC, v);
+      }
+      tmem_wait_ld();
+      tc_fence_before();
+      arrive_warp(bar(kBarOEmpty));  // O may now be overwritten by the next tile
+      uint32_t w[8];
+#pragma unroll
+      for (int q = 0; q < kOC / 4; ++q)
+        w[q] = pack4(requant_byte(static_cast<int32_t>(v[4 * q + 0]), hp.Mo, hp.so),
+                     requant_byte(static_cast<int32_t>(v[4 * q + 1]), hp.Mo, hp.so),
+                     requant_byte(static_cast<int32_t>(v[4 * q + 2]), hp.Mo, hp.so),
+                     requant_byte(static_cast<int32_t>(v[4 * q + 3]), hp.Mo, hp.so));
+      const int row = T.q0 + r;
+      if (row < args.Lq) {
+        uint4* o = reinterpret_cast<uint4*>(args.out + (static_cast<size_t>(T.bh) * args.Lq + row) * D + grp * kOC);
+        o[0] = make_uint4(w[0], w[1], w[2], w[3]);
+        if constexpr (kOC == 32) o[1] = make_uint4(w[4], w[5], w[6], w[7]);
       }
     }
-  } else if (warp == 4) {
+  } else if (warp == kProducerWarp) {
     // ============================ TMA producer ============================
     if (lane == 0) {
       tma_prefetch_desc(&args.tm_q);
       tma_prefetch_desc(&args.tm_k);
       tma_prefetch_desc(&args.tm_v);
-      mbar_arrive_expect_tx(bar_q_full, C::kQBytes);
-      tma_load_3d(sQ, &args.tm_q, bar_q_full, 0, q0, bh);
-      uint32_t n = 0;  // loads issued, in the MMA warp's consumption order
+      uint32_t n = 0;   // K/V loads issued, in the MMA warp's consumption order
+      uint32_t nq = 0;  // Q loads issued
       bool ok = true;
-      auto load = [&](const CUtensorMap* tm, int j) {
+      auto load = [&](const CUtensorMap* tm, int j, int bh) {
         if (!ok) return;
         const uint32_t slot = n % C::kStages;
         const uint32_t use = n / C::kStages;
@@ -334,12 +452,23 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_kernel(const __grid_const
         tma_load_3d(sKV + slot * C::kTileBytes, tm, bar_kv_full(slot), 0, j * kBN, bh);
         ++n;
       };
-      for (int pass = 0; pass < 2; ++pass)
-        for (int j = 0; j < nkt; ++j) load(&args.tm_k, j);
-      load(&args.tm_k, 0);
-      for (int j = 0; j < nkt; ++j) {
-        if (j + 1 < nkt) load(&args.tm_k, j + 1);
-        load(&args.tm_v, j);
+      for (int it = 0; ok; ++it) {
+        const int L = tile_index(it, blockIdx.x, gridDim.x);
+        if (L >= args.n_tiles) break;
+        const Tile T = tile_of(args, L);
+        const uint32_t qb = nq & 1;
+        if (!mbar_wait(bar(kBarQEmpty + qb), ((nq >> 1) & 1) ^ 1, kRoleProducer)) { ok = false; break; }
+        mbar_arrive_expect_tx(bar(kBarQFull + qb), C::kQBytes);
+        tma_load_3d(sQ(qb), &args.tm_q, bar(kBarQFull + qb), 0, T.q0, T.bh);
+        ++nq;
+        for (int pass = 0; pass < 2; ++pass)
+          for (int j = 0; j < T.nkt; ++j) load(&args.tm_k, j, T.bh);
+        load(&args.tm_k, 0, T.bh);
+        if (T.nkt > 1) load(&args.tm_k, 1, T.bh);
+        for (int j = 0; j < T.nkt; ++j) {
+          if (j + 2 < T.nkt) load(&args.tm_k, j + 2, T.bh);
+          load(&args.tm_v, j, T.bh);
+        }
       }
       // never leave with a copy in flight: wait for the last load of each slot
       for (uint32_t slot = 0; slot < static_cast<uint32_t>(C::kStages); ++slot) {
@@ -348,62 +477,86 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_kernel(const __grid_const
           mbar_wait(bar_kv_full(slot), (uses - 1) & 1, kRoleProducer);
         }
       }
-      mbar_wait(bar_q_full, 0, kRoleProducer);
+      for (uint32_t i = 0; i < 2 && i < nq; ++i) {
+        const uint32_t last = nq - 1 - i;  // the last load of each Q buffer
+        mbar_wait(bar(kBarQFull + (last & 1)), (last >> 1) & 1, kRoleProducer);
+      }
     }
   } else {
     // ============================= MMA issuer =============================
     if (lane == 0) {
       constexpr uint32_t idesc_qk = idesc_i8(kBM, kBN, 1, 1, 0);  // s8 x s8, K-major B
       constexpr uint32_t idesc_pv = idesc_i8(kBM, D, 0, 1, 1);    // u8 x s8, N-major B
-      const uint64_t q_desc = smem_desc(sQ, 16, C::kSBO, C::kSwizzle);
-      bool ok = mbar_wait(bar_q_full, 0, kRoleMma);
+      bool ok = true;
       uint32_t n = 0;   // K/V tiles consumed
       uint32_t sc = 0;  // S tiles produced
-      auto issue_qk = [&]() {
-        if (!ok) return;
-        const uint32_t buf = sc & 1;
-        if (!mbar_wait(bar_s_empty(buf), ((sc >> 1) & 1) ^ 1, kRoleMma)) { ok = false; return; }
-        const uint32_t slot = n % C::kStages;
-        if (!mbar_wait(bar_kv_full(slot), (n / C::kStages) & 1, kRoleMma)) { ok = false; return; }
-        tc_fence_after();
-        const uint64_t k_desc = smem_desc(sKV + slot * C::kTileBytes, 16, C::kSBO, C::kSwizzle);
+      uint32_t pc = 0;  // P tiles consumed
+      for (int it = 0; ok; ++it) {
+        const int L = tile_index(it, blockIdx.x, gridDim.x);
+        if (L >= args.n_tiles) break;
+        const Tile T = tile_of(args, L);
+        const uint32_t qb = it & 1;
+        if (!mbar_wait(bar(kBarQFull + qb), (it >> 1) & 1, kRoleMma)) { ok = false; break; }
+        const uint64_t q_desc = smem_desc(sQ(qb), 16, C::kSBO, C::kSwizzle);
+        auto issue_qk = [&]() {
+          if (!ok) return;
+          const uint32_t buf = sc & 1;
+          const uint32_t slot = n % C::kStages;
+          if (!mbar_wait2(bar(kBarSEmpty + buf), ((sc >> 1) & 1) ^ 1, bar_kv_full(slot), (n / C::kStages) & 1,
+                          kRoleMma)) {
+            ok = false;
+            return;
+          }
+          tc_fence_after();
+          const uint64_t k_desc = smem_desc(sKV + slot * C::kTileBytes, 16, C::kSBO, C::kSwizzle);
 #pragma unroll
-        for (int kk = 0; kk < D / 32; ++kk)  // K = 32 bytes per MMA: advance 32 B
-          mma_i8_ss(tmem + kColS + buf * kBN, q_desc + 2 * kk, k_desc + 2 * kk, idesc_qk, kk > 0);
-        mma_commit(bar_kv_empty(slot));
-        mma_commit(bar_s_full(buf));
-        ++n;
-        ++sc;
-      };
-      for (int t = 0; t < 2 * nkt; ++t) issue_qk();  // passes A and B
-      issue_qk();                                     // pass C, tile 0
-      for (int j = 0; ok && j < nkt; ++j) {
-        if (j + 1 < nkt) issue_qk();
+          for (int kk = 0; kk < D / 32; ++kk)  // K = 32 bytes per MMA: advance 32 B
+            mma_i8_ss(tmem + kColS + buf * kBN, q_desc + 2 * kk, k_desc + 2 * kk, idesc_qk, kk > 0);
+          mma_commit(bar_kv_empty(slot));
+          mma_commit(bar(kBarSFull + buf));
+          ++n;
+          ++sc;
+        };
+        for (int t = 0; t < 2 * T.nkt; ++t) issue_qk();  // passes A and B
+        // pass C: S tile j+2 reuses the buffer of tile j, which the softmax
+        // warps release right after loading it, so QK(j+2) goes before P.V(j)
+        issue_qk();
+        if (T.nkt > 1) issue_qk();
+        for (int j = 0; ok && j < T.nkt; ++j, ++pc) {
+          if (j + 2 < T.nkt) issue_qk();
+          if (!ok) break;
+          // O of the previous tile must have been read before it is overwritten
+          if (j == 0 && !mbar_wait(bar(kBarOEmpty), (it & 1) ^ 1, kRoleMma)) { ok = false; break; }
+          const uint32_t pb = pc & (kPBufs - 1);
+          const uint32_t slot = n % C::kStages;
+          if (!mbar_wait2(bar(kBarPFull + pb), (pc / kPBufs) & 1, bar_kv_full(slot), (n / C::kStages) & 1,
+                          kRoleMma)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint64_t v_desc = smem_desc(sKV + slot * C::kTileBytes, 16, C::kSBO, C::kSwizzle);
+#pragma unroll
+          for (int kk = 0; kk < kBN / 32; ++kk)  // 32 keys per MMA: 8 TMEM columns of P, 32 V rows
+            mma_i8_ts(tmem + kColO, tmem + kColP + pb * 32 + kk * 8, v_desc + ((32u * D * kk) >> 4),
+                      idesc_pv, (j > 0 || kk > 0) ? 1u : 0u);
+          mma_commit(bar_kv_empty(slot));
+          mma_commit(bar(kBarPEmpty + pb));
+          ++n;
+        }
         if (!ok) break;
-        const uint32_t pb = j & 1;
-        if (!mbar_wait(bar_p_full(pb), (j >> 1) & 1, kRoleMma)) { ok = false; break; }
-        const uint32_t slot = n % C::kStages;
-        if (!mbar_wait(bar_kv_full(slot), (n / C::kStages) & 1, kRoleMma)) { ok = false; break; }
-        tc_fence_after();
-        const uint64_t v_desc = smem_desc(sKV + slot * C::kTileBytes, 16, C::kSBO, C::kSwizzle);
-#pragma unroll
-        for (int kk = 0; kk < kBN / 32; ++kk)  // 32 keys per MMA: 8 TMEM columns of P, 32 V rows
-          mma_i8_ts(tmem + kColO, tmem + kColP + pb * 32 + kk * 8, v_desc + ((32u * D * kk) >> 4),
-                    idesc_pv, (j > 0 || kk > 0) ? 1u : 0u);
-        mma_commit(bar_kv_empty(slot));
-        mma_commit(bar_p_empty(pb));
-        ++n;
+        mma_commit(bar(kBarQEmpty + qb));  // every MMA that read this Q buffer
+        mma_commit(bar(kBarOFull));
       }
-      if (ok) mma_commit(bar_o_full);
       // every MMA this thread issued is complete before TMEM is released
-      mma_commit(bar_drain);
-      mbar_wait(bar_drain, 0, kRoleMma);
+      mma_commit(bar(kBarDrain));
+      mbar_wait(bar(kBarDrain), 0, kRoleMma);
     }
   }
 
   tc_fence_before();
   __syncthreads();
-  if (warp == 5) {
+  if (warp == kMmaWarp) {
     tc_fence_after();
     tmem_dealloc(tmem, kTmemCols);
   }
