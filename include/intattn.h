@@ -113,6 +113,32 @@ int intattn_decode(const int8_t *q, const int8_t *k_cache, const int8_t *v_cache
                    float clip_c, int8_t *out, void *workspace, size_t workspace_bytes,
                    intattn_stream_t stream);
 
+/* Capacity in bytes of the library's static decode scratch (48 MiB). */
+#define INTATTN_STATIC_SCRATCH_BYTES (48u * 1024u * 1024u)
+
+/* Decode without any allocation: intattn_decode with the scratch taken from a
+ * fixed array inside this library instead of a caller workspace.  The paper
+ * has no counterpart; it exists for callers that cannot allocate device
+ * memory on their call path -- for example a plugin that runs under a host
+ * framework's own caching allocator and has no workspace to hand over, or a
+ * latency-bound serving loop that must not call cudaMalloc (which can
+ * synchronise the device and take allocator locks).
+ *   Arguments, layout, result and return codes: as intattn_decode.
+ *   Limit: intattn_decode_workspace_size(B, H, Lk, d) must not exceed
+ *   INTATTN_STATIC_SCRATCH_BYTES, else INTATTN_ERR_WORKSPACE (nothing runs).
+ *   The array (one per GPU that loads the library, kept until exit) is
+ *   shared by every call and keeps the previous call's contents; the kernels
+ *   overwrite what they read and clear their own counters, so no clearing is
+ *   needed, but two calls on one device that overlap on the GPU (for
+ *   example on two streams) race on it: order them on one stream.
+ *   The first call on each device looks up the array's device address
+ *   (cudaGetSymbolAddress) with that device current; make that first call
+ *   before any stream capture.  Calls no cudaMalloc, cudaFree or allocating
+ *   library routine. */
+int intattn_decode_static_scratch(const int8_t *q, const int8_t *k_cache, const int8_t *v_cache,
+                                  const intattn_scales_t *scales, int B, int H, int Lk, int Lmax, int d,
+                                  float clip_c, int8_t *out, intattn_stream_t stream);
+
 /* Synchronises `stream`, then returns and clears the device error word that a
  * kernel sets when one of its bounded waits runs out (INTATTN_ERR_TIMEOUT), or
  * INTATTN_OK.  INTATTN_ERR_CUDA if the synchronisation itself fails. */

@@ -22,7 +22,8 @@ MAX_HEADS = 128
 
 # every function declared in include/intattn.h
 EXPORTED = ("intattn_derive_params", "intattn_forward", "intattn_decode_workspace_size",
-            "intattn_decode", "intattn_device_error", "intattn_strerror")
+            "intattn_decode", "intattn_decode_static_scratch", "intattn_device_error",
+            "intattn_strerror")
 
 
 class IntAttnError(RuntimeError):
@@ -84,6 +85,8 @@ def lib() -> ctypes.CDLL:
         L.intattn_decode_workspace_size.restype = ctypes.c_size_t
         L.intattn_decode.argtypes = [vp, vp, vp, ctypes.POINTER(_Scales), i32, i32, i32, i32, i32,
                                      f32, vp, vp, ctypes.c_size_t, vp]
+        L.intattn_decode_static_scratch.argtypes = [vp, vp, vp, ctypes.POINTER(_Scales), i32, i32, i32,
+                                                    i32, i32, f32, vp, vp]
         L.intattn_device_error.argtypes = [vp]
         L.intattn_strerror.argtypes = [i32]
         L.intattn_strerror.restype = ctypes.c_char_p

@@ -197,6 +197,33 @@ int decode_launch(const DecodeArgs& a, cudaStream_t stream) {
   return note_launch(cudaGetLastError());
 }
 
+// ------------------------------------------------ static decode scratch
+// Decode scratch for callers that cannot allocate device memory (see
+// intattn_decode_static_scratch in intattn.h).  One array per GPU that loads
+// this library, held until the process exits.  Host code must not pass the
+// array's name to a kernel: on the host it is only a stand-in for the
+// symbol, so its device address is looked up once per device below.
+static __device__ __align__(256) unsigned char g_decode_scratch[INTATTN_STATIC_SCRATCH_BYTES];
+
+std::mutex g_scratch_mutex;
+void* g_scratch_ptr[64] = {};
+
+// Device address of g_decode_scratch on the current device (set up on the
+// first call per device, with that device current).
+int static_scratch_address(void** out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return INTATTN_ERR_CUDA;
+  std::lock_guard<std::mutex> lock(g_scratch_mutex);
+  if (g_scratch_ptr[dev] == nullptr) {
+    void* p = nullptr;
+    const cudaError_t e = cudaGetSymbolAddress(&p, g_decode_scratch);
+    if (e != cudaSuccess || p == nullptr) return note_launch(e == cudaSuccess ? cudaErrorInvalidSymbol : e);
+    g_scratch_ptr[dev] = p;
+  }
+  *out = g_scratch_ptr[dev];
+  return INTATTN_OK;
+}
+
 }  // namespace
 
 extern "C" {
@@ -293,6 +320,47 @@ int intattn_decode(const int8_t* q, const int8_t* k_cache, const int8_t* v_cache
   a.ws_max = reinterpret_cast<int32_t*>(ws + L.off_max);
   a.ws_part = reinterpret_cast<int32_t*>(ws + L.off_part);
   a.ws_cnt = reinterpret_cast<uint32_t*>(ws + L.off_cnt);
+  a.BH = static_cast<int32_t>(BH);
+  a.H = H;
+  a.Lk = Lk;
+  a.Lmax = Lmax;
+  a.nsplit = L.nsplit;
+  a.chunk = intattn::decode::kChunk;
+  a.per_head = scales->per_head ? 1 : 0;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  return d == 64 ? decode_launch<64>(a, st) : decode_launch<128>(a, st);
+}
+
+int intattn_decode_static_scratch(const int8_t* q, const int8_t* k_cache, const int8_t* v_cache,
+                                  const intattn_scales_t* scales, int B, int H, int Lk, int Lmax, int d,
+                                  float clip_c, int8_t* out, intattn_stream_t stream) {
+  // same checks and kernels as intattn_decode; only the scratch differs
+  if (B < 0 || H <= 0 || Lk < 1 || Lk > 65535 || Lmax < Lk) return INTATTN_ERR_INVALID_ARG;
+  if (d != 64 && d != 128) return INTATTN_ERR_UNSUPPORTED;
+  if (!scales) return INTATTN_ERR_INVALID_ARG;
+  DecodeArgs a;
+  std::memset(&a, 0, sizeof(a));
+  int rc = derive(scales, H, d, clip_c, a.lut, a.hp, INTATTN_MAX_HEADS);
+  if (rc) return rc;
+  const long long BH = static_cast<long long>(B) * H;
+  if (BH == 0) return INTATTN_OK;
+  if (BH > 65535) return INTATTN_ERR_UNSUPPORTED;
+  if (!q || !k_cache || !v_cache || !out) return INTATTN_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k_cache) || !aligned16(v_cache)) return INTATTN_ERR_UNSUPPORTED;
+  const DecodeLayout L = decode_layout(BH, Lk, d);
+  if (L.total > static_cast<size_t>(INTATTN_STATIC_SCRATCH_BYTES)) return INTATTN_ERR_WORKSPACE;
+  void* scratch = nullptr;
+  rc = static_scratch_address(&scratch);
+  if (rc) return rc;
+  char* ws = static_cast<char*>(scratch);
+  a.q = q;
+  a.k = k_cache;
+  a.v = v_cache;
+  a.out = out;
+  a.ws_s = reinterpret_cast<int32_t*>(ws + L.off_s);
+  a.ws_max = reinterpret_cast<int32_t*>(ws + L.off_max);
+  a.ws_part = reinterpret_cast<int32_t*>(ws + L.off_part);
+  a.ws_cnt = reinterpret_cast<uint32_t*>(ws + L.off_cnt);  // zeroed by the first kernel of each call
   a.BH = static_cast<int32_t>(BH);
   a.H = H;
   a.Lk = Lk;
