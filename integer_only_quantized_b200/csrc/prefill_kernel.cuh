@@ -61,10 +61,15 @@ namespace prefill {
 
 constexpr int kBM = 128;                  // query rows per tile (MMA M)
 constexpr int kBN = 128;                  // keys per S tile (QK MMA N)
-constexpr int kGroups = 4;                // partial results per query row (team x half)
-constexpr int kCols = kBN / 2;            // S columns per thread and tile (a key half)
-constexpr int kSoftWarps = 16;            // two teams of eight
-constexpr int kTeamWarps = 8;
+#ifndef INTATTN_SOFTMAX_TEAMS
+#define INTATTN_SOFTMAX_TEAMS 2
+#endif
+constexpr int kTeams = INTATTN_SOFTMAX_TEAMS;  // teams taking alternate S tiles
+constexpr int kSoftWarps = 16;
+constexpr int kTeamWarps = kSoftWarps / kTeams;
+constexpr int kColGroups = kTeamWarps / 4;  // column groups per team
+constexpr int kCols = kBN / kColGroups;     // S columns per thread and tile
+constexpr int kGroups = kTeams * kColGroups;  // partial results per query row (= 4)
 constexpr int kProducerWarp = kSoftWarps;
 constexpr int kMmaWarp = kSoftWarps + 1;
 constexpr int kThreads = 32 * (kSoftWarps + 2);  // 576
@@ -77,7 +82,7 @@ constexpr int kPBufs = 4;
 constexpr uint32_t kNbAll = 1;   // all softmax warps
 constexpr uint32_t kNbTeam = 2;  // + team: the warps of one team
 
-static_assert(kCols == 64, "two 32-column TMEM loads per thread and tile");
+static_assert(kGroups == 4 && kCols % 32 == 0, "4 partials per row, whole 32-column TMEM loads");
 
 enum Role : unsigned { kRoleSoftmax = 1, kRoleProducer = 2, kRoleMma = 3 };
 
@@ -213,9 +218,9 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_kernel(const __grid_const
   if (warp < kSoftWarps) {
     // ======================= IndexSoftmax warps =======================
     const int quad = warp & 3;
-    const int half = (warp >> 2) & 1;
-    const int team = warp >> 3;
-    const int grp = team * 2 + half;  // slot of this thread's partial results
+    const int half = (warp >> 2) % kColGroups;  // column group within the team
+    const int team = warp / kTeamWarps;
+    const int grp = team * kColGroups + half;   // slot of this thread's partial results
     const int r = quad * 32 + lane;   // query row within the tile == TMEM lane
     const uint32_t tlane = tmem + (static_cast<uint32_t>(quad * 32) << 16);
     const uint32_t trow = tlane + half * kCols;
@@ -242,21 +247,22 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_kernel(const __grid_const
     };
     // S tile `idx` (running index; this team's tiles have idx % 2 == team,
     // which is also the buffer) -> registers; released as soon as it is loaded
-    auto load_s = [&](uint32_t idx, uint32_t (&v)[64]) {
+    auto load_s = [&](uint32_t idx, uint32_t (&v)[kCols]) {
       const uint32_t buf = idx & 1;
       if (!team_wait(bar(kBarSFull + buf), (idx >> 1) & 1)) return false;
       tc_fence_after();
-      uint32_t (&v0)[32] = *reinterpret_cast<uint32_t(*)[32]>(&v[0]);
-      uint32_t (&v1)[32] = *reinterpret_cast<uint32_t(*)[32]>(&v[32]);
-      tmem_ld32(trow + kColS + buf * kBN, v0);
-      tmem_ld32(trow + kColS + buf * kBN + 32, v1);
+#pragma unroll
+      for (int c = 0; c < kCols / 32; ++c)
+        tmem_ld32(trow + kColS + buf * kBN + 32 * c, *reinterpret_cast<uint32_t(*)[32]>(&v[32 * c]));
       tmem_wait_ld();
       tc_fence_before();
       arrive_warp(bar(kBarSEmpty + buf));
       return true;
     };
     // first tile of a pass of nkt tiles that belongs to this team
-    auto first_j = [&](uint32_t s0) { return static_cast<int>((static_cast<uint32_t>(team) - s0) & 1u); };
+    auto first_j = [&](uint32_t s0) {
+      return kTeams == 1 ? 0 : static_cast<int>((static_cast<uint32_t>(team) - s0) & 1u);
+    };
 
     for (int it = 0; ok; ++it) {
       const int L = tile_index(it, blockIdx.x, gridDim.x);
@@ -269,19 +275,19 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_kernel(const __grid_const
         const int last = (j + 1) * kBN - 1;
         return last < args.Lk && (!args.causal || last <= T.q0 + off);
       };
-      // keys of this thread's 64-key segment of tile j that are visible: a prefix
+      // keys of this thread's segment of tile j that are visible: a prefix
       const int key_lim = args.causal ? min(args.Lk, row_limit + 1) : args.Lk;
       auto nvalid = [&](int j) { return min(max(key_lim - (j * kBN + half * kCols), 0), kCols); };
 
       // ---- pass A: row max over valid keys ----
       int32_t m = INT_MIN;
-      for (int j = first_j(sc); j < T.nkt; j += 2) {
-        uint32_t v[64];
+      for (int j = first_j(sc); j < T.nkt; j += kTeams) {
+        uint32_t v[kCols];
         if (!load_s(sc + j, v)) { ok = false; break; }
         int32_t m4[4] = {INT_MIN, INT_MIN, INT_MIN, INT_MIN};
         if (tile_full(j)) {
 #pragma unroll
-          for (int k = 0; k < 64; k += 8) {
+          for (int k = 0; k < kCols; k += 8) {
             m4[0] = __vimax3_s32(m4[0], static_cast<int32_t>(v[k + 0]), static_cast<int32_t>(v[k + 1]));
             m4[1] = __vimax3_s32(m4[1], static_cast<int32_t>(v[k + 2]), static_cast<int32_t>(v[k + 3]));
             m4[2] = __vimax3_s32(m4[2], static_cast<int32_t>(v[k + 4]), static_cast<int32_t>(v[k + 5]));
@@ -290,7 +296,7 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_kernel(const __grid_const
         } else {
           const int nv = nvalid(j);
 #pragma unroll
-          for (int k = 0; k < 64; ++k) m4[k & 3] = imax(m4[k & 3], k < nv ? static_cast<int32_t>(v[k]) : INT_MIN);
+          for (int k = 0; k < kCols; ++k) m4[k & 3] = imax(m4[k & 3], k < nv ? static_cast<int32_t>(v[k]) : INT_MIN);
         }
         m = imax(m, imax(imax(m4[0], m4[1]), imax(m4[2], m4[3])));
       }
@@ -325,18 +331,18 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_kernel(const __grid_const
 
       // ---- pass B: Z = sum of pseudo-exponentials ----
       int32_t Z = 0;
-      for (int j = first_j(sc); j < T.nkt; j += 2) {
-        uint32_t v[64];
+      for (int j = first_j(sc); j < T.nkt; j += kTeams) {
+        uint32_t v[kCols];
         if (!load_s(sc + j, v)) { ok = false; break; }
         float z4[4] = {0.f, 0.f, 0.f, 0.f};
         if (tile_full(j)) {
 #pragma unroll
-          for (int k = 0; k < 64; ++k)
+          for (int k = 0; k < kCols; ++k)
             z4[k & 3] += __int_as_float(__shfl_sync(0xffffffffu, lut_lane, static_cast<int>(idx_bits(v[k]))));
         } else {
           const int nv = nvalid(j);
 #pragma unroll
-          for (int k = 0; k < 64; ++k) {
+          for (int k = 0; k < kCols; ++k) {
             const uint32_t ib = k < nv ? idx_bits(v[k]) : kMaskedBits;
             z4[k & 3] += __int_as_float(__shfl_sync(0xffffffffu, lut_lane, static_cast<int>(ib)));
           }
@@ -367,16 +373,16 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_kernel(const __grid_const
       all_sync(true);  // the table is complete
 
       // ---- pass C: P tiles into TMEM for the P.V MMAs ----
-      for (int j = first_j(sc); j < T.nkt; j += 2) {
+      for (int j = first_j(sc); j < T.nkt; j += kTeams) {
         const uint32_t pi = pc + j;  // running P index of this tile
         const uint32_t pb = pi & (kPBufs - 1);
         if (!team_wait(bar(kBarPEmpty + pb), ((pi / kPBufs) & 1) ^ 1)) { ok = false; break; }
-        uint32_t v[64];
+        uint32_t v[kCols];
         if (!load_s(sc + j, v)) { ok = false; break; }
-        uint32_t pw[16];
+        uint32_t pw[kCols / 4];
         if (tile_full(j)) {
 #pragma unroll
-          for (int q = 0; q < 16; ++q) {
+          for (int q = 0; q < kCols / 4; ++q) {
             uint32_t p[4];
 #pragma unroll
             for (int b = 0; b < 4; ++b) p[b] = lds_u32(idx_bits(v[q * 4 + b]) * 512u + prow);
@@ -385,7 +391,7 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_kernel(const __grid_const
         } else {
           const int nv = nvalid(j);
 #pragma unroll
-          for (int q = 0; q < 16; ++q) {
+          for (int q = 0; q < kCols / 4; ++q) {
             uint32_t p[4];
 #pragma unroll
             for (int b = 0; b < 4; ++b) {
@@ -396,7 +402,11 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_kernel(const __grid_const
             pw[q] = pack4(p[0], p[1], p[2], p[3]);
           }
         }
-        tmem_st16(tlane + kColP + pb * 32 + half * 16, pw);
+        if constexpr (kCols == 64) {
+          tmem_st16(tlane + kColP + pb * 32 + half * 16, *reinterpret_cast<const uint32_t(*)[16]>(pw));
+        } else {
+          tmem_st8(tlane + kColP + pb * 32 + half * 8, *reinterpret_cast<const uint32_t(*)[8]>(pw));
+        }
         tmem_wait_st();
         tc_fence_before();
         arrive_warp(bar(kBarPFull + pb));
@@ -436,122 +446,123 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_kernel(const __grid_const
     }
   } else if (warp == kProducerWarp) {
     // ============================ TMA producer ============================
+    // The whole warp runs this loop on uniform values; one elected lane issues.
     if (lane == 0) {
       tma_prefetch_desc(&args.tm_q);
       tma_prefetch_desc(&args.tm_k);
       tma_prefetch_desc(&args.tm_v);
-      uint32_t n = 0;   // K/V loads issued, in the MMA warp's consumption order
-      uint32_t nq = 0;  // Q loads issued
-      bool ok = true;
-      auto load = [&](const CUtensorMap* tm, int j, int bh) {
-        if (!ok) return;
-        const uint32_t slot = n % C::kStages;
-        const uint32_t use = n / C::kStages;
-        if (!mbar_wait(bar_kv_empty(slot), (use & 1) ^ 1, kRoleProducer)) { ok = false; return; }
-        mbar_arrive_expect_tx(bar_kv_full(slot), C::kTileBytes);
-        tma_load_3d(sKV + slot * C::kTileBytes, tm, bar_kv_full(slot), 0, j * kBN, bh);
-        ++n;
-      };
-      for (int it = 0; ok; ++it) {
-        const int L = tile_index(it, blockIdx.x, gridDim.x);
-        if (L >= args.n_tiles) break;
-        const Tile T = tile_of(args, L);
-        const uint32_t qb = nq & 1;
-        if (!mbar_wait(bar(kBarQEmpty + qb), ((nq >> 1) & 1) ^ 1, kRoleProducer)) { ok = false; break; }
-        mbar_arrive_expect_tx(bar(kBarQFull + qb), C::kQBytes);
-        tma_load_3d(sQ(qb), &args.tm_q, bar(kBarQFull + qb), 0, T.q0, T.bh);
-        ++nq;
-        for (int pass = 0; pass < 2; ++pass)
-          for (int j = 0; j < T.nkt; ++j) load(&args.tm_k, j, T.bh);
-        load(&args.tm_k, 0, T.bh);
-        if (T.nkt > 1) load(&args.tm_k, 1, T.bh);
-        for (int j = 0; j < T.nkt; ++j) {
-          if (j + 2 < T.nkt) load(&args.tm_k, j + 2, T.bh);
-          load(&args.tm_v, j, T.bh);
-        }
+    }
+    uint32_t n = 0;   // K/V loads issued, in the MMA warp's consumption order
+    uint32_t nq = 0;  // Q loads issued
+    bool ok = true;
+    auto load = [&](const CUtensorMap* tm, int j, int bh) {
+      if (!ok) return;
+      const uint32_t slot = n % C::kStages;
+      const uint32_t use = n / C::kStages;
+      if (!mbar_wait_warp(bar_kv_empty(slot), (use & 1) ^ 1, kRoleProducer)) { ok = false; return; }
+      tma_load_3d_elect(sKV + slot * C::kTileBytes, tm, bar_kv_full(slot), C::kTileBytes, 0, j * kBN, bh);
+      ++n;
+    };
+    for (int it = 0; ok; ++it) {
+      const int L = tile_index(it, blockIdx.x, gridDim.x);
+      if (L >= args.n_tiles) break;
+      const Tile T = tile_of(args, L);
+      const uint32_t qb = nq & 1;
+      if (!mbar_wait_warp(bar(kBarQEmpty + qb), ((nq >> 1) & 1) ^ 1, kRoleProducer)) { ok = false; break; }
+      tma_load_3d_elect(sQ(qb), &args.tm_q, bar(kBarQFull + qb), C::kQBytes, 0, T.q0, T.bh);
+      ++nq;
+      for (int pass = 0; pass < 2; ++pass)
+        for (int j = 0; j < T.nkt; ++j) load(&args.tm_k, j, T.bh);
+      load(&args.tm_k, 0, T.bh);
+      if (T.nkt > 1) load(&args.tm_k, 1, T.bh);
+      for (int j = 0; j < T.nkt; ++j) {
+        if (j + 2 < T.nkt) load(&args.tm_k, j + 2, T.bh);
+        load(&args.tm_v, j, T.bh);
       }
-      // never leave with a copy in flight: wait for the last load of each slot
-      for (uint32_t slot = 0; slot < static_cast<uint32_t>(C::kStages); ++slot) {
-        if (n > slot) {
-          const uint32_t uses = (n - slot - 1) / C::kStages + 1;
-          mbar_wait(bar_kv_full(slot), (uses - 1) & 1, kRoleProducer);
-        }
+    }
+    // never leave with a copy in flight: wait for the last load of each slot
+    for (uint32_t slot = 0; slot < static_cast<uint32_t>(C::kStages); ++slot) {
+      if (n > slot) {
+        const uint32_t uses = (n - slot - 1) / C::kStages + 1;
+        mbar_wait_warp(bar_kv_full(slot), (uses - 1) & 1, kRoleProducer);
       }
-      for (uint32_t i = 0; i < 2 && i < nq; ++i) {
-        const uint32_t last = nq - 1 - i;  // the last load of each Q buffer
-        mbar_wait(bar(kBarQFull + (last & 1)), (last >> 1) & 1, kRoleProducer);
-      }
+    }
+    for (uint32_t i = 0; i < 2 && i < nq; ++i) {
+      const uint32_t last = nq - 1 - i;  // the last load of each Q buffer
+      mbar_wait_warp(bar(kBarQFull + (last & 1)), (last >> 1) & 1, kRoleProducer);
     }
   } else {
     // ============================= MMA issuer =============================
-    if (lane == 0) {
-      constexpr uint32_t idesc_qk = idesc_i8(kBM, kBN, 1, 1, 0);  // s8 x s8, K-major B
-      constexpr uint32_t idesc_pv = idesc_i8(kBM, D, 0, 1, 1);    // u8 x s8, N-major B
-      bool ok = true;
-      uint32_t n = 0;   // K/V tiles consumed
-      uint32_t sc = 0;  // S tiles produced
-      uint32_t pc = 0;  // P tiles consumed
-      for (int it = 0; ok; ++it) {
-        const int L = tile_index(it, blockIdx.x, gridDim.x);
-        if (L >= args.n_tiles) break;
-        const Tile T = tile_of(args, L);
-        const uint32_t qb = it & 1;
-        if (!mbar_wait(bar(kBarQFull + qb), (it >> 1) & 1, kRoleMma)) { ok = false; break; }
-        const uint64_t q_desc = smem_desc(sQ(qb), 16, C::kSBO, C::kSwizzle);
-        auto issue_qk = [&]() {
-          if (!ok) return;
-          const uint32_t buf = sc & 1;
-          const uint32_t slot = n % C::kStages;
-          if (!mbar_wait2(bar(kBarSEmpty + buf), ((sc >> 1) & 1) ^ 1, bar_kv_full(slot), (n / C::kStages) & 1,
-                          kRoleMma)) {
-            ok = false;
-            return;
-          }
-          tc_fence_after();
-          const uint64_t k_desc = smem_desc(sKV + slot * C::kTileBytes, 16, C::kSBO, C::kSwizzle);
-#pragma unroll
-          for (int kk = 0; kk < D / 32; ++kk)  // K = 32 bytes per MMA: advance 32 B
-            mma_i8_ss(tmem + kColS + buf * kBN, q_desc + 2 * kk, k_desc + 2 * kk, idesc_qk, kk > 0);
-          mma_commit(bar_kv_empty(slot));
-          mma_commit(bar(kBarSFull + buf));
-          ++n;
-          ++sc;
-        };
-        for (int t = 0; t < 2 * T.nkt; ++t) issue_qk();  // passes A and B
-        // pass C: S tile j+2 reuses the buffer of tile j, which the softmax
-        // warps release right after loading it, so QK(j+2) goes before P.V(j)
-        issue_qk();
-        if (T.nkt > 1) issue_qk();
-        for (int j = 0; ok && j < T.nkt; ++j, ++pc) {
-          if (j + 2 < T.nkt) issue_qk();
-          if (!ok) break;
-          // O of the previous tile must have been read before it is overwritten
-          if (j == 0 && !mbar_wait(bar(kBarOEmpty), (it & 1) ^ 1, kRoleMma)) { ok = false; break; }
-          const uint32_t pb = pc & (kPBufs - 1);
-          const uint32_t slot = n % C::kStages;
-          if (!mbar_wait2(bar(kBarPFull + pb), (pc / kPBufs) & 1, bar_kv_full(slot), (n / C::kStages) & 1,
-                          kRoleMma)) {
-            ok = false;
-            break;
-          }
-          tc_fence_after();
-          const uint64_t v_desc = smem_desc(sKV + slot * C::kTileBytes, 16, C::kSBO, C::kSwizzle);
-#pragma unroll
-          for (int kk = 0; kk < kBN / 32; ++kk)  // 32 keys per MMA: 8 TMEM columns of P, 32 V rows
-            mma_i8_ts(tmem + kColO, tmem + kColP + pb * 32 + kk * 8, v_desc + ((32u * D * kk) >> 4),
-                      idesc_pv, (j > 0 || kk > 0) ? 1u : 0u);
-          mma_commit(bar_kv_empty(slot));
-          mma_commit(bar(kBarPEmpty + pb));
-          ++n;
+    // The whole warp runs this loop on uniform values (descriptors stay in
+    // uniform registers); one elected lane issues each tcgen05 instruction.
+    constexpr uint32_t idesc_qk = idesc_i8(kBM, kBN, 1, 1, 0);  // s8 x s8, K-major B
+    constexpr uint32_t idesc_pv = idesc_i8(kBM, D, 0, 1, 1);    // u8 x s8, N-major B
+    const uint64_t kv_desc0 = smem_desc(sKV, 16, C::kSBO, C::kSwizzle);
+    constexpr uint32_t kSlotDesc = C::kTileBytes >> 4;  // descriptor step between ring slots
+    bool ok = true;
+    uint32_t n = 0;   // K/V tiles consumed
+    uint32_t sc = 0;  // S tiles produced
+    uint32_t pc = 0;  // P tiles consumed
+    for (int it = 0; ok; ++it) {
+      const int L = tile_index(it, blockIdx.x, gridDim.x);
+      if (L >= args.n_tiles) break;
+      const Tile T = tile_of(args, L);
+      const uint32_t qb = it & 1;
+      if (!mbar_wait_warp(bar(kBarQFull + qb), (it >> 1) & 1, kRoleMma)) { ok = false; break; }
+      const uint64_t q_desc = smem_desc(sQ(qb), 16, C::kSBO, C::kSwizzle);
+      auto issue_qk = [&]() {
+        if (!ok) return;
+        const uint32_t buf = sc & 1;
+        const uint32_t slot = n % C::kStages;
+        if (!mbar_wait_warp(bar(kBarSEmpty + buf), ((sc >> 1) & 1) ^ 1, kRoleMma) ||
+            !mbar_wait_warp(bar_kv_full(slot), (n / C::kStages) & 1, kRoleMma)) {
+          ok = false;
+          return;
         }
+        tc_fence_after();
+        const uint64_t k_desc = kv_desc0 + slot * kSlotDesc;
+#pragma unroll
+        for (int kk = 0; kk < D / 32; ++kk)  // K = 32 bytes per MMA: advance 32 B
+          mma_i8_ss_elect(tmem + kColS + buf * kBN, q_desc + 2 * kk, k_desc + 2 * kk, idesc_qk, kk > 0);
+        mma_commit_elect(bar_kv_empty(slot));
+        mma_commit_elect(bar(kBarSFull + buf));
+        ++n;
+        ++sc;
+      };
+      for (int t = 0; t < 2 * T.nkt; ++t) issue_qk();  // passes A and B
+      // pass C: S tile j+2 reuses the buffer of tile j, which the softmax
+      // warps release right after loading it, so QK(j+2) goes before P.V(j)
+      issue_qk();
+      if (T.nkt > 1) issue_qk();
+      for (int j = 0; ok && j < T.nkt; ++j, ++pc) {
+        if (j + 2 < T.nkt) issue_qk();
         if (!ok) break;
-        mma_commit(bar(kBarQEmpty + qb));  // every MMA that read this Q buffer
-        mma_commit(bar(kBarOFull));
+        // O of the previous tile must have been read before it is overwritten
+        if (j == 0 && !mbar_wait_warp(bar(kBarOEmpty), (it & 1) ^ 1, kRoleMma)) { ok = false; break; }
+        const uint32_t pb = pc & (kPBufs - 1);
+        const uint32_t slot = n % C::kStages;
+        if (!mbar_wait_warp(bar(kBarPFull + pb), (pc / kPBufs) & 1, kRoleMma) ||
+            !mbar_wait_warp(bar_kv_full(slot), (n / C::kStages) & 1, kRoleMma)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        const uint64_t v_desc = kv_desc0 + slot * kSlotDesc;
+#pragma unroll
+        for (int kk = 0; kk < kBN / 32; ++kk)  // 32 keys per MMA: 8 TMEM columns of P, 32 V rows
+          mma_i8_ts_elect(tmem + kColO, tmem + kColP + pb * 32 + kk * 8, v_desc + ((32u * D * kk) >> 4),
+                          idesc_pv, (j > 0 || kk > 0) ? 1u : 0u);
+        mma_commit_elect(bar_kv_empty(slot));
+        mma_commit_elect(bar(kBarPEmpty + pb));
+        ++n;
       }
-      // every MMA this thread issued is complete before TMEM is released
-      mma_commit(bar(kBarDrain));
-      mbar_wait(bar(kBarDrain), 0, kRoleMma);
+      if (!ok) break;
+      mma_commit_elect(bar(kBarQEmpty + qb));  // every MMA that read this Q buffer
+      mma_commit_elect(bar(kBarOFull));
     }
+    // every MMA this warp issued is complete before TMEM is released
+    mma_commit_elect(bar(kBarDrain));
+    mbar_wait_warp(bar(kBarDrain), 0, kRoleMma);
   }
 
   tc_fence_before();
