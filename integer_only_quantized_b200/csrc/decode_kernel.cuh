@@ -2,16 +2,17 @@
 //
 // Same integer definition as the prefill path with Lq = 1 and no mask.  The
 // work is an HBM stream of the K and V rows (2*Lk*d bytes per (b, h)), so it
-// is split over key chunks to fill every SM, in two launches:
+// is split over key chunks to fill every SM, in three launches:
 //   decode_qk  per (b, h, chunk): S_j = q.K_j with 16-byte vector loads and
 //              dp4a; S to the workspace, chunk max to the workspace.
-//   decode_pv  per (b, h, chunk): m = max of the chunk maxima; Z over all Lk
-//              scores of the row (16 KB from L2 per (b, h)); R and the u8
-//              probabilities of this chunk; V chunk streamed with 16-byte
-//              loads, P.V by dp4a after a 4x4 byte transpose; int32 partial
-//              sums to the workspace.  The last CTA of a (b, h) (atomic
-//              ticket) adds the partials and requantises.  Integer addition
-//              is associative, so the result does not depend on the order.
+//   decode_z   per (b, h): m = max of the chunk maxima, Z over all Lk scores
+//              (from L2), the reciprocal R; (m, R) to the workspace.
+//   decode_pv  per (b, h, chunk): the u8 probabilities of this chunk from
+//              (m, R); V chunk streamed with 16-byte loads, P.V by dp4a after
+//              a 4x4 byte transpose; int32 partial sums to the workspace.
+//              The last CTA of a (b, h) (atomic ticket) adds the partials and
+//              requantises.  Integer addition is associative, so the result
+//              does not depend on the order.
 #pragma once
 #include <climits>
 #include <cstdint>
@@ -26,11 +27,12 @@ struct DecodeArgs {
   const int8_t* k;   // [BH, Lmax, d]
   const int8_t* v;   // [BH, Lmax, d]
   int8_t* out;       // [BH, d]
-  int32_t* ws_s;     // [BH, Lk]          scores
+  int32_t* ws_s;     // [BH, ld_s]        scores (row stride ld_s = Lk rounded up to 4)
   int32_t* ws_max;   // [BH, nsplit]      chunk maxima
   int32_t* ws_part;  // [BH, nsplit, d]   partial P.V sums
   uint32_t* ws_cnt;  // [BH]              arrival tickets
-  int32_t BH, H, Lk, Lmax, nsplit, chunk, per_head;
+  int32_t* ws_mr;    // [BH, 2]           row max and reciprocal R
+  int32_t BH, H, Lk, Lmax, nsplit, chunk, per_head, ld_s;
   uint32_t lut[32];
   HeadParamsDev hp[INTATTN_MAX_HEADS];
 };
@@ -88,7 +90,7 @@ __global__ void __launch_bounds__(kThreads) decode_qk_kernel(const __grid_consta
 
   const uint4 qv = *reinterpret_cast<const uint4*>(a.q + static_cast<size_t>(bh) * D + piece * 16);
   const int8_t* kbase = a.k + static_cast<size_t>(bh) * a.Lmax * D + piece * 16;
-  int32_t* srow = a.ws_s + static_cast<size_t>(bh) * a.Lk;
+  int32_t* srow = a.ws_s + static_cast<size_t>(bh) * a.ld_s;
   int32_t mx = INT_MIN;
 
   for (int base = j0; base < j1; base += Lt::kRowsPerStep) {
@@ -163,28 +165,17 @@ __global__ void __launch_bounds__(kThreads) decode_qk_kernel(const __grid_consta
   }
 }
 
+// Row max, row sum Z and reciprocal R of one (b, h): one CTA per row.
 template <int D>
-__global__ void __launch_bounds__(kThreads) decode_pv_kernel(const __grid_constant__ DecodeArgs a) {
-  using Lt = Layout<D>;
-  const int bh = blockIdx.y;
-  const int sp = blockIdx.x;
-  const int j0 = sp * a.chunk;
-  const int j1 = min(a.Lk, j0 + a.chunk);
+__global__ void __launch_bounds__(kThreads) decode_z_kernel(const __grid_constant__ DecodeArgs a) {
+  const int bh = blockIdx.x;
   const int tid = threadIdx.x;
   const int lane = tid & 31;
   const int h = bh % a.H;
   const HeadParamsDev hp = a.hp[a.per_head ? h : 0];
-
   __shared__ uint32_t lut_s[32];
-  __shared__ uint32_t ptab_s[32];
   __shared__ int32_t red[kThreads / 32];
-  __shared__ uint32_t pk[kChunk / 4];              // u8 probabilities of this chunk
-  __shared__ int32_t part[kThreads * 16];          // per-thread partial sums
-  __shared__ int last_flag;
-
   if (tid < 32) lut_s[tid] = a.lut[tid];
-
-  // row max from the chunk maxima
   int32_t m = INT_MIN;
   for (int i = 0; i < a.nsplit; ++i) m = imax32(m, __ldcg(a.ws_max + static_cast<size_t>(bh) * a.nsplit + i));
   const long long lo64 = static_cast<long long>(m) - hp.D;
@@ -193,25 +184,63 @@ __global__ void __launch_bounds__(kThreads) decode_pv_kernel(const __grid_consta
   const uint32_t sh = static_cast<uint32_t>(hp.s);
   const uint32_t Cm = static_cast<uint32_t>(m) * Mu + (1u << (sh - 1));
   __syncthreads();
-
-  // Z over the whole row
-  const int32_t* srow = a.ws_s + static_cast<size_t>(bh) * a.Lk;
+  // idx = (min(m - S, D) M + 2^(s-1)) >> s as (Cm - max(S, m - D) M) >> s in
+  // wrapping 32-bit arithmetic (the true value lies in [0, 2^31))
+  // rows start on 16-byte boundaries (ld_s is a multiple of 4)
+  const int4* srow = reinterpret_cast<const int4*>(a.ws_s + static_cast<size_t>(bh) * a.ld_s);
   int32_t z = 0;
-  for (int j = tid; j < a.Lk; j += kThreads) {
-    const int32_t t = imax32(__ldcg(srow + j), lo);
+  const int n4 = a.Lk / 4;
+  for (int i = tid; i < n4; i += kThreads) {
+    const int4 s4 = __ldcg(srow + i);
+    z += static_cast<int32_t>(lut_s[(Cm - static_cast<uint32_t>(imax32(s4.x, lo)) * Mu) >> sh]);
+    z += static_cast<int32_t>(lut_s[(Cm - static_cast<uint32_t>(imax32(s4.y, lo)) * Mu) >> sh]);
+    z += static_cast<int32_t>(lut_s[(Cm - static_cast<uint32_t>(imax32(s4.z, lo)) * Mu) >> sh]);
+    z += static_cast<int32_t>(lut_s[(Cm - static_cast<uint32_t>(imax32(s4.w, lo)) * Mu) >> sh]);
+  }
+  for (int j = 4 * n4 + tid; j < a.Lk; j += kThreads) {
+    const int32_t t = imax32(__ldcg(a.ws_s + static_cast<size_t>(bh) * a.ld_s + j), lo);
     z += static_cast<int32_t>(lut_s[(Cm - static_cast<uint32_t>(t) * Mu) >> sh]);
   }
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) z += __shfl_xor_sync(0xffffffffu, z, o);
   if (lane == 0) red[tid >> 5] = z;
   __syncthreads();
-  if (tid < 32) {
+  if (tid == 0) {
     int32_t Z = 0;
     for (int w = 0; w < kThreads / 32; ++w) Z += red[w];
     const unsigned long long R =
         ((255ull << 32) + static_cast<unsigned long long>(Z >> 1)) / static_cast<unsigned long long>(Z);
-    ptab_s[tid] = static_cast<uint32_t>((static_cast<unsigned long long>(lut_s[tid]) * R + (1ull << 31)) >> 32);
+    a.ws_mr[2 * bh] = m;
+    a.ws_mr[2 * bh + 1] = static_cast<int32_t>(R);
   }
+}
+
+template <int D>
+__global__ void __launch_bounds__(kThreads) decode_pv_kernel(const __grid_constant__ DecodeArgs a) {
+  using Lt = Layout<D>;
+  const int bh = blockIdx.y;
+  const int sp = blockIdx.x;
+  const int j0 = sp * a.chunk;
+  const int j1 = min(a.Lk, j0 + a.chunk);
+  const int tid = threadIdx.x;
+  const int h = bh % a.H;
+  const HeadParamsDev hp = a.hp[a.per_head ? h : 0];
+
+  __shared__ uint32_t ptab_s[32];
+  __shared__ uint32_t pk[kChunk / 4];              // u8 probabilities of this chunk
+  __shared__ int32_t part[kThreads * 16];          // per-thread partial sums
+  __shared__ int last_flag;
+
+  const int32_t m = __ldcg(a.ws_mr + 2 * bh);
+  const unsigned long long R = static_cast<uint32_t>(__ldcg(a.ws_mr + 2 * bh + 1));
+  if (tid < 32)
+    ptab_s[tid] = static_cast<uint32_t>((static_cast<unsigned long long>(a.lut[tid]) * R + (1ull << 31)) >> 32);
+  const long long lo64 = static_cast<long long>(m) - hp.D;
+  const int32_t lo = lo64 < INT_MIN ? INT_MIN : static_cast<int32_t>(lo64);
+  const uint32_t Mu = static_cast<uint32_t>(hp.M);
+  const uint32_t sh = static_cast<uint32_t>(hp.s);
+  const uint32_t Cm = static_cast<uint32_t>(m) * Mu + (1u << (sh - 1));
+  const int32_t* srow = a.ws_s + static_cast<size_t>(bh) * a.ld_s;
   __syncthreads();
 
   // u8 probabilities of this chunk, 4 per word (rows past j1 get 0)

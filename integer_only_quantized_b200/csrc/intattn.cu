@@ -170,8 +170,8 @@ int prefill_launch(const PrefillArgs& args, int grid, cudaStream_t stream) {
 }
 
 struct DecodeLayout {
-  int nsplit;
-  size_t off_s, off_max, off_part, off_cnt, total;
+  int nsplit, ld_s;
+  size_t off_s, off_max, off_part, off_cnt, off_mr, total;
 };
 
 size_t round256(size_t x) { return (x + 255) & ~size_t(255); }
@@ -180,10 +180,12 @@ DecodeLayout decode_layout(long long BH, int Lk, int d) {
   DecodeLayout L{};
   L.nsplit = (Lk + intattn::decode::kChunk - 1) / intattn::decode::kChunk;
   L.off_s = 0;
-  L.off_max = L.off_s + round256(static_cast<size_t>(BH) * Lk * 4);
+  L.ld_s = (Lk + 3) & ~3;  // 16-byte aligned score rows
+  L.off_max = L.off_s + round256(static_cast<size_t>(BH) * L.ld_s * 4);
   L.off_part = L.off_max + round256(static_cast<size_t>(BH) * L.nsplit * 4);
   L.off_cnt = L.off_part + round256(static_cast<size_t>(BH) * L.nsplit * d * 4);
-  L.total = L.off_cnt + round256(static_cast<size_t>(BH) * 4);
+  L.off_mr = L.off_cnt + round256(static_cast<size_t>(BH) * 4);
+  L.total = L.off_mr + round256(static_cast<size_t>(BH) * 8);
   return L;
 }
 
@@ -193,6 +195,9 @@ int decode_launch(const DecodeArgs& a, cudaStream_t stream) {
   intattn::decode::decode_qk_kernel<D><<<grid, intattn::decode::kThreads, 0, stream>>>(a);
   const int rc = note_launch(cudaGetLastError());
   if (rc != INTATTN_OK) return rc;
+  intattn::decode::decode_z_kernel<D><<<a.BH, intattn::decode::kThreads, 0, stream>>>(a);
+  const int rz = note_launch(cudaGetLastError());
+  if (rz != INTATTN_OK) return rz;
   intattn::decode::decode_pv_kernel<D><<<grid, intattn::decode::kThreads, 0, stream>>>(a);
   return note_launch(cudaGetLastError());
 }
@@ -320,11 +325,13 @@ int intattn_decode(const int8_t* q, const int8_t* k_cache, const int8_t* v_cache
   a.ws_max = reinterpret_cast<int32_t*>(ws + L.off_max);
   a.ws_part = reinterpret_cast<int32_t*>(ws + L.off_part);
   a.ws_cnt = reinterpret_cast<uint32_t*>(ws + L.off_cnt);
+  a.ws_mr = reinterpret_cast<int32_t*>(ws + L.off_mr);
   a.BH = static_cast<int32_t>(BH);
   a.H = H;
   a.Lk = Lk;
   a.Lmax = Lmax;
   a.nsplit = L.nsplit;
+  a.ld_s = L.ld_s;
   a.chunk = intattn::decode::kChunk;
   a.per_head = scales->per_head ? 1 : 0;
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
@@ -361,11 +368,13 @@ int intattn_decode_static_scratch(const int8_t* q, const int8_t* k_cache, const 
   a.ws_max = reinterpret_cast<int32_t*>(ws + L.off_max);
   a.ws_part = reinterpret_cast<int32_t*>(ws + L.off_part);
   a.ws_cnt = reinterpret_cast<uint32_t*>(ws + L.off_cnt);  // zeroed by the first kernel of each call
+  a.ws_mr = reinterpret_cast<int32_t*>(ws + L.off_mr);
   a.BH = static_cast<int32_t>(BH);
   a.H = H;
   a.Lk = Lk;
   a.Lmax = Lmax;
   a.nsplit = L.nsplit;
+  a.ld_s = L.ld_s;
   a.chunk = intattn::decode::kChunk;
   a.per_head = scales->per_head ? 1 : 0;
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
