@@ -245,18 +245,24 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_kernel(const __grid_const
       __syncwarp();
       if (lane == 0) mbar_arrive(b);
     };
-    // S tile `idx` (running index; this team's tiles have idx % 2 == team,
-    // which is also the buffer) -> registers; released as soon as it is loaded
-    auto load_s = [&](uint32_t idx, uint32_t (&v)[kCols]) {
+    // S tile `idx` in 32-column chunks: load chunk c, then body(v, c); the
+    // buffer is released after its last chunk is loaded, so only 32 scores
+    // per thread are live at a time.
+    auto walk_s = [&](uint32_t idx, auto&& body) {
       const uint32_t buf = idx & 1;
       if (!team_wait(bar(kBarSFull + buf), (idx >> 1) & 1)) return false;
       tc_fence_after();
 #pragma unroll
-      for (int c = 0; c < kCols / 32; ++c)
-        tmem_ld32(trow + kColS + buf * kBN + 32 * c, *reinterpret_cast<uint32_t(*)[32]>(&v[32 * c]));
-      tmem_wait_ld();
-      tc_fence_before();
-      arrive_warp(bar(kBarSEmpty + buf));
+      for (int c = 0; c < kCols / 32; ++c) {
+        uint32_t v[32];
+        tmem_ld32(trow + kColS + buf * kBN + 32 * c, v);
+        tmem_wait_ld();
+        if (c == kCols / 32 - 1) {
+          tc_fence_before();
+          arrive_warp(bar(kBarSEmpty + buf));
+        }
+        body(v, c);
+      }
       return true;
     };
     // first tile of a pass of nkt tiles that belongs to this team
@@ -282,22 +288,26 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_kernel(const __grid_const
       // ---- pass A: row max over valid keys ----
       int32_t m = INT_MIN;
       for (int j = first_j(sc); j < T.nkt; j += kTeams) {
-        uint32_t v[kCols];
-        if (!load_s(sc + j, v)) { ok = false; break; }
         int32_t m4[4] = {INT_MIN, INT_MIN, INT_MIN, INT_MIN};
-        if (tile_full(j)) {
+        const bool full = tile_full(j);
+        const int nv = nvalid(j);
+        const bool got = walk_s(sc + j, [&](const uint32_t (&v)[32], int c) {
+          if (full) {
 #pragma unroll
-          for (int k = 0; k < kCols; k += 8) {
-            m4[0] = __vimax3_s32(m4[0], static_cast<int32_t>(v[k + 0]), static_cast<int32_t>(v[k + 1]));
-            m4[1] = __vimax3_s32(m4[1], static_cast<int32_t>(v[k + 2]), static_cast<int32_t>(v[k + 3]));
-            m4[2] = __vimax3_s32(m4[2], static_cast<int32_t>(v[k + 4]), static_cast<int32_t>(v[k + 5]));
-            m4[3] = __vimax3_s32(m4[3], static_cast<int32_t>(v[k + 6]), static_cast<int32_t>(v[k + 7]));
+            for (int k = 0; k < 32; k += 8) {
+              m4[0] = __vimax3_s32(m4[0], static_cast<int32_t>(v[k + 0]), static_cast<int32_t>(v[k + 1]));
+              m4[1] = __vimax3_s32(m4[1], static_cast<int32_t>(v[k + 2]), static_cast<int32_t>(v[k + 3]));
+              m4[2] = __vimax3_s32(m4[2], static_cast<int32_t>(v[k + 4]), static_cast<int32_t>(v[k + 5]));
+              m4[3] = __vimax3_s32(m4[3], static_cast<int32_t>(v[k + 6]), static_cast<int32_t>(v[k + 7]));
+            }
+          } else {
+            const int nc = nv - 32 * c;
+#pragma unroll
+            for (int k = 0; k < 32; ++k)
+              m4[k & 3] = imax(m4[k & 3], k < nc ? static_cast<int32_t>(v[k]) : INT_MIN);
           }
-        } else {
-          const int nv = nvalid(j);
-#pragma unroll
-          for (int k = 0; k < kCols; ++k) m4[k & 3] = imax(m4[k & 3], k < nv ? static_cast<int32_t>(v[k]) : INT_MIN);
-        }
+        });
+        if (!got) { ok = false; break; }
         m = imax(m, imax(imax(m4[0], m4[1]), imax(m4[2], m4[3])));
       }
       sc += T.nkt;
@@ -332,21 +342,24 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_kernel(const __grid_const
       // ---- pass B: Z = sum of pseudo-exponentials ----
       int32_t Z = 0;
       for (int j = first_j(sc); j < T.nkt; j += kTeams) {
-        uint32_t v[kCols];
-        if (!load_s(sc + j, v)) { ok = false; break; }
         float z4[4] = {0.f, 0.f, 0.f, 0.f};
-        if (tile_full(j)) {
+        const bool full = tile_full(j);
+        const int nv = nvalid(j);
+        const bool got = walk_s(sc + j, [&](const uint32_t (&v)[32], int c) {
+          if (full) {
 #pragma unroll
-          for (int k = 0; k < kCols; ++k)
-            z4[k & 3] += __int_as_float(__shfl_sync(0xffffffffu, lut_lane, static_cast<int>(idx_bits(v[k]))));
-        } else {
-          const int nv = nvalid(j);
+            for (int k = 0; k < 32; ++k)
+              z4[k & 3] += __int_as_float(__shfl_sync(0xffffffffu, lut_lane, static_cast<int>(idx_bits(v[k]))));
+          } else {
+            const int nc = nv - 32 * c;
 #pragma unroll
-          for (int k = 0; k < kCols; ++k) {
-            const uint32_t ib = k < nv ? idx_bits(v[k]) : kMaskedBits;
-            z4[k & 3] += __int_as_float(__shfl_sync(0xffffffffu, lut_lane, static_cast<int>(ib)));
+            for (int k = 0; k < 32; ++k) {
+              const uint32_t ib = k < nc ? idx_bits(v[k]) : kMaskedBits;
+              z4[k & 3] += __int_as_float(__shfl_sync(0xffffffffu, lut_lane, static_cast<int>(ib)));
+            }
           }
-        }
+        });
+        if (!got) { ok = false; break; }
         Z += __float2int_rn((z4[0] + z4[1]) + (z4[2] + z4[3]));
       }
       sc += T.nkt;
@@ -377,36 +390,35 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_kernel(const __grid_const
         const uint32_t pi = pc + j;  // running P index of this tile
         const uint32_t pb = pi & (kPBufs - 1);
         if (!team_wait(bar(kBarPEmpty + pb), ((pi / kPBufs) & 1) ^ 1)) { ok = false; break; }
-        uint32_t v[kCols];
-        if (!load_s(sc + j, v)) { ok = false; break; }
-        uint32_t pw[kCols / 4];
-        if (tile_full(j)) {
+        const bool full = tile_full(j);
+        const int nv = nvalid(j);
+        const bool got = walk_s(sc + j, [&](const uint32_t (&v)[32], int c) {
+          uint32_t pw[8];
+          if (full) {
 #pragma unroll
-          for (int q = 0; q < kCols / 4; ++q) {
-            uint32_t p[4];
+            for (int q = 0; q < 8; ++q) {
+              uint32_t p[4];
 #pragma unroll
-            for (int b = 0; b < 4; ++b) p[b] = lds_u32(idx_bits(v[q * 4 + b]) * 512u + prow);
-            pw[q] = pack4(p[0], p[1], p[2], p[3]);
-          }
-        } else {
-          const int nv = nvalid(j);
-#pragma unroll
-          for (int q = 0; q < kCols / 4; ++q) {
-            uint32_t p[4];
-#pragma unroll
-            for (int b = 0; b < 4; ++b) {
-              const int k = q * 4 + b;
-              const uint32_t ib = k < nv ? idx_bits(v[k]) : kMaskedBits;
-              p[b] = lds_u32(ib * 512u + prow);
+              for (int b = 0; b < 4; ++b) p[b] = lds_u32(idx_bits(v[q * 4 + b]) * 512u + prow);
+              pw[q] = pack4(p[0], p[1], p[2], p[3]);
             }
-            pw[q] = pack4(p[0], p[1], p[2], p[3]);
+          } else {
+            const int nc = nv - 32 * c;
+#pragma unroll
+            for (int q = 0; q < 8; ++q) {
+              uint32_t p[4];
+#pragma unroll
+              for (int b = 0; b < 4; ++b) {
+                const int k = q * 4 + b;
+                const uint32_t ib = k < nc ? idx_bits(v[k]) : kMaskedBits;
+                p[b] = lds_u32(ib * 512u + prow);
+              }
+              pw[q] = pack4(p[0], p[1], p[2], p[3]);
+            }
           }
-        }
-        if constexpr (kCols == 64) {
-          tmem_st16(tlane + kColP + pb * 32 + half * 16, *reinterpret_cast<const uint32_t(*)[16]>(pw));
-        } else {
-          tmem_st8(tlane + kColP + pb * 32 + half * 8, *reinterpret_cast<const uint32_t(*)[8]>(pw));
-        }
+          tmem_st8(tlane + kColP + pb * 32 + half * (kCols / 4) + c * 8, pw);
+        });
+        if (!got) { ok = false; break; }
         tmem_wait_st();
         tc_fence_before();
         arrive_warp(bar(kBarPFull + pb));
