@@ -139,6 +139,13 @@ int intattn_decode_static_scratch(const int8_t *q, const int8_t *k_cache, const 
                                   const intattn_scales_t *scales, int B, int H, int Lk, int Lmax, int d,
                                   float clip_c, int8_t *out, intattn_stream_t stream);
 
+/* Diagnostic for the failure detection: launches one CTA whose wait on a
+ * barrier can never complete.  The wait gives up after the kernels' time
+ * limit (2 s) and sets the device error word, so a following
+ * intattn_device_error(stream) returns INTATTN_ERR_TIMEOUT.  Nothing faults
+ * or hangs and the context stays usable. */
+int intattn_selftest_timeout(intattn_stream_t stream);
+
 /* Synchronises `stream`, then returns and clears the device error word that a
  * kernel sets when one of its bounded waits runs out (INTATTN_ERR_TIMEOUT), or
  * INTATTN_OK.  INTATTN_ERR_CUDA if the synchronisation itself fails. */

@@ -22,8 +22,8 @@ MAX_HEADS = 128
 
 # every function declared in include/intattn.h
 EXPORTED = ("intattn_derive_params", "intattn_forward", "intattn_decode_workspace_size",
-            "intattn_decode", "intattn_decode_static_scratch", "intattn_device_error",
-            "intattn_strerror")
+            "intattn_decode", "intattn_decode_static_scratch", "intattn_selftest_timeout",
+            "intattn_device_error", "intattn_strerror")
 
 
 class IntAttnError(RuntimeError):
@@ -87,6 +87,7 @@ def lib() -> ctypes.CDLL:
                                      f32, vp, vp, ctypes.c_size_t, vp]
         L.intattn_decode_static_scratch.argtypes = [vp, vp, vp, ctypes.POINTER(_Scales), i32, i32, i32,
                                                     i32, i32, f32, vp, vp]
+        L.intattn_selftest_timeout.argtypes = [vp]
         L.intattn_device_error.argtypes = [vp]
         L.intattn_strerror.argtypes = [i32]
         L.intattn_strerror.restype = ctypes.c_char_p
@@ -189,3 +190,12 @@ def device_error(stream=None) -> int:
     """Synchronise and return/clear the device error word (OK or ERR_TIMEOUT)."""
     import torch
     return int(lib().intattn_device_error(_stream_handle(stream, torch.device("cuda"))))
+
+
+def selftest_timeout(stream=None) -> int:
+    """Run the bounded-wait self-test; returns device_error() afterwards
+    (ERR_TIMEOUT when failure detection works)."""
+    import torch
+    _check(lib().intattn_selftest_timeout(_stream_handle(stream, torch.device("cuda"))),
+           "intattn_selftest_timeout")
+    return device_error(stream)

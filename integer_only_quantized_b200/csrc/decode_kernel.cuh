@@ -243,6 +243,21 @@ __global__ void __launch_bounds__(kThreads) decode_pv_kernel(const __grid_consta
   const int32_t* srow = a.ws_s + static_cast<size_t>(bh) * a.ld_s;
   __syncthreads();
 
+  // V rows are streamed with 16-byte loads, one step ahead of the math: the
+  // first step is issued before the probabilities are computed
+  const int piece = tid % Lt::kCPR;
+  const int grp = tid / Lt::kCPR;
+  const int8_t* vbase = a.v + static_cast<size_t>(bh) * a.Lmax * D + piece * 16;
+  auto load4 = [&](int r0, uint4 (&vv)[4]) {
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const int j = r0 + i;
+      vv[i] = (j < j1) ? ld_stream(vbase + static_cast<size_t>(j) * D) : make_uint4(0, 0, 0, 0);
+    }
+  };
+  uint4 cur[4];
+  load4(j0 + 4 * grp, cur);
+
   // u8 probabilities of this chunk, 4 per word (rows past j1 get 0)
   for (int w = tid; w < a.chunk / 4; w += kThreads) {
     uint32_t word = 0;
@@ -258,26 +273,20 @@ __global__ void __launch_bounds__(kThreads) decode_pv_kernel(const __grid_consta
   }
   __syncthreads();
 
-  // stream V: acc[c] over this thread's 16 columns
-  const int piece = tid % Lt::kCPR;
-  const int grp = tid / Lt::kCPR;
-  const int8_t* vbase = a.v + static_cast<size_t>(bh) * a.Lmax * D + piece * 16;
+  // acc[c] over this thread's 16 columns
   int32_t acc[16];
 #pragma unroll
   for (int c = 0; c < 16; ++c) acc[c] = 0;
   for (int base = j0; base < j1; base += Lt::kRowsPerStep) {
     const int r0 = base + 4 * grp;
-    uint4 vv[4];
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      const int j = r0 + i;
-      vv[i] = (j < j1) ? ld_stream(vbase + static_cast<size_t>(j) * D) : make_uint4(0, 0, 0, 0);
-    }
+    const bool more = base + Lt::kRowsPerStep < j1;
+    uint4 nxt[4];
+    if (more) load4(r0 + Lt::kRowsPerStep, nxt);
     const uint32_t p4 = pk[(r0 - j0) >> 2];  // P of rows r0..r0+3, one byte each
-    const uint32_t* w0 = reinterpret_cast<const uint32_t*>(&vv[0]);
-    const uint32_t* w1 = reinterpret_cast<const uint32_t*>(&vv[1]);
-    const uint32_t* w2 = reinterpret_cast<const uint32_t*>(&vv[2]);
-    const uint32_t* w3 = reinterpret_cast<const uint32_t*>(&vv[3]);
+    const uint32_t* w0 = reinterpret_cast<const uint32_t*>(&cur[0]);
+    const uint32_t* w1 = reinterpret_cast<const uint32_t*>(&cur[1]);
+    const uint32_t* w2 = reinterpret_cast<const uint32_t*>(&cur[2]);
+    const uint32_t* w3 = reinterpret_cast<const uint32_t*>(&cur[3]);
 #pragma unroll
     for (int q = 0; q < 4; ++q) {
       // bytes (row i, column 4q+c) -> word c holds the 4 rows of column 4q+c
@@ -289,6 +298,10 @@ __global__ void __launch_bounds__(kThreads) decode_pv_kernel(const __grid_consta
       acc[4 * q + 1] = dp4a_su(__byte_perm(ab_lo, cd_lo, 0x7632), p4, acc[4 * q + 1]);
       acc[4 * q + 2] = dp4a_su(__byte_perm(ab_hi, cd_hi, 0x5410), p4, acc[4 * q + 2]);
       acc[4 * q + 3] = dp4a_su(__byte_perm(ab_hi, cd_hi, 0x7632), p4, acc[4 * q + 3]);
+    }
+    if (more) {
+#pragma unroll
+      for (int i = 0; i < 4; ++i) cur[i] = nxt[i];
     }
   }
   // reduce over the row groups: column piece*16 + c

@@ -202,6 +202,21 @@ int decode_launch(const DecodeArgs& a, cudaStream_t stream) {
   return note_launch(cudaGetLastError());
 }
 
+// ------------------------------------------------------ failure self-test
+// One CTA waits on an mbarrier that nothing will ever arrive on; the bounded
+// wait gives up after its time limit and records the timeout in the device
+// error word, exactly as a stalled pipeline role would.
+__global__ void selftest_timeout_kernel() {
+  __shared__ uint64_t bar;
+  const uint32_t b = intattn::smem_u32(&bar);
+  if (threadIdx.x == 0) {
+    intattn::mbar_init(b, 1);
+    intattn::mbar_fence_init();
+  }
+  __syncthreads();
+  intattn::mbar_wait_warp(b, 0, 15u);
+}
+
 // ------------------------------------------------ static decode scratch
 // Decode scratch for callers that cannot allocate device memory (see
 // intattn_decode_static_scratch in intattn.h).  One array per GPU that loads
@@ -379,6 +394,11 @@ int intattn_decode_static_scratch(const int8_t* q, const int8_t* k_cache, const 
   a.per_head = scales->per_head ? 1 : 0;
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   return d == 64 ? decode_launch<64>(a, st) : decode_launch<128>(a, st);
+}
+
+int intattn_selftest_timeout(intattn_stream_t stream) {
+  selftest_timeout_kernel<<<1, 32, 0, reinterpret_cast<cudaStream_t>(stream)>>>();
+  return note_launch(cudaGetLastError());
 }
 
 int intattn_device_error(intattn_stream_t stream) {
