@@ -17,8 +17,9 @@
 //               (64 of the 128 keys of an S tile).  Row max and row sum
 //               combine the four partial results of a row (two teams x two
 //               halves) through shared memory.
-//   warp 16     TMA producer (one thread): Q (double-buffered), then K/V
-//               tiles through a ring of shared-memory slots.
+//   warp 16     TMA producer: K/V tiles through a ring of shared-memory
+//               slots, one issuing lane per slot; one more lane loads Q
+//               (double-buffered).
 //   warp 17     TMEM allocator and MMA issuer (one thread): tcgen05.mma
 //               kind::i8 for S = Q.K^T (both operands in shared memory) and
 //               O += P.V (P from TMEM, V from shared memory, N-major).
@@ -110,8 +111,8 @@ struct Cfg {
   static constexpr int kNumBars = kBarKvFull + 2 * kStages;
   static constexpr uint32_t kOffQ = 0;                                  // [2] Q tiles
   static constexpr uint32_t kOffKV = kOffQ + 2 * kQBytes;
-  static constexpr uint32_t kOffPtab = kOffKV + kStages * kTileBytes;    // [32][kBM] u32
-  static constexpr uint32_t kOffRed = kOffPtab + 32 * kBM * 4;          // [2][kGroups][kBM] int32
+  static constexpr uint32_t kOffPtab = kOffKV + kStages * kTileBytes;    // [33][kBM] u32
+  static constexpr uint32_t kOffRed = kOffPtab + 33 * kBM * 4;          // [2][kGroups][kBM] int32
   static constexpr uint32_t kOffLut = kOffRed + 2 * kGroups * kBM * 4;
   static constexpr uint32_t kOffBars = kOffLut + 32 * 4;
   static constexpr uint32_t kOffTmem = kOffBars + kNumBars * 8;
@@ -122,6 +123,13 @@ struct Cfg {
 };
 
 __device__ __forceinline__ int32_t imax(int32_t a, int32_t b) { return a > b ? a : b; }
+
+// a b + c, rounded toward zero, then clamped to [0, 1] (one fma.rz.sat).
+__device__ __forceinline__ float fma_rz_sat(float a, float b, float c) {
+  float d;
+  asm("fma.rz.sat.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+  return d;
+}
 
 // Requantise one int32 accumulator: clamp(floor((acc Mo + 2^(so-1)) / 2^so)).
 __device__ __forceinline__ uint32_t requant_byte(int32_t acc, int32_t Mo, int32_t so) {
@@ -224,11 +232,14 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_kernel(const __grid_const
     const int r = quad * 32 + lane;   // query row within the tile == TMEM lane
     const uint32_t tlane = tmem + (static_cast<uint32_t>(quad * 32) << 16);
     const uint32_t trow = tlane + half * kCols;
-    const uint32_t prow = smem_u32(ptab) + 4u * r;  // Ptab[i][r] at prow + 512 i
-    // lane i holds LUT[i] as a float; a shuffle whose source lane is the low
-    // 5 bits of the index bits looks it up.  Per tile a thread sums 32 values
-    // below 2^15, so the float partial sums are exact.
-    const int32_t lut_lane = __float_as_int(__int2float_rn(static_cast<int32_t>(lut_s[lane])));
+    const uint32_t prow = smem_u32(ptab) + 4u * r;  // row k of the table at prow + 512 k
+    // The index code k of a score (see idx_bits below) is idx + 1, or 0 / 32
+    // for a masked / clipped key.  Lane k holds LUT[k-1] as a float (lane 0:
+    // 0); a shuffle whose source lane is the low 5 bits of the code looks it
+    // up.  Per tile a thread sums 32 values below 2^15: the float sums are exact.
+    const int32_t lut_lane =
+        __float_as_int(lane == 0 ? 0.f : __int2float_rn(static_cast<int32_t>(lut_s[lane - 1])));
+    if (warp < 4) ptab[r] = 0u;  // table row 0 (masked keys) stays 0
     bool ok = true;
     uint32_t sc = 0;  // S tiles of the CTA so far (both teams, all passes and tiles)
     uint32_t pc = 0;  // P tiles of the CTA so far
@@ -316,28 +327,30 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_kernel(const __grid_const
       m = imax(imax(red[r], red[kBM + r]), imax(red[2 * kBM + r], red[3 * kBM + r]));
 
       // LUT index of a score, idx = floor((min(m - S, D) M + 2^(s-1)) / 2^s),
-      // evaluated exactly on the FP32 pipe (the integer pipe is the scarcer one):
-      //  * (0x4B000000 + m) - S, read as a float, is 2^23 + (m - S) exactly
-      //    (0 <= m - S <= 2^22);
-      //  * fminf clips the gap at D' = min(D, 2^22 + 1) (D' = D whenever a gap
-      //    can reach D);
-      //  * every valid parameter set has s in {24, 25, 26}, so Ms = M 2^-s and
-      //    c0 = 1/2 - 2^23 Ms are exact floats, and one fused multiply-add
-      //    rounded toward zero gives RZ(gap M / 2^s + 1/2), whose floor is idx;
-      //  * adding 2^23 rounded toward zero leaves 0x4B000000 + idx in the bits:
-      //    the low 5 bits are idx, and (bits * 512) mod 2^32 is idx * 512.
-      // A masked key uses the bits 0x4B00001F: index 31, LUT[31] = 0, Ptab[31] = 0.
+      // evaluated exactly on the FP32 pipe (the integer pipe is the scarcer
+      // one), as the code k = idx + 1 (idx <= 30) or k = 32 (clipped):
+      //  * (0x4B000000 + m) - S, read as a float, is X = 2^23 + g exactly,
+      //    g = m - S in [0, 2^22];
+      //  * with v = g M / 2^s + 1/2, the definition's index is min(floor(v), 31):
+      //    D is the smallest gap whose index reaches 31 and M <= 2^s;
+      //  * every valid parameter set has s in {24, 25, 26}, so Ms' = M 2^-(s+5)
+      //    and c1 = (3/2 - 2^23 M 2^-s) / 32 are exact floats, and
+      //    X Ms' + c1 = (v + 1) / 32; one fma rounded toward zero and saturated
+      //    to [0, 1] gives y = min(RZ((v + 1) / 32), 1);
+      //  * 32 y + 2^23 rounded toward zero is 2^23 + min(floor(v) + 1, 32) (the
+      //    scaling by 32 commutes with the rounding), so the bits are
+      //    0x4B000000 + k: the low 5 bits are k mod 32, and (bits * 512) mod
+      //    2^32 is k * 512, the offset of row k of the table.
+      // A masked key uses the bits 0x4B000000: code 0, lane 0 and row 0 hold 0.
       const uint32_t Cx = 0x4B000000u + static_cast<uint32_t>(m);
-      const int32_t Dp = hp.D < (1 << 22) + 1 ? hp.D : (1 << 22) + 1;
-      const float Xclip = __uint_as_float(0x4B000000u + static_cast<uint32_t>(Dp));
-      const float Mf = __int2float_rn(hp.M);                                                     // exact: M <= 2^24
-      const float Ms = Mf * __uint_as_float(static_cast<uint32_t>(127 - hp.s) << 23);           // M 2^-s
-      const float c0 = 0.5f - Mf * __uint_as_float(static_cast<uint32_t>(127 + 23 - hp.s) << 23);  // exact
+      const float Mf = __int2float_rn(hp.M);                                                   // exact: M <= 2^24
+      const float Ms32 = Mf * __uint_as_float(static_cast<uint32_t>(127 - 5 - hp.s) << 23);   // M 2^-(s+5)
+      const float c1 = (1.5f - Mf * __uint_as_float(static_cast<uint32_t>(127 + 23 - hp.s) << 23)) * 0.03125f;
       auto idx_bits = [&](uint32_t sv) {
-        const float X = fminf(__uint_as_float(Cx - sv), Xclip);
-        return __float_as_uint(__fadd_rz(__fmaf_rz(X, Ms, c0), 8388608.0f));
+        const float y = fma_rz_sat(__uint_as_float(Cx - sv), Ms32, c1);
+        return __float_as_uint(__fmaf_rz(y, 32.0f, 8388608.0f));
       };
-      constexpr uint32_t kMaskedBits = 0x4B00001Fu;
+      constexpr uint32_t kMaskedBits = 0x4B000000u;
 
       // ---- pass B: Z = sum of pseudo-exponentials ----
       int32_t Z = 0;
@@ -368,8 +381,8 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_kernel(const __grid_const
       Z = (red[kGroups * kBM + r] + red[(kGroups + 1) * kBM + r]) +
           (red[(kGroups + 2) * kBM + r] + red[(kGroups + 3) * kBM + r]);
 
-      // reciprocal and this row's probability table (each of the four threads
-      // of a row writes 8 of the 32 entries)
+      // reciprocal and this row's probability table: row k = Ptab[k - 1]
+      // (each of the four threads of a row writes 8 of the rows 1..32)
       {
         // R = floor(N / Z), N = 255 2^32 + floor(Z/2) < 2^40: the double
         // quotient is within one unit of R, and one integer step makes it exact.
@@ -381,7 +394,8 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_kernel(const __grid_const
         else if ((R + 1) * Zu <= N) ++R;
 #pragma unroll
         for (int i = grp * 8; i < grp * 8 + 8; ++i)
-          ptab[i * kBM + r] = static_cast<uint32_t>((static_cast<unsigned long long>(lut_s[i]) * R + (1ull << 31)) >> 32);
+          ptab[(i + 1) * kBM + r] =
+              static_cast<uint32_t>((static_cast<unsigned long long>(lut_s[i]) * R + (1ull << 31)) >> 32);
       }
       all_sync(true);  // the table is complete
 
@@ -458,51 +472,71 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_kernel(const __grid_const
     }
   } else if (warp == kProducerWarp) {
     // ============================ TMA producer ============================
-    // The whole warp runs this loop on uniform values; one elected lane issues.
+    // The tensor loads one thread issues are served one after another, so a
+    // single issuing thread caps the load rate of the SM far below what the
+    // passes consume.  Lane s < kStages therefore owns ring slot s and issues
+    // every K/V load that lands there (load n goes to slot n % kStages), and
+    // lane kQLane issues the Q loads.  Each lane walks the same load sequence
+    // and waits, with the per-thread bounded wait, only on its own barriers.
+    constexpr int kQLane = 31;
+    static_assert(C::kStages <= kQLane, "one lane per ring slot");
     if (lane == 0) {
       tma_prefetch_desc(&args.tm_q);
       tma_prefetch_desc(&args.tm_k);
       tma_prefetch_desc(&args.tm_v);
     }
-    uint32_t n = 0;   // K/V loads issued, in the MMA warp's consumption order
-    uint32_t nq = 0;  // Q loads issued
-    bool ok = true;
-    auto load = [&](const CUtensorMap* tm, int j, int bh) {
-      if (!ok) return;
-      const uint32_t slot = n % C::kStages;
-      const uint32_t use = n / C::kStages;
-      if (!mbar_wait_warp(bar_kv_empty(slot), (use & 1) ^ 1, kRoleProducer)) { ok = false; return; }
-      tma_load_3d_elect(sKV + slot * C::kTileBytes, tm, bar_kv_full(slot), C::kTileBytes, 0, j * kBN, bh);
-      ++n;
-    };
-    for (int it = 0; ok; ++it) {
-      const int L = tile_index(it, blockIdx.x, gridDim.x);
-      if (L >= args.n_tiles) break;
-      const Tile T = tile_of(args, L);
-      const uint32_t qb = nq & 1;
-      if (!mbar_wait_warp(bar(kBarQEmpty + qb), ((nq >> 1) & 1) ^ 1, kRoleProducer)) { ok = false; break; }
-      tma_load_3d_elect(sQ(qb), &args.tm_q, bar(kBarQFull + qb), C::kQBytes, 0, T.q0, T.bh);
-      ++nq;
-      for (int pass = 0; pass < 2; ++pass)
-        for (int j = 0; j < T.nkt; ++j) load(&args.tm_k, j, T.bh);
-      load(&args.tm_k, 0, T.bh);
-      if (T.nkt > 1) load(&args.tm_k, 1, T.bh);
-      for (int j = 0; j < T.nkt; ++j) {
-        if (j + 2 < T.nkt) load(&args.tm_k, j + 2, T.bh);
-        load(&args.tm_v, j, T.bh);
+    __syncwarp();
+    if (lane < C::kStages) {
+      const uint32_t slot = static_cast<uint32_t>(lane);
+      const uint32_t dst = sKV + slot * C::kTileBytes;
+      uint32_t n = 0;     // position in the K/V load sequence (MMA consumption order)
+      uint32_t mine = 0;  // loads this lane issued
+      bool ok = true;
+      auto load = [&](const CUtensorMap* tm, int j, int bh) {
+        if (ok && n % C::kStages == slot) {
+          if (!mbar_wait(bar_kv_empty(slot), (mine & 1) ^ 1, kRoleProducer)) {
+            ok = false;
+          } else {
+            mbar_arrive_expect_tx(bar_kv_full(slot), C::kTileBytes);
+            tma_load_3d(dst, tm, bar_kv_full(slot), 0, j * kBN, bh);
+            ++mine;
+          }
+        }
+        ++n;
+      };
+      for (int it = 0; ok; ++it) {
+        const int L = tile_index(it, blockIdx.x, gridDim.x);
+        if (L >= args.n_tiles) break;
+        const Tile T = tile_of(args, L);
+        for (int pass = 0; pass < 2; ++pass)
+          for (int j = 0; j < T.nkt; ++j) load(&args.tm_k, j, T.bh);
+        load(&args.tm_k, 0, T.bh);
+        if (T.nkt > 1) load(&args.tm_k, 1, T.bh);
+        for (int j = 0; j < T.nkt; ++j) {
+          if (j + 2 < T.nkt) load(&args.tm_k, j + 2, T.bh);
+          load(&args.tm_v, j, T.bh);
+        }
+      }
+      // never leave with a copy in flight: wait for this slot's last load
+      if (mine > 0) mbar_wait(bar_kv_full(slot), (mine - 1) & 1, kRoleProducer);
+    } else if (lane == kQLane) {
+      uint32_t nq = 0;  // Q loads issued
+      for (int it = 0;; ++it) {
+        const int L = tile_index(it, blockIdx.x, gridDim.x);
+        if (L >= args.n_tiles) break;
+        const Tile T = tile_of(args, L);
+        const uint32_t qb = nq & 1;
+        if (!mbar_wait(bar(kBarQEmpty + qb), ((nq >> 1) & 1) ^ 1, kRoleProducer)) break;
+        mbar_arrive_expect_tx(bar(kBarQFull + qb), C::kQBytes);
+        tma_load_3d(sQ(qb), &args.tm_q, bar(kBarQFull + qb), 0, T.q0, T.bh);
+        ++nq;
+      }
+      for (uint32_t i = 0; i < 2 && i < nq; ++i) {
+        const uint32_t last = nq - 1 - i;  // the last load of each Q buffer
+        mbar_wait(bar(kBarQFull + (last & 1)), (last >> 1) & 1, kRoleProducer);
       }
     }
-    // never leave with a copy in flight: wait for the last load of each slot
-    for (uint32_t slot = 0; slot < static_cast<uint32_t>(C::kStages); ++slot) {
-      if (n > slot) {
-        const uint32_t uses = (n - slot - 1) / C::kStages + 1;
-        mbar_wait_warp(bar_kv_full(slot), (uses - 1) & 1, kRoleProducer);
-      }
-    }
-    for (uint32_t i = 0; i < 2 && i < nq; ++i) {
-      const uint32_t last = nq - 1 - i;  // the last load of each Q buffer
-      mbar_wait_warp(bar(kBarQFull + (last & 1)), (last >> 1) & 1, kRoleProducer);
-    }
+    __syncwarp();
   } else {
     // ============================= MMA issuer =============================
     // The whole warp runs this loop on uniform values (descriptors stay in
