@@ -71,6 +71,7 @@ constexpr int kTeamWarps = kSoftWarps / kTeams;
 constexpr int kColGroups = kTeamWarps / 4;  // column groups per team
 constexpr int kCols = kBN / kColGroups;     // S columns per thread and tile
 constexpr int kGroups = kTeams * kColGroups;  // partial results per query row (= 4)
+constexpr int kSoftBase = 0;               // first softmax warp
 constexpr int kProducerWarp = kSoftWarps;
 constexpr int kMmaWarp = kSoftWarps + 1;
 constexpr int kThreads = 32 * (kSoftWarps + 2);  // 576
@@ -103,7 +104,7 @@ enum Bar : int {
 
 template <int D>
 struct Cfg {
-  static constexpr int kStages = (D == 64) ? 6 : 4;
+  static constexpr int kStages = (D == 64) ? 8 : 6;
   static constexpr uint32_t kTileBytes = kBN * D;  // one K or V tile
   static constexpr uint32_t kQBytes = kBM * D;
   static constexpr uint32_t kSwizzle = (D == 128) ? 2u : 4u;  // 128B / 64B swizzle
@@ -223,11 +224,14 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_kernel(const __grid_const
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
 
-  if (warp < kSoftWarps) {
+  if (warp >= kSoftBase && warp < kSoftBase + kSoftWarps) {
     // ======================= IndexSoftmax warps =======================
+    // A warp reaches the TMEM lanes of quadrant warp % 4; four consecutive
+    // softmax warps cover the four quadrants.
+    const int sw = warp - kSoftBase;
     const int quad = warp & 3;
-    const int half = (warp >> 2) % kColGroups;  // column group within the team
-    const int team = warp / kTeamWarps;
+    const int half = (sw >> 2) % kColGroups;  // column group within the team
+    const int team = sw / kTeamWarps;
     const int grp = team * kColGroups + half;   // slot of this thread's partial results
     const int r = quad * 32 + lane;   // query row within the tile == TMEM lane
     const uint32_t tlane = tmem + (static_cast<uint32_t>(quad * 32) << 16);
@@ -239,18 +243,18 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_kernel(const __grid_const
     // up.  Per tile a thread sums 32 values below 2^15: the float sums are exact.
     const int32_t lut_lane =
         __float_as_int(lane == 0 ? 0.f : __int2float_rn(static_cast<int32_t>(lut_s[lane - 1])));
-    if (warp < 4) ptab[r] = 0u;  // table row 0 (masked keys) stays 0
+    if (sw < 4) ptab[r] = 0u;  // table row 0 (masked keys) stays 0
     bool ok = true;
     uint32_t sc = 0;  // S tiles of the CTA so far (both teams, all passes and tiles)
     uint32_t pc = 0;  // P tiles of the CTA so far
-    const bool leader = (warp & (kTeamWarps - 1)) == 0;  // warps 0 and 8 poll for their team
+    const bool leader = (sw & (kTeamWarps - 1)) == 0;  // the first warp of a team polls for it
     // wait for a barrier phase: the team leader polls, the team sleeps in a
     // named barrier that hands everyone the leader's verdict
     auto team_wait = [&](uint32_t b, uint32_t parity) {
       const bool got = leader ? mbar_wait(b, parity, kRoleSoftmax) : true;
       return bar_red_and(kNbTeam + team, 32 * kTeamWarps, got);
     };
-    // all sixteen softmax warps: every warp's `ok`, and (warp 0 polling) a phase
+    // all sixteen softmax warps: every warp's `ok`, and (softmax warp 0 polling) a phase
     auto all_sync = [&](bool mine) { return bar_red_and(kNbAll, 32 * kSoftWarps, mine); };
     auto arrive_warp = [&](uint32_t b) {  // one arrival per warp
       __syncwarp();
@@ -442,7 +446,7 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_kernel(const __grid_const
 
       // ---- epilogue: O (int32, TMEM) -> requantised int8 rows ----
       {
-        const bool got = (ok && warp == 0) ? mbar_wait(bar(kBarOFull), it & 1, kRoleSoftmax) : ok;
+        const bool got = (ok && sw == 0) ? mbar_wait(bar(kBarOFull), it & 1, kRoleSoftmax) : ok;
         if (!all_sync(got)) { ok = false; break; }
       }
       tc_fence_after();
@@ -537,18 +541,25 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_kernel(const __grid_const
       }
     }
     __syncwarp();
-  } else {
+  } else if (warp == kMmaWarp) {
     // ============================= MMA issuer =============================
     // The whole warp runs this loop on uniform values (descriptors stay in
-    // uniform registers); one elected lane issues each tcgen05 instruction.
+    // uniform registers) and waits for both inputs of an MMA group with one
+    // vote per poll; one elected lane issues the group and its commits.
     constexpr uint32_t idesc_qk = idesc_i8(kBM, kBN, 1, 1, 0);  // s8 x s8, K-major B
     constexpr uint32_t idesc_pv = idesc_i8(kBM, D, 0, 1, 1);    // u8 x s8, N-major B
     const uint64_t kv_desc0 = smem_desc(sKV, 16, C::kSBO, C::kSwizzle);
     constexpr uint32_t kSlotDesc = C::kTileBytes >> 4;  // descriptor step between ring slots
     bool ok = true;
-    uint32_t n = 0;   // K/V tiles consumed
+    uint32_t slot = 0, kv_par = 0;  // ring slot and phase parity of the next K/V tile
     uint32_t sc = 0;  // S tiles produced
     uint32_t pc = 0;  // P tiles consumed
+    auto next_slot = [&]() {
+      if (++slot == static_cast<uint32_t>(C::kStages)) {
+        slot = 0;
+        kv_par ^= 1;
+      }
+    };
     for (int it = 0; ok; ++it) {
       const int L = tile_index(it, blockIdx.x, gridDim.x);
       if (L >= args.n_tiles) break;
@@ -559,20 +570,21 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_kernel(const __grid_const
       auto issue_qk = [&]() {
         if (!ok) return;
         const uint32_t buf = sc & 1;
-        const uint32_t slot = n % C::kStages;
-        if (!mbar_wait_warp(bar(kBarSEmpty + buf), ((sc >> 1) & 1) ^ 1, kRoleMma) ||
-            !mbar_wait_warp(bar_kv_full(slot), (n / C::kStages) & 1, kRoleMma)) {
+        if (!mbar_wait2_warp(bar(kBarSEmpty + buf), ((sc >> 1) & 1) ^ 1, bar_kv_full(slot), kv_par, kRoleMma)) {
           ok = false;
           return;
         }
         tc_fence_after();
         const uint64_t k_desc = kv_desc0 + slot * kSlotDesc;
+        if (elect_one()) {
 #pragma unroll
-        for (int kk = 0; kk < D / 32; ++kk)  // K = 32 bytes per MMA: advance 32 B
-          mma_i8_ss_elect(tmem + kColS + buf * kBN, q_desc + 2 * kk, k_desc + 2 * kk, idesc_qk, kk > 0);
-        mma_commit_elect(bar_kv_empty(slot));
-        mma_commit_elect(bar(kBarSFull + buf));
-        ++n;
+          for (int kk = 0; kk < D / 32; ++kk)  // K = 32 bytes per MMA: advance 32 B
+            mma_i8_ss(tmem + kColS + buf * kBN, q_desc + 2 * kk, k_desc + 2 * kk, idesc_qk, kk > 0);
+          mma_commit(bar_kv_empty(slot));
+          mma_commit(bar(kBarSFull + buf));
+        }
+        __syncwarp();
+        next_slot();
         ++sc;
       };
       for (int t = 0; t < 2 * T.nkt; ++t) issue_qk();  // passes A and B
@@ -586,21 +598,22 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_kernel(const __grid_const
         // O of the previous tile must have been read before it is overwritten
         if (j == 0 && !mbar_wait_warp(bar(kBarOEmpty), (it & 1) ^ 1, kRoleMma)) { ok = false; break; }
         const uint32_t pb = pc & (kPBufs - 1);
-        const uint32_t slot = n % C::kStages;
-        if (!mbar_wait_warp(bar(kBarPFull + pb), (pc / kPBufs) & 1, kRoleMma) ||
-            !mbar_wait_warp(bar_kv_full(slot), (n / C::kStages) & 1, kRoleMma)) {
+        if (!mbar_wait2_warp(bar(kBarPFull + pb), (pc / kPBufs) & 1, bar_kv_full(slot), kv_par, kRoleMma)) {
           ok = false;
           break;
         }
         tc_fence_after();
         const uint64_t v_desc = kv_desc0 + slot * kSlotDesc;
+        if (elect_one()) {
 #pragma unroll
-        for (int kk = 0; kk < kBN / 32; ++kk)  // 32 keys per MMA: 8 TMEM columns of P, 32 V rows
-          mma_i8_ts_elect(tmem + kColO, tmem + kColP + pb * 32 + kk * 8, v_desc + ((32u * D * kk) >> 4),
-                          idesc_pv, (j > 0 || kk > 0) ? 1u : 0u);
-        mma_commit_elect(bar_kv_empty(slot));
-        mma_commit_elect(bar(kBarPEmpty + pb));
-        ++n;
+          for (int kk = 0; kk < kBN / 32; ++kk)  // 32 keys per MMA: 8 TMEM columns of P, 32 V rows
+            mma_i8_ts(tmem + kColO, tmem + kColP + pb * 32 + kk * 8, v_desc + ((32u * D * kk) >> 4), idesc_pv,
+                      (j > 0 || kk > 0) ? 1u : 0u);
+          mma_commit(bar_kv_empty(slot));
+          mma_commit(bar(kBarPEmpty + pb));
+        }
+        __syncwarp();
+        next_slot();
       }
       if (!ok) break;
       mma_commit_elect(bar(kBarQEmpty + qb));  // every MMA that read this Q buffer

@@ -127,6 +127,32 @@ __device__ __forceinline__ bool mbar_wait_warp(uint32_t bar, uint32_t parity, un
   }
 }
 
+// Warp-wide wait for two barriers at once: the warp leaves as one when a lane
+// has seen both phases complete (one vote per poll).  Same time limit.
+__device__ __forceinline__ bool mbar_wait2_warp(uint32_t bar_a, uint32_t par_a, uint32_t bar_b, uint32_t par_b,
+                                                unsigned role) {
+  if (__any_sync(0xffffffffu, mbar_try_wait(bar_a, par_a) && mbar_try_wait(bar_b, par_b))) return true;
+  const unsigned long long t0 = globaltimer_ns();
+  while (true) {
+    if (__any_sync(0xffffffffu, mbar_try_wait(bar_a, par_a) && mbar_try_wait(bar_b, par_b))) return true;
+    if (globaltimer_ns() - t0 > kWaitTimeoutNs) {
+      if ((threadIdx.x & 31) == 0) atomicOr(&g_device_error, kErrTimeout | (role << 8));
+      return false;
+    }
+  }
+}
+
+// True on exactly one lane of the (converged) warp.
+__device__ __forceinline__ bool elect_one() {
+  uint32_t e;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "elect.sync _|p, 0xffffffff;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(e));
+  return e != 0;
+}
+
 // -------------------------------------------------------------------- TMA
 __device__ __forceinline__ void tma_prefetch_desc(const void* tmap) {
   asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(tmap)) : "memory");
