@@ -34,10 +34,12 @@
 // S is recomputed by the tensor cores in each pass; K streams three times
 // (from L2 after the first), V once.
 //
-// Every mbarrier wait is bounded (polls with a time limit).  In each softmax
-// team one leader warp polls and the other warps sleep in a named barrier
-// that ANDs the leader's verdict (bar.red.and), so all warps of a team leave
-// together, also on a timeout, and no warp can be left waiting.
+// Every mbarrier wait is bounded (polls with a time limit).  Each softmax
+// warp polls its own barriers (one vote per poll).  A warp whose wait runs
+// out leaves its pass loop; every softmax warp still reaches the same
+// sequence of all-warp named barriers (one per pass and per epilogue), which
+// AND the warps' verdicts (bar.red.and), so all warps then leave together
+// and none is left waiting.
 #pragma once
 #include <cuda.h>
 #include <climits>
@@ -82,7 +84,6 @@ constexpr uint32_t kColP = 384;  // four P buffers of 32 columns (128 u8 keys ea
 constexpr int kPBufs = 4;
 // named barriers (id 0 is __syncthreads)
 constexpr uint32_t kNbAll = 1;   // all softmax warps
-constexpr uint32_t kNbTeam = 2;  // + team: the warps of one team
 
 static_assert(kGroups == 4 && kCols % 32 == 0, "4 partials per row, whole 32-column TMEM loads");
 
@@ -247,13 +248,10 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_kernel(const __grid_const
     bool ok = true;
     uint32_t sc = 0;  // S tiles of the CTA so far (both teams, all passes and tiles)
     uint32_t pc = 0;  // P tiles of the CTA so far
-    const bool leader = (sw & (kTeamWarps - 1)) == 0;  // the first warp of a team polls for it
-    // wait for a barrier phase: the team leader polls, the team sleeps in a
-    // named barrier that hands everyone the leader's verdict
-    auto team_wait = [&](uint32_t b, uint32_t parity) {
-      const bool got = leader ? mbar_wait(b, parity, kRoleSoftmax) : true;
-      return bar_red_and(kNbTeam + team, 32 * kTeamWarps, got);
-    };
+    // wait for a barrier phase (every warp polls for itself: a leader that
+    // polls and wakes its team through a named barrier adds that barrier's
+    // latency to every S tile)
+    auto team_wait = [&](uint32_t b, uint32_t parity) { return mbar_wait_warp(b, parity, kRoleSoftmax); };
     // all sixteen softmax warps: every warp's `ok`, and (softmax warp 0 polling) a phase
     auto all_sync = [&](bool mine) { return bar_red_and(kNbAll, 32 * kSoftWarps, mine); };
     auto arrive_warp = [&](uint32_t b) {  // one arrival per warp
