@@ -96,9 +96,9 @@ def load_peaks():
     return dict(FALLBACK_PEAKS), "fallback"
 
 
-def kernel_traffic(kernel: str, workload: str):
-    """DRAM bytes per launch from a committed ncu summary, only while the
-    kernel source still has the hash the counters were taken with."""
+def kernel_traffic(kernel: str, workload: str, key: str = "bytes_per_launch"):
+    """DRAM bytes per launch (or per call) from a committed ncu summary, only
+    while the kernel source still has the hash the counters were taken with."""
     import hashlib
     path = os.path.join(ROOT, "profiles", "traffic.json")
     if not os.path.exists(path):
@@ -114,7 +114,7 @@ def kernel_traffic(kernel: str, workload: str):
             h.update(f.read())
     if h.hexdigest()[:16] != ent.get("source_hash"):
         return None
-    return ent.get("bytes_per_launch")
+    return ent.get(key)
 
 
 # ----------------------------------------------------------------- clocks
@@ -336,11 +336,13 @@ def run_decode(args, dev, stream, world, peaks, peak_src):
         raise RuntimeError("a kernel wait timed out in decode")
     gbs = w.decode_bytes / (ms * 1e-3) / 1e9
     return {"workload": w.name, "value": round(aggregate_value(w.decode_bytes, world, ms * 1e-3) / 1e9, 1),
-            "unit": "GB/s", "ms_per_call": round(ms, 5), "launches_per_call": 2,
+            "unit": "GB/s", "ms_per_call": round(ms, 5), "launches_per_call": 3,
             "bytes_per_call": int(w.decode_bytes),
             "roofline": {"bound": "hbm", "achieved": round(gbs, 1), "peak": peaks["hbm_gbs"],
                          "unit": "GB/s", "frac": round(gbs / peaks["hbm_gbs"], 4),
-                         "peak_source": f"{peak_src} hbm_gbs", "traffic": None},
+                         "peak_source": f"{peak_src} hbm_gbs",
+                         "traffic": kernel_traffic("decode", w.name, "bytes_per_call"),
+                         "traffic_unit": "DRAM bytes per call (decode_qk + decode_z + decode_pv)"},
             "l2": "K/V caches 2 GiB > 126 MiB L2"}
 
 
