@@ -252,11 +252,11 @@ def make_inputs_torch(w: Workload, device) -> DeviceInputs:
     v, s_v = one("v", Lkv)
     # output scale from an fp64 row sample, as in make_inputs
     rows = torch.as_tensor(_sample_rows(w.Lq), device=device)
-    sq = torch.as_tensor(np.broadcast_to(s_q, (w.H,)) if w.per_head else np.full(w.H, s_q[0]),
+    sq = torch.as_tensor(np.array(np.broadcast_to(s_q, (w.H,))) if w.per_head else np.full(w.H, s_q[0]),
                          device=device, dtype=torch.float64)
-    sk = torch.as_tensor(np.broadcast_to(s_k, (w.H,)) if w.per_head else np.full(w.H, s_k[0]),
+    sk = torch.as_tensor(np.array(np.broadcast_to(s_k, (w.H,))) if w.per_head else np.full(w.H, s_k[0]),
                          device=device, dtype=torch.float64)
-    sv = torch.as_tensor(np.broadcast_to(s_v, (w.H,)) if w.per_head else np.full(w.H, s_v[0]),
+    sv = torch.as_tensor(np.array(np.broadcast_to(s_v, (w.H,))) if w.per_head else np.full(w.H, s_v[0]),
                          device=device, dtype=torch.float64)
     amax = torch.zeros(w.H, dtype=torch.float64, device=device)
     for b in range(w.B):
