@@ -298,7 +298,9 @@ def run_ours(args):
     }
 
     if not args.no_decode:
-        line["decode"] = run_decode(args, dev, stream, world, peaks, peak_src)
+        line["decode"] = run_decode(args, dev, stream, world, peaks, peak_src, args.decode_workload)
+        line["decode_int4"] = run_decode(args, dev, stream, world, peaks, peak_src,
+                                         "llama7b_decode_int4_b64_lk4096")
     if not args.no_cpu_baseline and rank == 0 and world == 1:
         line["cpu_baseline"] = cpu_baseline(w, x, args.cpu_seconds)
     if rank == 0:
@@ -308,26 +310,33 @@ def run_ours(args):
         dist.destroy_process_group()
 
 
-def run_decode(args, dev, stream, world, peaks, peak_src):
-    """Decode over the int8 KV cache: GB/s of K/V cache rows + q + out."""
+def run_decode(args, dev, stream, world, peaks, peak_src, name):
+    """Decode over the int8 (or packed int4) KV cache: GB/s of K/V cache rows
+    + q + out."""
     import torch
 
     import integer_only_quantized_b200 as ia
     from integer_only_quantized_b200 import workloads as wl
-    w = wl.WORKLOADS[args.decode_workload]
+    w = wl.WORKLOADS[name]
     x = wl.make_inputs_torch(w, dev)
     sc = ia.Scales(x.s_q, x.s_k, x.s_v, x.s_o, per_head=w.per_head)
     ws = torch.empty(ia.decode_workspace_size(w.B, w.H, w.Lk, w.d), dtype=torch.uint8, device=dev)
     out = torch.empty_like(x.q)
+    if w.kv_bits == 4:
+        kc, vc = wl.pack_int4_torch(x.k), wl.pack_int4_torch(x.v)
+        del x.k, x.v
+        call = lambda: ia.decode_int4(x.q, kc, vc, sc, w.Lk, w.clip_c, out=out, workspace=ws, stream=stream)
+    else:
+        call = lambda: ia.decode(x.q, x.k, x.v, sc, w.Lk, w.clip_c, out=out, workspace=ws, stream=stream)
     steps = max(10, min(args.steps, 100))
     for _ in range(max(3, args.warmup)):
-        ia.decode(x.q, x.k, x.v, sc, w.Lk, w.clip_c, out=out, workspace=ws, stream=stream)
+        call()
     torch.cuda.synchronize(dev)
     barrier(world, dev)
     t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     t0.record(stream)
     for _ in range(steps):
-        ia.decode(x.q, x.k, x.v, sc, w.Lk, w.clip_c, out=out, workspace=ws, stream=stream)
+        call()
     t1.record(stream)
     torch.cuda.synchronize(dev)
     barrier(world, dev)
@@ -343,7 +352,8 @@ def run_decode(args, dev, stream, world, peaks, peak_src):
                          "peak_source": f"{peak_src} hbm_gbs",
                          "traffic": kernel_traffic("decode", w.name, "bytes_per_call"),
                          "traffic_unit": "DRAM bytes per call (decode_qk + decode_z + decode_pv)"},
-            "l2": "K/V caches 2 GiB > 126 MiB L2"}
+            "kv_bits": w.kv_bits,
+            "l2": f"K/V caches {2 * w.B * w.H * w.Lmax * w.d * w.kv_bits / 8 / 2**30:.0f} GiB > 126 MiB L2"}
 
 
 # ------------------------------------------------------- CPU oracle legs

@@ -113,6 +113,20 @@ int intattn_decode(const int8_t *q, const int8_t *k_cache, const int8_t *v_cache
                    float clip_c, int8_t *out, void *workspace, size_t workspace_bytes,
                    intattn_stream_t stream);
 
+/* Decode over an int4 KV cache (IntAttention Methodology item 3 with 4-bit
+ * keys and values: the same integer definition, with K and V codes in
+ * [-8, 7] and s_k, s_v the scales of those codes).  Halves the bytes a
+ * decode step streams.
+ *   k_cache, v_cache: [B, H, Lmax, d/2] bytes; byte t of a row holds channel
+ *   2t in bits 0-3 and channel 2t+1 in bits 4-7, each a 4-bit two's
+ *   complement value.  q [B, H, 1, d] int8, out [B, H, 1, d] int8.
+ *   Workspace: as intattn_decode (intattn_decode_workspace_size).
+ *   Arguments, contracts and return codes: as intattn_decode. */
+int intattn_decode_int4(const int8_t *q, const uint8_t *k_cache, const uint8_t *v_cache,
+                        const intattn_scales_t *scales, int B, int H, int Lk, int Lmax, int d,
+                        float clip_c, int8_t *out, void *workspace, size_t workspace_bytes,
+                        intattn_stream_t stream);
+
 /* Capacity in bytes of the library's static decode scratch (48 MiB). */
 #define INTATTN_STATIC_SCRATCH_BYTES (48u * 1024u * 1024u)
 

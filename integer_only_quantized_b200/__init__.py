@@ -22,8 +22,8 @@ MAX_HEADS = 128
 
 # every function declared in include/intattn.h
 EXPORTED = ("intattn_derive_params", "intattn_forward", "intattn_decode_workspace_size",
-            "intattn_decode", "intattn_decode_static_scratch", "intattn_selftest_timeout",
-            "intattn_device_error", "intattn_strerror")
+            "intattn_decode", "intattn_decode_int4", "intattn_decode_static_scratch",
+            "intattn_selftest_timeout", "intattn_device_error", "intattn_strerror")
 
 
 class IntAttnError(RuntimeError):
@@ -85,6 +85,8 @@ def lib() -> ctypes.CDLL:
         L.intattn_decode_workspace_size.restype = ctypes.c_size_t
         L.intattn_decode.argtypes = [vp, vp, vp, ctypes.POINTER(_Scales), i32, i32, i32, i32, i32,
                                      f32, vp, vp, ctypes.c_size_t, vp]
+        L.intattn_decode_int4.argtypes = [vp, vp, vp, ctypes.POINTER(_Scales), i32, i32, i32, i32, i32,
+                                          f32, vp, vp, ctypes.c_size_t, vp]
         L.intattn_decode_static_scratch.argtypes = [vp, vp, vp, ctypes.POINTER(_Scales), i32, i32, i32,
                                                     i32, i32, f32, vp, vp]
         L.intattn_selftest_timeout.argtypes = [vp]
@@ -183,6 +185,45 @@ def decode(q, k_cache, v_cache, scales: Scales, Lk: int, clip_c: float, out=None
                               _stream_handle(stream, q.device))
     del keep
     _check(rc, "intattn_decode")
+    return out
+
+
+def _check_u8_tensor(t, name: str):
+    import torch
+    if not isinstance(t, torch.Tensor) or t.dtype != torch.uint8 or not t.is_cuda:
+        raise TypeError(f"{name} must be a CUDA uint8 tensor")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+
+
+def decode_int4(q, k_cache, v_cache, scales: Scales, Lk: int, clip_c: float, out=None, workspace=None,
+                stream=None):
+    """out[B,H,1,d] int8 over an int4 KV cache: k_cache/v_cache are uint8
+    [B, H, Lmax, d/2], two 4-bit two's-complement channels per byte (channel
+    2t in the low nibble of byte t)."""
+    import torch
+    _check_tensor(q, "q")
+    for t, n in ((k_cache, "k_cache"), (v_cache, "v_cache")):
+        _check_u8_tensor(t, n)
+    B, H, one, d = q.shape
+    if one != 1:
+        raise ValueError("decode takes one query per (b, h): q is [B, H, 1, d]")
+    Lmax = k_cache.shape[2]
+    if k_cache.shape != (B, H, Lmax, d // 2) or v_cache.shape != k_cache.shape:
+        raise ValueError("int4 caches must be [B, H, Lmax, d/2] bytes")
+    if out is None:
+        out = torch.empty_like(q)
+    _check_tensor(out, "out")
+    need = decode_workspace_size(B, H, Lk, d)
+    if workspace is None:
+        workspace = torch.empty(max(need, 1), dtype=torch.uint8, device=q.device)
+    sc, keep = scales._c()
+    rc = lib().intattn_decode_int4(q.data_ptr(), k_cache.data_ptr(), v_cache.data_ptr(), ctypes.byref(sc), B,
+                                   H, int(Lk), Lmax, d, float(clip_c), out.data_ptr(), workspace.data_ptr(),
+                                   workspace.numel() * workspace.element_size(),
+                                   _stream_handle(stream, q.device))
+    del keep
+    _check(rc, "intattn_decode_int4")
     return out
 
 

@@ -1,4 +1,5 @@
-// Decode kernels: one query per (batch, head) against an int8 KV cache.
+// Decode kernels: one query per (batch, head) against an int8 or int4 KV
+// cache.
 //
 // Same integer definition as the prefill path with Lq = 1 and no mask.  The
 // work is an HBM stream of the K and V rows (2*Lk*d bytes per (b, h)), so it
@@ -13,6 +14,13 @@
 //              The last CTA of a (b, h) (atomic ticket) adds the partials and
 //              requantises.  Integer addition is associative, so the result
 //              does not depend on the order.
+// int4 cache (kInt4): rows of D/2 bytes, byte t holding channel 2t in bits
+// 0-3 and channel 2t+1 in bits 4-7, each a two's-complement value in
+// [-8, 7].  A thread unpacks its 8-byte piece (16 channels) into the biased
+// unsigned bytes u = x + 8 ((nibble ^ 8), one logic op per 4 channels), in
+// the channel order {0,2,4,6} {1,3,5,7} {8,..,14} {9,..,15}; dp4a then works
+// on u and the bias is removed exactly: q.x = q.u - 8 sum(q), and
+// sum P x = sum P u - 8 sum(P).
 #pragma once
 #include <climits>
 #include <cstdint>
@@ -24,8 +32,8 @@ namespace intattn {
 
 struct DecodeArgs {
   const int8_t* q;   // [BH, d]
-  const int8_t* k;   // [BH, Lmax, d]
-  const int8_t* v;   // [BH, Lmax, d]
+  const int8_t* k;   // [BH, Lmax, d] int8, or [BH, Lmax, d/2] packed int4
+  const int8_t* v;   // same layout as k
   int8_t* out;       // [BH, d]
   int32_t* ws_s;     // [BH, ld_s]        scores (row stride ld_s = Lk rounded up to 4)
   int32_t* ws_max;   // [BH, nsplit]      chunk maxima
@@ -50,6 +58,31 @@ __device__ __forceinline__ uint4 ld_stream(const void* p) {
   return r;
 }
 
+__device__ __forceinline__ uint2 ld_stream8(const void* p) {
+  uint2 r;
+  asm volatile("ld.global.nc.L1::no_allocate.v2.u32 {%0, %1}, [%2];" : "=r"(r.x), "=r"(r.y) : "l"(p));
+  return r;
+}
+
+// 8 packed int4 channels (one word) -> biased bytes u = x + 8 of the even
+// channels (lo) and of the odd channels (hi)
+__device__ __forceinline__ uint32_t nib_lo(uint32_t w) { return (w & 0x0F0F0F0Fu) ^ 0x08080808u; }
+__device__ __forceinline__ uint32_t nib_hi(uint32_t w) { return ((w >> 4) & 0x0F0F0F0Fu) ^ 0x08080808u; }
+
+// One row piece of 16 channels as four words of four bytes: int8 cache:
+// channels 4q..4q+3 in word q (signed); int4 cache: channel groups
+// {0,2,4,6}, {1,3,5,7}, {8,..,14}, {9,..,15} (biased unsigned).
+template <bool kInt4>
+__device__ __forceinline__ uint4 load_piece(const int8_t* p, bool valid) {
+  if constexpr (kInt4) {
+    if (!valid) return make_uint4(0x08080808u, 0x08080808u, 0x08080808u, 0x08080808u);  // x = 0
+    const uint2 w = ld_stream8(p);
+    return make_uint4(nib_lo(w.x), nib_hi(w.x), nib_lo(w.y), nib_hi(w.y));
+  } else {
+    return valid ? ld_stream(p) : make_uint4(0, 0, 0, 0);
+  }
+}
+
 __device__ __forceinline__ int32_t dp4a_ss(uint32_t a, uint32_t b, int32_t c) {
   int32_t d;
   asm("dp4a.s32.s32 %0, %1, %2, %3;" : "=r"(d) : "r"(a), "r"(b), "r"(c));
@@ -59,6 +92,12 @@ __device__ __forceinline__ int32_t dp4a_ss(uint32_t a, uint32_t b, int32_t c) {
 __device__ __forceinline__ int32_t dp4a_su(uint32_t a, uint32_t b, int32_t c) {
   int32_t d;
   asm("dp4a.s32.u32 %0, %1, %2, %3;" : "=r"(d) : "r"(a), "r"(b), "r"(c));
+  return d;
+}
+
+__device__ __forceinline__ int32_t dp4a_uu(uint32_t a, uint32_t b, int32_t c) {
+  int32_t d;
+  asm("dp4a.u32.u32 %0, %1, %2, %3;" : "=r"(d) : "r"(a), "r"(b), "r"(c));
   return d;
 }
 
@@ -74,9 +113,11 @@ struct Layout {
   static_assert(kChunk % kRowsPerStep == 0, "chunk must be whole steps");
 };
 
-template <int D>
+template <int D, bool kInt4>
 __global__ void __launch_bounds__(kThreads) decode_qk_kernel(const __grid_constant__ DecodeArgs a) {
   using Lt = Layout<D>;
+  constexpr int kRowBytes = kInt4 ? D / 2 : D;
+  constexpr int kPieceBytes = kInt4 ? 8 : 16;
   const int bh = blockIdx.y;
   const int sp = blockIdx.x;
   const int j0 = sp * a.chunk;
@@ -88,8 +129,15 @@ __global__ void __launch_bounds__(kThreads) decode_qk_kernel(const __grid_consta
 
   if (sp == 0 && tid == 0) a.ws_cnt[bh] = 0u;  // ticket for decode_pv
 
-  const uint4 qv = *reinterpret_cast<const uint4*>(a.q + static_cast<size_t>(bh) * D + piece * 16);
-  const int8_t* kbase = a.k + static_cast<size_t>(bh) * a.Lmax * D + piece * 16;
+  uint4 qv = *reinterpret_cast<const uint4*>(a.q + static_cast<size_t>(bh) * D + piece * 16);
+  int32_t qbias = 0;  // 8 sum(q) over the piece (int4: dot products run on u = x + 8)
+  if constexpr (kInt4) {
+    qbias = 8 * dp4a_ss(qv.x, 0x01010101u, dp4a_ss(qv.y, 0x01010101u, dp4a_ss(qv.z, 0x01010101u,
+                                                                                 dp4a_ss(qv.w, 0x01010101u, 0))));
+    qv = make_uint4(__byte_perm(qv.x, qv.y, 0x6420), __byte_perm(qv.x, qv.y, 0x7531),
+                    __byte_perm(qv.z, qv.w, 0x6420), __byte_perm(qv.z, qv.w, 0x7531));
+  }
+  const int8_t* kbase = a.k + static_cast<size_t>(bh) * a.Lmax * kRowBytes + piece * kPieceBytes;
   int32_t* srow = a.ws_s + static_cast<size_t>(bh) * a.ld_s;
   int32_t mx = INT_MIN;
 
@@ -99,16 +147,25 @@ __global__ void __launch_bounds__(kThreads) decode_qk_kernel(const __grid_consta
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
       const int j = r0 + i;
-      kv[i] = (j < j1) ? ld_stream(kbase + static_cast<size_t>(j) * D) : make_uint4(0, 0, 0, 0);
+      kv[i] = load_piece<kInt4>(kbase + static_cast<size_t>(j) * kRowBytes, j < j1);
     }
     int32_t s[4];
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
-      int32_t acc = 0;
-      acc = dp4a_ss(kv[i].x, qv.x, acc);
-      acc = dp4a_ss(kv[i].y, qv.y, acc);
-      acc = dp4a_ss(kv[i].z, qv.z, acc);
-      acc = dp4a_ss(kv[i].w, qv.w, acc);
+      int32_t acc;
+      if constexpr (kInt4) {
+        acc = -qbias;
+        acc = dp4a_su(qv.x, kv[i].x, acc);
+        acc = dp4a_su(qv.y, kv[i].y, acc);
+        acc = dp4a_su(qv.z, kv[i].z, acc);
+        acc = dp4a_su(qv.w, kv[i].w, acc);
+      } else {
+        acc = 0;
+        acc = dp4a_ss(kv[i].x, qv.x, acc);
+        acc = dp4a_ss(kv[i].y, qv.y, acc);
+        acc = dp4a_ss(kv[i].z, qv.z, acc);
+        acc = dp4a_ss(kv[i].w, qv.w, acc);
+      }
       s[i] = acc;
     }
     // reduce the CPR partial sums of each of the 4 rows (transpose-reduce)
@@ -215,9 +272,11 @@ __global__ void __launch_bounds__(kThreads) decode_z_kernel(const __grid_constan
   }
 }
 
-template <int D>
-__global__ void __launch_bounds__(kThreads) decode_pv_kernel(const __grid_constant__ DecodeArgs a) {
+template <int D, bool kInt4>
+__global__ void __launch_bounds__(kThreads, 4) decode_pv_kernel(const __grid_constant__ DecodeArgs a) {
   using Lt = Layout<D>;
+  constexpr int kRowBytes = kInt4 ? D / 2 : D;
+  constexpr int kPieceBytes = kInt4 ? 8 : 16;
   const int bh = blockIdx.y;
   const int sp = blockIdx.x;
   const int j0 = sp * a.chunk;
@@ -247,12 +306,12 @@ __global__ void __launch_bounds__(kThreads) decode_pv_kernel(const __grid_consta
   // first step is issued before the probabilities are computed
   const int piece = tid % Lt::kCPR;
   const int grp = tid / Lt::kCPR;
-  const int8_t* vbase = a.v + static_cast<size_t>(bh) * a.Lmax * D + piece * 16;
+  const int8_t* vbase = a.v + static_cast<size_t>(bh) * a.Lmax * kRowBytes + piece * kPieceBytes;
   auto load4 = [&](int r0, uint4 (&vv)[4]) {
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
       const int j = r0 + i;
-      vv[i] = (j < j1) ? ld_stream(vbase + static_cast<size_t>(j) * D) : make_uint4(0, 0, 0, 0);
+      vv[i] = load_piece<kInt4>(vbase + static_cast<size_t>(j) * kRowBytes, j < j1);
     }
   };
   uint4 cur[4];
@@ -277,12 +336,14 @@ __global__ void __launch_bounds__(kThreads) decode_pv_kernel(const __grid_consta
   int32_t acc[16];
 #pragma unroll
   for (int c = 0; c < 16; ++c) acc[c] = 0;
+  int32_t psum = 0;  // sum of this thread's P (int4: the bias correction)
   for (int base = j0; base < j1; base += Lt::kRowsPerStep) {
     const int r0 = base + 4 * grp;
     const bool more = base + Lt::kRowsPerStep < j1;
     uint4 nxt[4];
     if (more) load4(r0 + Lt::kRowsPerStep, nxt);
     const uint32_t p4 = pk[(r0 - j0) >> 2];  // P of rows r0..r0+3, one byte each
+    if constexpr (kInt4) psum = dp4a_uu(p4, 0x01010101u, psum);
     const uint32_t* w0 = reinterpret_cast<const uint32_t*>(&cur[0]);
     const uint32_t* w1 = reinterpret_cast<const uint32_t*>(&cur[1]);
     const uint32_t* w2 = reinterpret_cast<const uint32_t*>(&cur[2]);
@@ -294,19 +355,35 @@ __global__ void __launch_bounds__(kThreads) decode_pv_kernel(const __grid_consta
       const uint32_t ab_hi = __byte_perm(w0[q], w1[q], 0x7362);
       const uint32_t cd_lo = __byte_perm(w2[q], w3[q], 0x5140);
       const uint32_t cd_hi = __byte_perm(w2[q], w3[q], 0x7362);
-      acc[4 * q + 0] = dp4a_su(__byte_perm(ab_lo, cd_lo, 0x5410), p4, acc[4 * q + 0]);
-      acc[4 * q + 1] = dp4a_su(__byte_perm(ab_lo, cd_lo, 0x7632), p4, acc[4 * q + 1]);
-      acc[4 * q + 2] = dp4a_su(__byte_perm(ab_hi, cd_hi, 0x5410), p4, acc[4 * q + 2]);
-      acc[4 * q + 3] = dp4a_su(__byte_perm(ab_hi, cd_hi, 0x7632), p4, acc[4 * q + 3]);
+      if constexpr (kInt4) {
+        acc[4 * q + 0] = dp4a_uu(__byte_perm(ab_lo, cd_lo, 0x5410), p4, acc[4 * q + 0]);
+        acc[4 * q + 1] = dp4a_uu(__byte_perm(ab_lo, cd_lo, 0x7632), p4, acc[4 * q + 1]);
+        acc[4 * q + 2] = dp4a_uu(__byte_perm(ab_hi, cd_hi, 0x5410), p4, acc[4 * q + 2]);
+        acc[4 * q + 3] = dp4a_uu(__byte_perm(ab_hi, cd_hi, 0x7632), p4, acc[4 * q + 3]);
+      } else {
+        acc[4 * q + 0] = dp4a_su(__byte_perm(ab_lo, cd_lo, 0x5410), p4, acc[4 * q + 0]);
+        acc[4 * q + 1] = dp4a_su(__byte_perm(ab_lo, cd_lo, 0x7632), p4, acc[4 * q + 1]);
+        acc[4 * q + 2] = dp4a_su(__byte_perm(ab_hi, cd_hi, 0x5410), p4, acc[4 * q + 2]);
+        acc[4 * q + 3] = dp4a_su(__byte_perm(ab_hi, cd_hi, 0x7632), p4, acc[4 * q + 3]);
+      }
     }
     if (more) {
 #pragma unroll
       for (int i = 0; i < 4; ++i) cur[i] = nxt[i];
     }
   }
-  // reduce over the row groups: column piece*16 + c
+  // reduce over the row groups: column piece*16 + c.  Slot 4g + i of acc is
+  // channel 4g + i (int8), or channel {2i, 2i+1, 8+2i, 9+2i}[g] (int4).
 #pragma unroll
-  for (int c = 0; c < 16; ++c) part[tid * 16 + c] = acc[c];
+  for (int c = 0; c < 16; ++c) {
+    if constexpr (kInt4) {
+      const int g = c >> 2, i = c & 3;
+      const int ch = (g & 2) * 4 + 2 * i + (g & 1);
+      part[tid * 16 + ch] = acc[c] - 8 * psum;
+    } else {
+      part[tid * 16 + c] = acc[c];
+    }
+  }
   __syncthreads();
   int32_t* gpart = a.ws_part + (static_cast<size_t>(bh) * a.nsplit + sp) * D;
   if (tid < D) {

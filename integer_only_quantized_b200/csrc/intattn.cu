@@ -189,16 +189,16 @@ DecodeLayout decode_layout(long long BH, int Lk, int d) {
   return L;
 }
 
-template <int D>
+template <int D, bool kInt4 = false>
 int decode_launch(const DecodeArgs& a, cudaStream_t stream) {
   const dim3 grid(a.nsplit, a.BH);
-  intattn::decode::decode_qk_kernel<D><<<grid, intattn::decode::kThreads, 0, stream>>>(a);
+  intattn::decode::decode_qk_kernel<D, kInt4><<<grid, intattn::decode::kThreads, 0, stream>>>(a);
   const int rc = note_launch(cudaGetLastError());
   if (rc != INTATTN_OK) return rc;
   intattn::decode::decode_z_kernel<D><<<a.BH, intattn::decode::kThreads, 0, stream>>>(a);
   const int rz = note_launch(cudaGetLastError());
   if (rz != INTATTN_OK) return rz;
-  intattn::decode::decode_pv_kernel<D><<<grid, intattn::decode::kThreads, 0, stream>>>(a);
+  intattn::decode::decode_pv_kernel<D, kInt4><<<grid, intattn::decode::kThreads, 0, stream>>>(a);
   return note_launch(cudaGetLastError());
 }
 
@@ -242,6 +242,51 @@ int static_scratch_address(void** out) {
   }
   *out = g_scratch_ptr[dev];
   return INTATTN_OK;
+}
+
+// Checks and kernel arguments shared by the decode entry points (the scratch
+// is filled in by the caller of this helper).
+int decode_setup(const int8_t* q, const int8_t* k_cache, const int8_t* v_cache, const intattn_scales_t* scales,
+                 int B, int H, int Lk, int Lmax, int d, float clip_c, int8_t* out, DecodeArgs* a,
+                 DecodeLayout* L, bool* empty) {
+  *empty = false;
+  if (B < 0 || H <= 0 || Lk < 1 || Lk > 65535 || Lmax < Lk) return INTATTN_ERR_INVALID_ARG;
+  if (d != 64 && d != 128) return INTATTN_ERR_UNSUPPORTED;
+  if (!scales) return INTATTN_ERR_INVALID_ARG;
+  static_assert(sizeof(DecodeArgs) <= 4096, "kernel argument block too large");
+  std::memset(a, 0, sizeof(*a));
+  int rc = derive(scales, H, d, clip_c, a->lut, a->hp, INTATTN_MAX_HEADS);
+  if (rc) return rc;
+  const long long BH = static_cast<long long>(B) * H;
+  if (BH == 0) {
+    *empty = true;
+    return INTATTN_OK;
+  }
+  if (BH > 65535) return INTATTN_ERR_UNSUPPORTED;  // grid y limit
+  if (!q || !k_cache || !v_cache || !out) return INTATTN_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k_cache) || !aligned16(v_cache)) return INTATTN_ERR_UNSUPPORTED;
+  *L = decode_layout(BH, Lk, d);
+  a->q = q;
+  a->k = k_cache;
+  a->v = v_cache;
+  a->out = out;
+  a->BH = static_cast<int32_t>(BH);
+  a->H = H;
+  a->Lk = Lk;
+  a->Lmax = Lmax;
+  a->nsplit = L->nsplit;
+  a->ld_s = L->ld_s;
+  a->chunk = intattn::decode::kChunk;
+  a->per_head = scales->per_head ? 1 : 0;
+  return INTATTN_OK;
+}
+
+void decode_scratch(DecodeArgs* a, const DecodeLayout& L, char* ws) {
+  a->ws_s = reinterpret_cast<int32_t*>(ws + L.off_s);
+  a->ws_max = reinterpret_cast<int32_t*>(ws + L.off_max);
+  a->ws_part = reinterpret_cast<int32_t*>(ws + L.off_part);
+  a->ws_cnt = reinterpret_cast<uint32_t*>(ws + L.off_cnt);  // zeroed by the first kernel of each call
+  a->ws_mr = reinterpret_cast<int32_t*>(ws + L.off_mr);
 }
 
 }  // namespace
@@ -315,83 +360,48 @@ size_t intattn_decode_workspace_size(int B, int H, int Lk, int d) {
 int intattn_decode(const int8_t* q, const int8_t* k_cache, const int8_t* v_cache, const intattn_scales_t* scales,
                    int B, int H, int Lk, int Lmax, int d, float clip_c, int8_t* out, void* workspace,
                    size_t workspace_bytes, intattn_stream_t stream) {
-  if (B < 0 || H <= 0 || Lk < 1 || Lk > 65535 || Lmax < Lk) return INTATTN_ERR_INVALID_ARG;
-  if (d != 64 && d != 128) return INTATTN_ERR_UNSUPPORTED;
-  if (!scales) return INTATTN_ERR_INVALID_ARG;
-  static_assert(sizeof(DecodeArgs) <= 4096, "kernel argument block too large");
   DecodeArgs a;
-  std::memset(&a, 0, sizeof(a));
-  int rc = derive(scales, H, d, clip_c, a.lut, a.hp, INTATTN_MAX_HEADS);
-  if (rc) return rc;
-  const long long BH = static_cast<long long>(B) * H;
-  if (BH == 0) return INTATTN_OK;
-  if (BH > 65535) return INTATTN_ERR_UNSUPPORTED;  // grid y limit
-  if (!q || !k_cache || !v_cache || !out) return INTATTN_ERR_INVALID_ARG;
-  if (!aligned16(q) || !aligned16(k_cache) || !aligned16(v_cache)) return INTATTN_ERR_UNSUPPORTED;
-  const DecodeLayout L = decode_layout(BH, Lk, d);
+  DecodeLayout L{};
+  bool empty = false;
+  int rc = decode_setup(q, k_cache, v_cache, scales, B, H, Lk, Lmax, d, clip_c, out, &a, &L, &empty);
+  if (rc || empty) return rc;
   if (!workspace || workspace_bytes < L.total || (reinterpret_cast<uintptr_t>(workspace) & 255u))
     return INTATTN_ERR_WORKSPACE;
-  char* ws = static_cast<char*>(workspace);
-  a.q = q;
-  a.k = k_cache;
-  a.v = v_cache;
-  a.out = out;
-  a.ws_s = reinterpret_cast<int32_t*>(ws + L.off_s);
-  a.ws_max = reinterpret_cast<int32_t*>(ws + L.off_max);
-  a.ws_part = reinterpret_cast<int32_t*>(ws + L.off_part);
-  a.ws_cnt = reinterpret_cast<uint32_t*>(ws + L.off_cnt);
-  a.ws_mr = reinterpret_cast<int32_t*>(ws + L.off_mr);
-  a.BH = static_cast<int32_t>(BH);
-  a.H = H;
-  a.Lk = Lk;
-  a.Lmax = Lmax;
-  a.nsplit = L.nsplit;
-  a.ld_s = L.ld_s;
-  a.chunk = intattn::decode::kChunk;
-  a.per_head = scales->per_head ? 1 : 0;
+  decode_scratch(&a, L, static_cast<char*>(workspace));
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   return d == 64 ? decode_launch<64>(a, st) : decode_launch<128>(a, st);
+}
+
+int intattn_decode_int4(const int8_t* q, const uint8_t* k_cache, const uint8_t* v_cache,
+                        const intattn_scales_t* scales, int B, int H, int Lk, int Lmax, int d, float clip_c,
+                        int8_t* out, void* workspace, size_t workspace_bytes, intattn_stream_t stream) {
+  DecodeArgs a;
+  DecodeLayout L{};
+  bool empty = false;
+  int rc = decode_setup(q, reinterpret_cast<const int8_t*>(k_cache), reinterpret_cast<const int8_t*>(v_cache),
+                        scales, B, H, Lk, Lmax, d, clip_c, out, &a, &L, &empty);
+  if (rc || empty) return rc;
+  if (!workspace || workspace_bytes < L.total || (reinterpret_cast<uintptr_t>(workspace) & 255u))
+    return INTATTN_ERR_WORKSPACE;
+  decode_scratch(&a, L, static_cast<char*>(workspace));
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  return d == 64 ? decode_launch<64, true>(a, st) : decode_launch<128, true>(a, st);
 }
 
 int intattn_decode_static_scratch(const int8_t* q, const int8_t* k_cache, const int8_t* v_cache,
                                   const intattn_scales_t* scales, int B, int H, int Lk, int Lmax, int d,
                                   float clip_c, int8_t* out, intattn_stream_t stream) {
   // same checks and kernels as intattn_decode; only the scratch differs
-  if (B < 0 || H <= 0 || Lk < 1 || Lk > 65535 || Lmax < Lk) return INTATTN_ERR_INVALID_ARG;
-  if (d != 64 && d != 128) return INTATTN_ERR_UNSUPPORTED;
-  if (!scales) return INTATTN_ERR_INVALID_ARG;
   DecodeArgs a;
-  std::memset(&a, 0, sizeof(a));
-  int rc = derive(scales, H, d, clip_c, a.lut, a.hp, INTATTN_MAX_HEADS);
-  if (rc) return rc;
-  const long long BH = static_cast<long long>(B) * H;
-  if (BH == 0) return INTATTN_OK;
-  if (BH > 65535) return INTATTN_ERR_UNSUPPORTED;
-  if (!q || !k_cache || !v_cache || !out) return INTATTN_ERR_INVALID_ARG;
-  if (!aligned16(q) || !aligned16(k_cache) || !aligned16(v_cache)) return INTATTN_ERR_UNSUPPORTED;
-  const DecodeLayout L = decode_layout(BH, Lk, d);
+  DecodeLayout L{};
+  bool empty = false;
+  int rc = decode_setup(q, k_cache, v_cache, scales, B, H, Lk, Lmax, d, clip_c, out, &a, &L, &empty);
+  if (rc || empty) return rc;
   if (L.total > static_cast<size_t>(INTATTN_STATIC_SCRATCH_BYTES)) return INTATTN_ERR_WORKSPACE;
   void* scratch = nullptr;
   rc = static_scratch_address(&scratch);
   if (rc) return rc;
-  char* ws = static_cast<char*>(scratch);
-  a.q = q;
-  a.k = k_cache;
-  a.v = v_cache;
-  a.out = out;
-  a.ws_s = reinterpret_cast<int32_t*>(ws + L.off_s);
-  a.ws_max = reinterpret_cast<int32_t*>(ws + L.off_max);
-  a.ws_part = reinterpret_cast<int32_t*>(ws + L.off_part);
-  a.ws_cnt = reinterpret_cast<uint32_t*>(ws + L.off_cnt);  // zeroed by the first kernel of each call
-  a.ws_mr = reinterpret_cast<int32_t*>(ws + L.off_mr);
-  a.BH = static_cast<int32_t>(BH);
-  a.H = H;
-  a.Lk = Lk;
-  a.Lmax = Lmax;
-  a.nsplit = L.nsplit;
-  a.ld_s = L.ld_s;
-  a.chunk = intattn::decode::kChunk;
-  a.per_head = scales->per_head ? 1 : 0;
+  decode_scratch(&a, L, static_cast<char*>(scratch));
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   return d == 64 ? decode_launch<64>(a, st) : decode_launch<128>(a, st);
 }

@@ -53,6 +53,7 @@ class Workload:
     clip_c: float
     decode: bool = False
     Lmax: int = 0              # decode: cache capacity (rows per (b, h))
+    kv_bits: int = 8           # 4: K and V codes in [-7, 7], stored as packed nibbles
 
     @property
     def seed(self) -> int:
@@ -67,8 +68,13 @@ class Workload:
     @property
     def decode_bytes(self) -> int:
         """K and V cache rows read plus the q and out vectors."""
-        kv = 2 * self.B * self.H * self.Lk * self.d
+        kv = 2 * self.B * self.H * self.Lk * self.d * self.kv_bits // 8
         return kv + 2 * self.B * self.H * self.d
+
+    @property
+    def kv_qmax(self) -> int:
+        """Largest K/V code magnitude of the symmetric quantisation."""
+        return 7 if self.kv_bits == 4 else 127
 
 
 WORKLOADS = {
@@ -86,6 +92,8 @@ WORKLOADS = {
                  "normal", 0.01, 16.0, "k", True, 10.0),
         Workload("llama7b_decode_b64_lk4096", 5, 64, 32, 1, 4096, 128, False,
                  "normal", 0.01, 16.0, "k", True, 10.0, decode=True, Lmax=4096),
+        Workload("llama7b_decode_int4_b64_lk4096", 6, 64, 32, 1, 4096, 128, False,
+                 "normal", 0.01, 16.0, "k", True, 10.0, decode=True, Lmax=4096, kv_bits=4),
     ]
 }
 
@@ -95,10 +103,10 @@ def custom_workload(name: str, B: int, H: int, Lq: int, Lk: int, d: int,
                     dist: str = "normal", outlier_frac: float = 0.02,
                     outlier_scale: float = 8.0, outlier_tensors: str = "qkv",
                     index: int = 100, decode: bool = False,
-                    Lmax: int = 0) -> Workload:
+                    Lmax: int = 0, kv_bits: int = 8) -> Workload:
     return Workload(name, index, B, H, Lq, Lk, d, causal, dist, outlier_frac,
                     outlier_scale, outlier_tensors, per_head, clip_c, decode,
-                    Lmax if Lmax else Lk)
+                    Lmax if Lmax else Lk, kv_bits)
 
 
 @dataclasses.dataclass
@@ -145,21 +153,22 @@ def _tensor_chunks(w: Workload, which: str, L: int, nthreads: int):
             yield b, x
 
 
-def _quantise(w: Workload, which: str, L: int, nthreads: int):
-    """Two passes over the seeded chunks: max|x| first, then int8 codes."""
+def _quantise(w: Workload, which: str, L: int, nthreads: int, qmax: int = 127):
+    """Two passes over the seeded chunks: max|x| first, then codes in
+    [-qmax, qmax] (int8 storage)."""
     amax = np.zeros(w.H, dtype=np.float64)
     for _, x in _tensor_chunks(w, which, L, nthreads):
         amax = np.maximum(amax, np.abs(x).max(axis=(1, 2)).astype(np.float64))
     if not w.per_head:
         amax = np.array([amax.max()])
-    scale = (amax / 127.0).astype(np.float32)
+    scale = (amax / float(qmax)).astype(np.float32)
     scale[scale == 0] = np.float32(1.0)
     out = np.empty((w.B, w.H, L, w.d), dtype=np.int8)
     sc = scale.astype(np.float64)
     sc_h = sc if w.per_head else np.repeat(sc, w.H)
     for b, x in _tensor_chunks(w, which, L, nthreads):
         y = np.rint(x.astype(np.float64) / sc_h[:, None, None])
-        out[b] = np.clip(y, -127, 127).astype(np.int8)
+        out[b] = np.clip(y, -qmax, qmax).astype(np.int8)
     return out, scale
 
 
@@ -200,10 +209,31 @@ def _output_scale(w: Workload, q, k, v, s_q, s_k, s_v) -> np.ndarray:
 def make_inputs(w: Workload, nthreads: int = 8) -> Inputs:
     Lkv = w.Lmax if w.decode else w.Lk
     q, s_q = _quantise(w, "q", w.Lq, nthreads)
-    k, s_k = _quantise(w, "k", Lkv, nthreads)
-    v, s_v = _quantise(w, "v", Lkv, nthreads)
+    k, s_k = _quantise(w, "k", Lkv, nthreads, w.kv_qmax)
+    v, s_v = _quantise(w, "v", Lkv, nthreads, w.kv_qmax)
     s_o = _output_scale(w, q, k, v, s_q, s_k, s_v)
     return Inputs(w, q, k, v, s_q, s_k, s_v, s_o)
+
+
+def pack_int4(x: np.ndarray) -> np.ndarray:
+    """int8 codes in [-8, 7], [..., d] -> uint8 [..., d/2]: byte t holds
+    channel 2t in bits 0-3 and channel 2t+1 in bits 4-7 (two's complement)."""
+    x = np.asarray(x)
+    if x.shape[-1] % 2 or x.min(initial=0) < -8 or x.max(initial=0) > 7:
+        raise ValueError("int4 packing needs an even last dimension and codes in [-8, 7]")
+    u = x.astype(np.uint8) & np.uint8(0x0F)
+    return (u[..., 0::2] | (u[..., 1::2] << np.uint8(4))).astype(np.uint8)
+
+
+def unpack_int4(p: np.ndarray) -> np.ndarray:
+    """Inverse of pack_int4: uint8 [..., d/2] -> int8 codes [..., d]."""
+    p = np.asarray(p, dtype=np.uint8)
+    lo = (p & np.uint8(0x0F)).astype(np.int16)
+    hi = (p >> np.uint8(4)).astype(np.int16)
+    out = np.empty(p.shape[:-1] + (2 * p.shape[-1],), dtype=np.int16)
+    out[..., 0::2] = lo
+    out[..., 1::2] = hi
+    return np.where(out >= 8, out - 16, out).astype(np.int8)
 
 
 @dataclasses.dataclass
@@ -228,7 +258,7 @@ def make_inputs_torch(w: Workload, device) -> DeviceInputs:
     g.manual_seed(w.seed)
     Lkv = w.Lmax if w.decode else w.Lk
 
-    def one(which, L):
+    def one(which, L, qmax=127):
         x = torch.randn((w.B, w.H, L, w.d), generator=g, device=device, dtype=torch.float32)
         if w.dist == "student_t4":
             chi = torch.randn((4, w.B, w.H, L, w.d), generator=g, device=device).pow(2).sum(0)
@@ -241,15 +271,15 @@ def make_inputs_torch(w: Workload, device) -> DeviceInputs:
         amax = x.abs().amax(dim=(0, 2, 3)).double()
         if not w.per_head:
             amax = amax.max().reshape(1)
-        scale = (amax / 127.0).float()
+        scale = (amax / float(qmax)).float()
         scale[scale == 0] = 1.0
         sh = scale.double() if w.per_head else scale.double().expand(w.H)
-        q = torch.clamp(torch.round(x.double() / sh.view(1, -1, 1, 1)), -127, 127).to(torch.int8)
+        q = torch.clamp(torch.round(x.double() / sh.view(1, -1, 1, 1)), -qmax, qmax).to(torch.int8)
         return q, scale.cpu().numpy().astype(np.float32)
 
     q, s_q = one("q", w.Lq)
-    k, s_k = one("k", Lkv)
-    v, s_v = one("v", Lkv)
+    k, s_k = one("k", Lkv, w.kv_qmax)
+    v, s_v = one("v", Lkv, w.kv_qmax)
     # output scale from an fp64 row sample, as in make_inputs
     rows = torch.as_tensor(_sample_rows(w.Lq), device=device)
     sq = torch.as_tensor(np.array(np.broadcast_to(s_q, (w.H,))) if w.per_head else np.full(w.H, s_q[0]),
@@ -274,3 +304,10 @@ def make_inputs_torch(w: Workload, device) -> DeviceInputs:
     s_o = (amax / 127.0).float().cpu().numpy().astype(np.float32)
     s_o[s_o == 0] = np.float32(1.0)
     return DeviceInputs(w, q.contiguous(), k.contiguous(), v.contiguous(), s_q, s_k, s_v, s_o)
+
+
+def pack_int4_torch(x):
+    """pack_int4 for a torch int8 tensor on any device (same byte layout)."""
+    import torch
+    u = (x.to(torch.int16) & 0x0F).to(torch.uint8)
+    return (u[..., 0::2] | (u[..., 1::2] << 4)).contiguous()

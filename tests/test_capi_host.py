@@ -23,7 +23,7 @@ def ia():
 def _declared_functions():
     src = open(os.path.join(ROOT, "include", "intattn.h")).read()
     src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
-    return sorted(set(re.findall(r"\b(intattn_[a-z_]+)\s*\(", src)))
+    return sorted(set(re.findall(r"\b(intattn_[a-z0-9_]+)\s*\(", src)))
 
 
 def test_library_exports_every_declared_function(ia):
