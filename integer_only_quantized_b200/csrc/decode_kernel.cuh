@@ -1,5 +1,5 @@
-// Decode kernels: one query per (batch, head) against an int8 or int4 KV
-// cache.
+// Decode kernels: one query per (batch, head) against an int8 or a packed
+// int4 KV cache.
 //
 // Same integer definition as the prefill path with Lq = 1 and no mask.  The
 // work is an HBM stream of the K and V rows (2*Lk*d bytes per (b, h)), so it
@@ -14,13 +14,13 @@
 //              The last CTA of a (b, h) (atomic ticket) adds the partials and
 //              requantises.  Integer addition is associative, so the result
 //              does not depend on the order.
-// int4 cache (kInt4): rows of D/2 bytes, byte t holding channel 2t in bits
-// 0-3 and channel 2t+1 in bits 4-7, each a two's-complement value in
-// [-8, 7].  A thread unpacks its 8-byte piece (16 channels) into the biased
-// unsigned bytes u = x + 8 ((nibble ^ 8), one logic op per 4 channels), in
-// the channel order {0,2,4,6} {1,3,5,7} {8,..,14} {9,..,15}; dp4a then works
-// on u and the bias is removed exactly: q.x = q.u - 8 sum(q), and
-// sum P x = sum P u - 8 sum(P).
+// The int4 cache (decode4_qk / decode_z / decode4_pv) has rows of D/2 bytes,
+// byte t holding channel 2t in bits 0-3 and channel 2t+1 in bits 4-7, each a
+// two's-complement value in [-8, 7].  A thread streams 16-byte pieces (32
+// channels) and unpacks each 8-channel word into the biased unsigned bytes
+// u = x + 8 of its even and of its odd channels (nibble ^ 8: one logic op
+// per 4 channels); dp4a works on u and the bias is removed exactly:
+// q.x = q.u - 8 sum(q), and sum P x = sum P u - 8 sum(P).
 #pragma once
 #include <climits>
 #include <cstdint>
@@ -48,7 +48,8 @@ struct DecodeArgs {
 namespace decode {
 
 constexpr int kThreads = 256;
-constexpr int kChunk = 512;  // keys per CTA (multiple of the rows one step covers)
+constexpr int kChunk = 512;    // keys per CTA, int8 cache (multiple of the rows one step covers)
+constexpr int kChunk4 = 2048;  // keys per CTA, int4 cache (the same bytes as 1024 int8 rows)
 
 __device__ __forceinline__ uint4 ld_stream(const void* p) {
   uint4 r;
@@ -62,25 +63,6 @@ __device__ __forceinline__ uint2 ld_stream8(const void* p) {
   uint2 r;
   asm volatile("ld.global.nc.L1::no_allocate.v2.u32 {%0, %1}, [%2];" : "=r"(r.x), "=r"(r.y) : "l"(p));
   return r;
-}
-
-// 8 packed int4 channels (one word) -> biased bytes u = x + 8 of the even
-// channels (lo) and of the odd channels (hi)
-__device__ __forceinline__ uint32_t nib_lo(uint32_t w) { return (w & 0x0F0F0F0Fu) ^ 0x08080808u; }
-__device__ __forceinline__ uint32_t nib_hi(uint32_t w) { return ((w >> 4) & 0x0F0F0F0Fu) ^ 0x08080808u; }
-
-// One row piece of 16 channels as four words of four bytes: int8 cache:
-// channels 4q..4q+3 in word q (signed); int4 cache: channel groups
-// {0,2,4,6}, {1,3,5,7}, {8,..,14}, {9,..,15} (biased unsigned).
-template <bool kInt4>
-__device__ __forceinline__ uint4 load_piece(const int8_t* p, bool valid) {
-  if constexpr (kInt4) {
-    if (!valid) return make_uint4(0x08080808u, 0x08080808u, 0x08080808u, 0x08080808u);  // x = 0
-    const uint2 w = ld_stream8(p);
-    return make_uint4(nib_lo(w.x), nib_hi(w.x), nib_lo(w.y), nib_hi(w.y));
-  } else {
-    return valid ? ld_stream(p) : make_uint4(0, 0, 0, 0);
-  }
 }
 
 __device__ __forceinline__ int32_t dp4a_ss(uint32_t a, uint32_t b, int32_t c) {
@@ -101,6 +83,11 @@ __device__ __forceinline__ int32_t dp4a_uu(uint32_t a, uint32_t b, int32_t c) {
   return d;
 }
 
+// 8 packed int4 channels (one word) -> biased bytes u = x + 8 of the even
+// channels (lo) and of the odd channels (hi)
+__device__ __forceinline__ uint32_t nib_lo(uint32_t w) { return (w & 0x0F0F0F0Fu) ^ 0x08080808u; }
+__device__ __forceinline__ uint32_t nib_hi(uint32_t w) { return ((w >> 4) & 0x0F0F0F0Fu) ^ 0x08080808u; }
+
 __device__ __forceinline__ int32_t imax32(int32_t a, int32_t b) { return a > b ? a : b; }
 
 // Thread layout shared by both kernels: CPR = D/16 threads cover one row in
@@ -113,11 +100,9 @@ struct Layout {
   static_assert(kChunk % kRowsPerStep == 0, "chunk must be whole steps");
 };
 
-template <int D, bool kInt4>
+template <int D>
 __global__ void __launch_bounds__(kThreads) decode_qk_kernel(const __grid_constant__ DecodeArgs a) {
   using Lt = Layout<D>;
-  constexpr int kRowBytes = kInt4 ? D / 2 : D;
-  constexpr int kPieceBytes = kInt4 ? 8 : 16;
   const int bh = blockIdx.y;
   const int sp = blockIdx.x;
   const int j0 = sp * a.chunk;
@@ -129,15 +114,8 @@ __global__ void __launch_bounds__(kThreads) decode_qk_kernel(const __grid_consta
 
   if (sp == 0 && tid == 0) a.ws_cnt[bh] = 0u;  // ticket for decode_pv
 
-  uint4 qv = *reinterpret_cast<const uint4*>(a.q + static_cast<size_t>(bh) * D + piece * 16);
-  int32_t qbias = 0;  // 8 sum(q) over the piece (int4: dot products run on u = x + 8)
-  if constexpr (kInt4) {
-    qbias = 8 * dp4a_ss(qv.x, 0x01010101u, dp4a_ss(qv.y, 0x01010101u, dp4a_ss(qv.z, 0x01010101u,
-                                                                                 dp4a_ss(qv.w, 0x01010101u, 0))));
-    qv = make_uint4(__byte_perm(qv.x, qv.y, 0x6420), __byte_perm(qv.x, qv.y, 0x7531),
-                    __byte_perm(qv.z, qv.w, 0x6420), __byte_perm(qv.z, qv.w, 0x7531));
-  }
-  const int8_t* kbase = a.k + static_cast<size_t>(bh) * a.Lmax * kRowBytes + piece * kPieceBytes;
+  const uint4 qv = *reinterpret_cast<const uint4*>(a.q + static_cast<size_t>(bh) * D + piece * 16);
+  const int8_t* kbase = a.k + static_cast<size_t>(bh) * a.Lmax * D + piece * 16;
   int32_t* srow = a.ws_s + static_cast<size_t>(bh) * a.ld_s;
   int32_t mx = INT_MIN;
 
@@ -147,25 +125,16 @@ __global__ void __launch_bounds__(kThreads) decode_qk_kernel(const __grid_consta
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
       const int j = r0 + i;
-      kv[i] = load_piece<kInt4>(kbase + static_cast<size_t>(j) * kRowBytes, j < j1);
+      kv[i] = (j < j1) ? ld_stream(kbase + static_cast<size_t>(j) * D) : make_uint4(0, 0, 0, 0);
     }
     int32_t s[4];
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
-      int32_t acc;
-      if constexpr (kInt4) {
-        acc = -qbias;
-        acc = dp4a_su(qv.x, kv[i].x, acc);
-        acc = dp4a_su(qv.y, kv[i].y, acc);
-        acc = dp4a_su(qv.z, kv[i].z, acc);
-        acc = dp4a_su(qv.w, kv[i].w, acc);
-      } else {
-        acc = 0;
-        acc = dp4a_ss(kv[i].x, qv.x, acc);
-        acc = dp4a_ss(kv[i].y, qv.y, acc);
-        acc = dp4a_ss(kv[i].z, qv.z, acc);
-        acc = dp4a_ss(kv[i].w, qv.w, acc);
-      }
+      int32_t acc = 0;
+      acc = dp4a_ss(kv[i].x, qv.x, acc);
+      acc = dp4a_ss(kv[i].y, qv.y, acc);
+      acc = dp4a_ss(kv[i].z, qv.z, acc);
+      acc = dp4a_ss(kv[i].w, qv.w, acc);
       s[i] = acc;
     }
     // reduce the CPR partial sums of each of the 4 rows (transpose-reduce)
@@ -272,11 +241,9 @@ __global__ void __launch_bounds__(kThreads) decode_z_kernel(const __grid_constan
   }
 }
 
-template <int D, bool kInt4>
-__global__ void __launch_bounds__(kThreads, 4) decode_pv_kernel(const __grid_constant__ DecodeArgs a) {
+template <int D>
+__global__ void __launch_bounds__(kThreads) decode_pv_kernel(const __grid_constant__ DecodeArgs a) {
   using Lt = Layout<D>;
-  constexpr int kRowBytes = kInt4 ? D / 2 : D;
-  constexpr int kPieceBytes = kInt4 ? 8 : 16;
   const int bh = blockIdx.y;
   const int sp = blockIdx.x;
   const int j0 = sp * a.chunk;
@@ -306,12 +273,12 @@ __global__ void __launch_bounds__(kThreads, 4) decode_pv_kernel(const __grid_con
   // first step is issued before the probabilities are computed
   const int piece = tid % Lt::kCPR;
   const int grp = tid / Lt::kCPR;
-  const int8_t* vbase = a.v + static_cast<size_t>(bh) * a.Lmax * kRowBytes + piece * kPieceBytes;
+  const int8_t* vbase = a.v + static_cast<size_t>(bh) * a.Lmax * D + piece * 16;
   auto load4 = [&](int r0, uint4 (&vv)[4]) {
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
       const int j = r0 + i;
-      vv[i] = load_piece<kInt4>(vbase + static_cast<size_t>(j) * kRowBytes, j < j1);
+      vv[i] = (j < j1) ? ld_stream(vbase + static_cast<size_t>(j) * D) : make_uint4(0, 0, 0, 0);
     }
   };
   uint4 cur[4];
@@ -336,14 +303,12 @@ __global__ void __launch_bounds__(kThreads, 4) decode_pv_kernel(const __grid_con
   int32_t acc[16];
 #pragma unroll
   for (int c = 0; c < 16; ++c) acc[c] = 0;
-  int32_t psum = 0;  // sum of this thread's P (int4: the bias correction)
   for (int base = j0; base < j1; base += Lt::kRowsPerStep) {
     const int r0 = base + 4 * grp;
     const bool more = base + Lt::kRowsPerStep < j1;
     uint4 nxt[4];
     if (more) load4(r0 + Lt::kRowsPerStep, nxt);
     const uint32_t p4 = pk[(r0 - j0) >> 2];  // P of rows r0..r0+3, one byte each
-    if constexpr (kInt4) psum = dp4a_uu(p4, 0x01010101u, psum);
     const uint32_t* w0 = reinterpret_cast<const uint32_t*>(&cur[0]);
     const uint32_t* w1 = reinterpret_cast<const uint32_t*>(&cur[1]);
     const uint32_t* w2 = reinterpret_cast<const uint32_t*>(&cur[2]);
@@ -355,34 +320,274 @@ __global__ void __launch_bounds__(kThreads, 4) decode_pv_kernel(const __grid_con
       const uint32_t ab_hi = __byte_perm(w0[q], w1[q], 0x7362);
       const uint32_t cd_lo = __byte_perm(w2[q], w3[q], 0x5140);
       const uint32_t cd_hi = __byte_perm(w2[q], w3[q], 0x7362);
-      if constexpr (kInt4) {
-        acc[4 * q + 0] = dp4a_uu(__byte_perm(ab_lo, cd_lo, 0x5410), p4, acc[4 * q + 0]);
-        acc[4 * q + 1] = dp4a_uu(__byte_perm(ab_lo, cd_lo, 0x7632), p4, acc[4 * q + 1]);
-        acc[4 * q + 2] = dp4a_uu(__byte_perm(ab_hi, cd_hi, 0x5410), p4, acc[4 * q + 2]);
-        acc[4 * q + 3] = dp4a_uu(__byte_perm(ab_hi, cd_hi, 0x7632), p4, acc[4 * q + 3]);
-      } else {
-        acc[4 * q + 0] = dp4a_su(__byte_perm(ab_lo, cd_lo, 0x5410), p4, acc[4 * q + 0]);
-        acc[4 * q + 1] = dp4a_su(__byte_perm(ab_lo, cd_lo, 0x7632), p4, acc[4 * q + 1]);
-        acc[4 * q + 2] = dp4a_su(__byte_perm(ab_hi, cd_hi, 0x5410), p4, acc[4 * q + 2]);
-        acc[4 * q + 3] = dp4a_su(__byte_perm(ab_hi, cd_hi, 0x7632), p4, acc[4 * q + 3]);
-      }
+      acc[4 * q + 0] = dp4a_su(__byte_perm(ab_lo, cd_lo, 0x5410), p4, acc[4 * q + 0]);
+      acc[4 * q + 1] = dp4a_su(__byte_perm(ab_lo, cd_lo, 0x7632), p4, acc[4 * q + 1]);
+      acc[4 * q + 2] = dp4a_su(__byte_perm(ab_hi, cd_hi, 0x5410), p4, acc[4 * q + 2]);
+      acc[4 * q + 3] = dp4a_su(__byte_perm(ab_hi, cd_hi, 0x7632), p4, acc[4 * q + 3]);
     }
     if (more) {
 #pragma unroll
       for (int i = 0; i < 4; ++i) cur[i] = nxt[i];
     }
   }
-  // reduce over the row groups: column piece*16 + c.  Slot 4g + i of acc is
-  // channel 4g + i (int8), or channel {2i, 2i+1, 8+2i, 9+2i}[g] (int4).
+  // reduce over the row groups: column piece*16 + c
 #pragma unroll
-  for (int c = 0; c < 16; ++c) {
-    if constexpr (kInt4) {
-      const int g = c >> 2, i = c & 3;
-      const int ch = (g & 2) * 4 + 2 * i + (g & 1);
-      part[tid * 16 + ch] = acc[c] - 8 * psum;
-    } else {
-      part[tid * 16 + c] = acc[c];
+  for (int c = 0; c < 16; ++c) part[tid * 16 + c] = acc[c];
+  __syncthreads();
+  int32_t* gpart = a.ws_part + (static_cast<size_t>(bh) * a.nsplit + sp) * D;
+  if (tid < D) {
+    const int pc = tid / 16, c = tid % 16;
+    int32_t sum = 0;
+    for (int g = 0; g < Lt::kGroups; ++g) sum += part[(g * Lt::kCPR + pc) * 16 + c];
+    gpart[tid] = sum;
+  }
+  // the last CTA of this (b, h) adds the partials and requantises
+  __threadfence();
+  __syncthreads();
+  if (tid == 0) {
+    const unsigned prev = atomicAdd(a.ws_cnt + bh, 1u);
+    last_flag = (prev == static_cast<unsigned>(a.nsplit - 1));
+  }
+  __syncthreads();
+  if (last_flag) {
+    __threadfence();
+    if (tid < D) {
+      int32_t tot = 0;
+      const int32_t* p0 = a.ws_part + static_cast<size_t>(bh) * a.nsplit * D + tid;
+      for (int i = 0; i < a.nsplit; ++i) tot += __ldcg(p0 + static_cast<size_t>(i) * D);
+      const long long t = static_cast<long long>(tot) * hp.Mo + (1ll << (hp.so - 1));
+      long long y = t >> hp.so;
+      y = y > 127 ? 127 : (y < -127 ? -127 : y);
+      a.out[static_cast<size_t>(bh) * D + tid] = static_cast<int8_t>(y);
     }
+    if (tid == 0) a.ws_cnt[bh] = 0u;
+  }
+}
+
+
+// ------------------------------------------------------------ int4 cache
+// Thread layout: CPR = D/32 threads cover one row in 16-byte pieces (32
+// channels); a thread handles 4 rows (a "quad") per step.
+template <int D>
+struct Layout4 {
+  static constexpr int kCPR = D / 32;
+  static constexpr int kGroups = kThreads / kCPR;
+  static constexpr int kRowsPerStep = 4 * kGroups;  // 256 (d=128) or 512 (d=64)
+  static_assert(kChunk4 % kRowsPerStep == 0, "chunk must be whole steps");
+};
+
+template <int D>
+__global__ void __launch_bounds__(kThreads) decode4_qk_kernel(const __grid_constant__ DecodeArgs a) {
+  using Lt = Layout4<D>;
+  constexpr int kRowBytes = D / 2;
+  const int bh = blockIdx.y;
+  const int sp = blockIdx.x;
+  const int j0 = sp * a.chunk;
+  const int j1 = min(a.Lk, j0 + a.chunk);
+  const int tid = threadIdx.x;
+  const int piece = tid % Lt::kCPR;
+  const int grp = tid / Lt::kCPR;
+  const int lane = tid & 31;
+
+  if (sp == 0 && tid == 0) a.ws_cnt[bh] = 0u;  // ticket for decode4_pv
+
+  // q over this piece's 32 channels, as even / odd channel words of each
+  // 8-channel group (the order the unpacked K words come in)
+  const uint4 qa = *reinterpret_cast<const uint4*>(a.q + static_cast<size_t>(bh) * D + piece * 32);
+  const uint4 qb = *reinterpret_cast<const uint4*>(a.q + static_cast<size_t>(bh) * D + piece * 32 + 16);
+  const uint32_t qw[8] = {__byte_perm(qa.x, qa.y, 0x6420), __byte_perm(qa.x, qa.y, 0x7531),
+                          __byte_perm(qa.z, qa.w, 0x6420), __byte_perm(qa.z, qa.w, 0x7531),
+                          __byte_perm(qb.x, qb.y, 0x6420), __byte_perm(qb.x, qb.y, 0x7531),
+                          __byte_perm(qb.z, qb.w, 0x6420), __byte_perm(qb.z, qb.w, 0x7531)};
+  const int32_t qbias =
+      8 * dp4a_ss(qa.x, 0x01010101u, dp4a_ss(qa.y, 0x01010101u, dp4a_ss(qa.z, 0x01010101u, dp4a_ss(qa.w, 0x01010101u,
+      dp4a_ss(qb.x, 0x01010101u, dp4a_ss(qb.y, 0x01010101u, dp4a_ss(qb.z, 0x01010101u, dp4a_ss(qb.w, 0x01010101u, 0))))))));
+  const int8_t* kbase = a.k + static_cast<size_t>(bh) * a.Lmax * kRowBytes + piece * 16;
+  int32_t* srow = a.ws_s + static_cast<size_t>(bh) * a.ld_s;
+  int32_t mx = INT_MIN;
+
+  for (int base = j0; base < j1; base += Lt::kRowsPerStep) {
+    const int r0 = base + 4 * grp;
+    uint4 kv[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const int j = r0 + i;
+      kv[i] = (j < j1) ? ld_stream(kbase + static_cast<size_t>(j) * kRowBytes) : make_uint4(0, 0, 0, 0);
+    }
+    int32_t s[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const uint32_t w[4] = {kv[i].x, kv[i].y, kv[i].z, kv[i].w};
+      int32_t acc = -qbias;
+#pragma unroll
+      for (int g = 0; g < 4; ++g) {
+        acc = dp4a_su(qw[2 * g], nib_lo(w[g]), acc);
+        acc = dp4a_su(qw[2 * g + 1], nib_hi(w[g]), acc);
+      }
+      s[i] = acc;
+    }
+    // reduce the CPR partial sums of each of the 4 rows (transpose-reduce)
+    if constexpr (Lt::kCPR == 4) {
+      const bool b1 = lane & 2;
+      const int32_t send0 = b1 ? s[0] : s[2], send1 = b1 ? s[1] : s[3];
+      const int32_t keep0 = b1 ? s[2] : s[0], keep1 = b1 ? s[3] : s[1];
+      const int32_t u0 = keep0 + __shfl_xor_sync(0xffffffffu, send0, 2);
+      const int32_t u1 = keep1 + __shfl_xor_sync(0xffffffffu, send1, 2);
+      const bool b0 = lane & 1;
+      const int32_t send = b0 ? u0 : u1, keep = b0 ? u1 : u0;
+      const int32_t row_val = keep + __shfl_xor_sync(0xffffffffu, send, 1);
+      const int j = r0 + (b1 ? 2 : 0) + (b0 ? 1 : 0);
+      if (j < j1) {
+        srow[j] = row_val;
+        mx = imax32(mx, row_val);
+      }
+    } else {  // CPR == 2: lane pair (2g, 2g+1) holds rows (0,1) / (2,3) after one exchange
+      const bool b0 = lane & 1;
+      const int32_t send0 = b0 ? s[0] : s[2], send1 = b0 ? s[1] : s[3];
+      const int32_t keep0 = b0 ? s[2] : s[0], keep1 = b0 ? s[3] : s[1];
+      const int32_t u0 = keep0 + __shfl_xor_sync(0xffffffffu, send0, 1);
+      const int32_t u1 = keep1 + __shfl_xor_sync(0xffffffffu, send1, 1);
+      const int j = r0 + (b0 ? 2 : 0);
+      if (j < j1) {
+        srow[j] = u0;
+        mx = imax32(mx, u0);
+      }
+      if (j + 1 < j1) {
+        srow[j + 1] = u1;
+        mx = imax32(mx, u1);
+      }
+    }
+  }
+  // chunk max
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) mx = imax32(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+  __shared__ int32_t red[kThreads / 32];
+  if (lane == 0) red[tid >> 5] = mx;
+  __syncthreads();
+  if (tid == 0) {
+    int32_t r = red[0];
+    for (int w = 1; w < kThreads / 32; ++w) r = imax32(r, red[w]);
+    a.ws_max[static_cast<size_t>(bh) * a.nsplit + sp] = r;
+  }
+}
+
+// P.V over the int4 cache: a thread owns 16 channels (an 8-byte piece of a
+// row) of 8 consecutive rows per step, so it holds 16 accumulators and keeps
+// two steps of loads (128 bytes) in flight at three CTAs per SM.
+template <int D>
+struct LayoutPv4 {
+  static constexpr int kCPR = D / 16;                // 8-byte pieces per row
+  static constexpr int kGroups = kThreads / kCPR;    // row octets per step
+  static constexpr int kRowsPerStep = 8 * kGroups;   // 256 (d=128) or 512 (d=64)
+  static_assert(kChunk4 % kRowsPerStep == 0, "chunk must be whole steps");
+};
+
+template <int D>
+__global__ void __launch_bounds__(kThreads, 3) decode4_pv_kernel(const __grid_constant__ DecodeArgs a) {
+  using Lt = LayoutPv4<D>;
+  constexpr int kRowBytes = D / 2;
+  const int bh = blockIdx.y;
+  const int sp = blockIdx.x;
+  const int j0 = sp * a.chunk;
+  const int j1 = min(a.Lk, j0 + a.chunk);
+  const int tid = threadIdx.x;
+  const int h = bh % a.H;
+  const HeadParamsDev hp = a.hp[a.per_head ? h : 0];
+
+  __shared__ uint32_t ptab_s[32];
+  __shared__ uint32_t pk[kChunk4 / 4];             // u8 probabilities of this chunk
+  __shared__ int32_t part[kThreads * 16];          // per-thread partial sums
+  __shared__ int last_flag;
+
+  const int32_t m = __ldcg(a.ws_mr + 2 * bh);
+  const unsigned long long R = static_cast<uint32_t>(__ldcg(a.ws_mr + 2 * bh + 1));
+  if (tid < 32)
+    ptab_s[tid] = static_cast<uint32_t>((static_cast<unsigned long long>(a.lut[tid]) * R + (1ull << 31)) >> 32);
+  const long long lo64 = static_cast<long long>(m) - hp.D;
+  const int32_t lo = lo64 < INT_MIN ? INT_MIN : static_cast<int32_t>(lo64);
+  const uint32_t Mu = static_cast<uint32_t>(hp.M);
+  const uint32_t sh = static_cast<uint32_t>(hp.s);
+  const uint32_t Cm = static_cast<uint32_t>(m) * Mu + (1u << (sh - 1));
+  const int32_t* srow = a.ws_s + static_cast<size_t>(bh) * a.ld_s;
+  __syncthreads();
+
+  // V rows streamed with 8-byte loads, one step ahead of the math
+  const int piece = tid % Lt::kCPR;
+  const int grp = tid / Lt::kCPR;
+  const int8_t* vbase = a.v + static_cast<size_t>(bh) * a.Lmax * kRowBytes + piece * 8;
+  auto load8 = [&](int r0, uint2 (&vv)[8]) {
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      const int j = r0 + i;
+      vv[i] = (j < j1) ? ld_stream8(vbase + static_cast<size_t>(j) * kRowBytes) : make_uint2(0, 0);
+    }
+  };
+  uint2 cur[8];
+  load8(j0 + 8 * grp, cur);
+
+  for (int w = tid; w < a.chunk / 4; w += kThreads) {
+    uint32_t word = 0;
+#pragma unroll
+    for (int b = 0; b < 4; ++b) {
+      const int j = j0 + 4 * w + b;
+      if (j < j1) {
+        const int32_t t = imax32(__ldcg(srow + j), lo);
+        word |= ptab_s[(Cm - static_cast<uint32_t>(t) * Mu) >> sh] << (8 * b);
+      }
+    }
+    pk[w] = word;
+  }
+  __syncthreads();
+
+  // acc[4u + c], u = 2g + e: channel 8g + 2c + e of this thread's 16
+  int32_t acc[16];
+#pragma unroll
+  for (int c = 0; c < 16; ++c) acc[c] = 0;
+  int32_t psum = 0;  // sum of this thread's P: the bias correction
+  for (int base = j0; base < j1; base += Lt::kRowsPerStep) {
+    const int r0 = base + 8 * grp;
+    const bool more = base + Lt::kRowsPerStep < j1;
+    uint2 nxt[8];
+    if (more) load8(r0 + Lt::kRowsPerStep, nxt);
+#pragma unroll
+    for (int hq = 0; hq < 2; ++hq) {  // the two row quads of the octet
+      const uint32_t p4 = pk[((r0 - j0) >> 2) + hq];  // P of 4 rows, one byte each (0 past j1)
+      psum = dp4a_uu(p4, 0x01010101u, psum);
+#pragma unroll
+      for (int g = 0; g < 2; ++g) {
+        const uint32_t y0 = g ? cur[4 * hq + 0].y : cur[4 * hq + 0].x;
+        const uint32_t y1 = g ? cur[4 * hq + 1].y : cur[4 * hq + 1].x;
+        const uint32_t y2 = g ? cur[4 * hq + 2].y : cur[4 * hq + 2].x;
+        const uint32_t y3 = g ? cur[4 * hq + 3].y : cur[4 * hq + 3].x;
+#pragma unroll
+        for (int e = 0; e < 2; ++e) {
+          const uint32_t x0 = e ? nib_hi(y0) : nib_lo(y0);
+          const uint32_t x1 = e ? nib_hi(y1) : nib_lo(y1);
+          const uint32_t x2 = e ? nib_hi(y2) : nib_lo(y2);
+          const uint32_t x3 = e ? nib_hi(y3) : nib_lo(y3);
+          // bytes (row i, column c) -> word c holds the 4 rows of column c
+          const uint32_t ab_lo = __byte_perm(x0, x1, 0x5140);
+          const uint32_t ab_hi = __byte_perm(x0, x1, 0x7362);
+          const uint32_t cd_lo = __byte_perm(x2, x3, 0x5140);
+          const uint32_t cd_hi = __byte_perm(x2, x3, 0x7362);
+          const int o = 4 * (2 * g + e);
+          acc[o + 0] = dp4a_uu(__byte_perm(ab_lo, cd_lo, 0x5410), p4, acc[o + 0]);
+          acc[o + 1] = dp4a_uu(__byte_perm(ab_lo, cd_lo, 0x7632), p4, acc[o + 1]);
+          acc[o + 2] = dp4a_uu(__byte_perm(ab_hi, cd_hi, 0x5410), p4, acc[o + 2]);
+          acc[o + 3] = dp4a_uu(__byte_perm(ab_hi, cd_hi, 0x7632), p4, acc[o + 3]);
+        }
+      }
+    }
+    if (more) {
+#pragma unroll
+      for (int i = 0; i < 8; ++i) cur[i] = nxt[i];
+    }
+  }
+  // per-thread sums by channel, bias removed; then reduce over the row groups
+#pragma unroll
+  for (int s = 0; s < 16; ++s) {
+    const int g = s >> 3, e = (s >> 2) & 1, c = s & 3;
+    part[tid * 16 + 8 * g + 2 * c + e] = acc[s] - 8 * psum;
   }
   __syncthreads();
   int32_t* gpart = a.ws_part + (static_cast<size_t>(bh) * a.nsplit + sp) * D;

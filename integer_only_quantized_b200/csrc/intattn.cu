@@ -176,9 +176,10 @@ struct DecodeLayout {
 
 size_t round256(size_t x) { return (x + 255) & ~size_t(255); }
 
-DecodeLayout decode_layout(long long BH, int Lk, int d) {
+// chunk: keys per CTA of the split; the int8 value gives the largest layout
+DecodeLayout decode_layout(long long BH, int Lk, int d, int chunk = intattn::decode::kChunk) {
   DecodeLayout L{};
-  L.nsplit = (Lk + intattn::decode::kChunk - 1) / intattn::decode::kChunk;
+  L.nsplit = (Lk + chunk - 1) / chunk;
   L.off_s = 0;
   L.ld_s = (Lk + 3) & ~3;  // 16-byte aligned score rows
   L.off_max = L.off_s + round256(static_cast<size_t>(BH) * L.ld_s * 4);
@@ -192,13 +193,21 @@ DecodeLayout decode_layout(long long BH, int Lk, int d) {
 template <int D, bool kInt4 = false>
 int decode_launch(const DecodeArgs& a, cudaStream_t stream) {
   const dim3 grid(a.nsplit, a.BH);
-  intattn::decode::decode_qk_kernel<D, kInt4><<<grid, intattn::decode::kThreads, 0, stream>>>(a);
+  if constexpr (kInt4) {
+    intattn::decode::decode4_qk_kernel<D><<<grid, intattn::decode::kThreads, 0, stream>>>(a);
+  } else {
+    intattn::decode::decode_qk_kernel<D><<<grid, intattn::decode::kThreads, 0, stream>>>(a);
+  }
   const int rc = note_launch(cudaGetLastError());
   if (rc != INTATTN_OK) return rc;
   intattn::decode::decode_z_kernel<D><<<a.BH, intattn::decode::kThreads, 0, stream>>>(a);
   const int rz = note_launch(cudaGetLastError());
   if (rz != INTATTN_OK) return rz;
-  intattn::decode::decode_pv_kernel<D, kInt4><<<grid, intattn::decode::kThreads, 0, stream>>>(a);
+  if constexpr (kInt4) {
+    intattn::decode::decode4_pv_kernel<D><<<grid, intattn::decode::kThreads, 0, stream>>>(a);
+  } else {
+    intattn::decode::decode_pv_kernel<D><<<grid, intattn::decode::kThreads, 0, stream>>>(a);
+  }
   return note_launch(cudaGetLastError());
 }
 
@@ -248,7 +257,7 @@ int static_scratch_address(void** out) {
 // is filled in by the caller of this helper).
 int decode_setup(const int8_t* q, const int8_t* k_cache, const int8_t* v_cache, const intattn_scales_t* scales,
                  int B, int H, int Lk, int Lmax, int d, float clip_c, int8_t* out, DecodeArgs* a,
-                 DecodeLayout* L, bool* empty) {
+                 DecodeLayout* L, bool* empty, int chunk = intattn::decode::kChunk) {
   *empty = false;
   if (B < 0 || H <= 0 || Lk < 1 || Lk > 65535 || Lmax < Lk) return INTATTN_ERR_INVALID_ARG;
   if (d != 64 && d != 128) return INTATTN_ERR_UNSUPPORTED;
@@ -265,7 +274,7 @@ int decode_setup(const int8_t* q, const int8_t* k_cache, const int8_t* v_cache, 
   if (BH > 65535) return INTATTN_ERR_UNSUPPORTED;  // grid y limit
   if (!q || !k_cache || !v_cache || !out) return INTATTN_ERR_INVALID_ARG;
   if (!aligned16(q) || !aligned16(k_cache) || !aligned16(v_cache)) return INTATTN_ERR_UNSUPPORTED;
-  *L = decode_layout(BH, Lk, d);
+  *L = decode_layout(BH, Lk, d, chunk);
   a->q = q;
   a->k = k_cache;
   a->v = v_cache;
@@ -276,7 +285,7 @@ int decode_setup(const int8_t* q, const int8_t* k_cache, const int8_t* v_cache, 
   a->Lmax = Lmax;
   a->nsplit = L->nsplit;
   a->ld_s = L->ld_s;
-  a->chunk = intattn::decode::kChunk;
+  a->chunk = chunk;
   a->per_head = scales->per_head ? 1 : 0;
   return INTATTN_OK;
 }
@@ -378,8 +387,11 @@ int intattn_decode_int4(const int8_t* q, const uint8_t* k_cache, const uint8_t* 
   DecodeArgs a;
   DecodeLayout L{};
   bool empty = false;
+  // fewer, longer splits than int8 (same bytes per CTA as 1024 int8 rows);
+  // the layout is never larger than the int8 one that the workspace size
+  // query reports
   int rc = decode_setup(q, reinterpret_cast<const int8_t*>(k_cache), reinterpret_cast<const int8_t*>(v_cache),
-                        scales, B, H, Lk, Lmax, d, clip_c, out, &a, &L, &empty);
+                        scales, B, H, Lk, Lmax, d, clip_c, out, &a, &L, &empty, intattn::decode::kChunk4);
   if (rc || empty) return rc;
   if (!workspace || workspace_bytes < L.total || (reinterpret_cast<uintptr_t>(workspace) & 255u))
     return INTATTN_ERR_WORKSPACE;
