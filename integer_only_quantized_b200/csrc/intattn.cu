@@ -387,13 +387,15 @@ int intattn_decode_int4(const int8_t* q, const uint8_t* k_cache, const uint8_t* 
   DecodeArgs a;
   DecodeLayout L{};
   bool empty = false;
-  // fewer, longer splits than int8 (same bytes per CTA as 1024 int8 rows);
-  // the layout is never larger than the int8 one that the workspace size
-  // query reports
+  // fewer, longer splits than int8 (the per-CTA set-up and reduction are
+  // amortised over more rows); the layout is never larger than the int8 one
+  // that the workspace size query reports
   int rc = decode_setup(q, reinterpret_cast<const int8_t*>(k_cache), reinterpret_cast<const int8_t*>(v_cache),
                         scales, B, H, Lk, Lmax, d, clip_c, out, &a, &L, &empty, intattn::decode::kChunk4);
   if (rc || empty) return rc;
-  if (!workspace || workspace_bytes < L.total || (reinterpret_cast<uintptr_t>(workspace) & 255u))
+  // the documented requirement is intattn_decode_workspace_size (>= L.total)
+  const size_t need = decode_layout(static_cast<long long>(B) * H, Lk, d).total;
+  if (!workspace || workspace_bytes < need || (reinterpret_cast<uintptr_t>(workspace) & 255u))
     return INTATTN_ERR_WORKSPACE;
   decode_scratch(&a, L, static_cast<char*>(workspace));
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
