@@ -301,6 +301,7 @@ def run_ours(args):
         line["decode"] = run_decode(args, dev, stream, world, peaks, peak_src, args.decode_workload)
         line["decode_int4"] = run_decode(args, dev, stream, world, peaks, peak_src,
                                          "llama7b_decode_int4_b64_lk4096")
+        line["quantize"] = run_quantize(args, dev, stream, world, peaks, peak_src)
     if not args.no_cpu_baseline and rank == 0 and world == 1:
         line["cpu_baseline"] = cpu_baseline(w, x, args.cpu_seconds)
     if rank == 0:
@@ -308,6 +309,44 @@ def run_ours(args):
     if world > 1:
         import torch.distributed as dist
         dist.destroy_process_group()
+
+
+def run_quantize(args, dev, stream, world, peaks, peak_src):
+    """Quantisation prologue on one LLaMA-7B-layer activation (bf16
+    [1, 32, 8192, 128], per-head scales): GB/s of the bf16 read + int8 write."""
+    import torch
+
+    import integer_only_quantized_b200 as ia
+    shape = (1, 32, 8192, 128)
+    n = 1
+    for s_ in shape:
+        n *= s_
+    g = torch.Generator(device=dev)
+    g.manual_seed(20251126)
+    xs = [torch.randn(shape, generator=g, device=dev, dtype=torch.float32).to(torch.bfloat16) for _ in range(3)]
+    out = torch.empty(shape, dtype=torch.int8, device=dev)
+    scales = torch.empty(shape[1], dtype=torch.float32, device=dev)
+    steps = max(10, min(args.steps, 60))
+    for i in range(max(3, args.warmup)):
+        ia.quantize(xs[i % 3], True, out=out, scales=scales, stream=stream)
+    torch.cuda.synchronize(dev)
+    barrier(world, dev)
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    t0.record(stream)
+    for i in range(steps):
+        ia.quantize(xs[i % 3], True, out=out, scales=scales, stream=stream)
+    t1.record(stream)
+    torch.cuda.synchronize(dev)
+    barrier(world, dev)
+    ms = max_over_ranks(t0.elapsed_time(t1) / steps, world, dev)
+    algo = 3 * n  # 2 bytes read + 1 byte written per element
+    gbs = algo / (ms * 1e-3) / 1e9
+    return {"workload": "llama7b_layer_bf16_b1h32l8192d128", "value": round(aggregate_value(algo, world, ms * 1e-3) / 1e9, 1),
+            "unit": "GB/s", "ms_per_call": round(ms, 5), "launches_per_call": 3, "bytes_per_call": algo,
+            "roofline": {"bound": "hbm", "achieved": round(gbs, 1), "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                         "frac": round(gbs / peaks["hbm_gbs"], 4), "peak_source": f"{peak_src} hbm_gbs",
+                         "traffic": None},
+            "l2": "inputs rotate over 3 copies (201 MB > 126 MB L2)"}
 
 
 def run_decode(args, dev, stream, world, peaks, peak_src, name):

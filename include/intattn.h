@@ -127,6 +127,27 @@ int intattn_decode_int4(const int8_t *q, const uint8_t *k_cache, const uint8_t *
                         float clip_c, int8_t *out, void *workspace, size_t workspace_bytes,
                         intattn_stream_t stream);
 
+/* Element types accepted by intattn_quantize. */
+enum { INTATTN_DTYPE_FP16 = 0, INTATTN_DTYPE_BF16 = 1 };
+
+/* Quantisation prologue (the step upstream of the integer pipeline: the
+ * forum page "IntAttention：面向边缘设备的纯整数注意力推理加速方案", section
+ * 动态量化策略, sets each layer's or head's range from the live activations).
+ *   x   [B, H, L, d] fp16 or bf16 (dtype), device, 16-byte aligned
+ *   out [B, H, L, d] int8 codes, device, 16-byte aligned
+ *   scales: DEVICE float buffer of H entries (per_head) or 1, overwritten
+ *   with the scales (real value = scale * code); used as scratch meanwhile.
+ * Definition: amax = max |x| over the tensor (or over head h);
+ *   s = amax / 127 in IEEE fp32 (s = 1 when amax = 0);
+ *   code = clamp(rint(x / s), -127, 127), fp32 division rounded to nearest,
+ *   rint half to even.  Symmetric: zero-point 0.  Inputs must be finite.
+ * L * d must be a multiple of 8.  Asynchronous on `stream`; the scales are on
+ * the device when the stream reaches the end of the call (a caller that
+ * passes them to intattn_forward reads them back first).
+ * B*H*L*d == 0 only sets the scales to 1. */
+int intattn_quantize(const void *x, int dtype, int B, int H, int L, int d, int per_head, int8_t *out,
+                     float *scales, intattn_stream_t stream);
+
 /* Capacity in bytes of the library's static decode scratch (48 MiB). */
 #define INTATTN_STATIC_SCRATCH_BYTES (48u * 1024u * 1024u)
 

@@ -22,8 +22,9 @@ MAX_HEADS = 128
 
 # every function declared in include/intattn.h
 EXPORTED = ("intattn_derive_params", "intattn_forward", "intattn_decode_workspace_size",
-            "intattn_decode", "intattn_decode_int4", "intattn_decode_static_scratch",
+            "intattn_decode", "intattn_decode_int4", "intattn_decode_static_scratch", "intattn_quantize",
             "intattn_selftest_timeout", "intattn_device_error", "intattn_strerror")
+DTYPE_FP16, DTYPE_BF16 = 0, 1
 
 
 class IntAttnError(RuntimeError):
@@ -89,6 +90,7 @@ def lib() -> ctypes.CDLL:
                                           f32, vp, vp, ctypes.c_size_t, vp]
         L.intattn_decode_static_scratch.argtypes = [vp, vp, vp, ctypes.POINTER(_Scales), i32, i32, i32,
                                                     i32, i32, f32, vp, vp]
+        L.intattn_quantize.argtypes = [vp, i32, i32, i32, i32, i32, i32, vp, vp, vp]
         L.intattn_selftest_timeout.argtypes = [vp]
         L.intattn_device_error.argtypes = [vp]
         L.intattn_strerror.argtypes = [i32]
@@ -225,6 +227,31 @@ def decode_int4(q, k_cache, v_cache, scales: Scales, Lk: int, clip_c: float, out
     del keep
     _check(rc, "intattn_decode_int4")
     return out
+
+
+def quantize(x, per_head: bool, out=None, scales=None, stream=None):
+    """int8 codes and device scales of an fp16 / bf16 CUDA tensor [B, H, L, d]
+    (symmetric, dynamic: s = max|x| / 127 per tensor or per head)."""
+    import torch
+    if not isinstance(x, torch.Tensor) or not x.is_cuda or x.dtype not in (torch.float16, torch.bfloat16):
+        raise TypeError("x must be a CUDA float16 or bfloat16 tensor")
+    if not x.is_contiguous() or x.dim() != 4:
+        raise ValueError("x must be a contiguous [B, H, L, d] tensor")
+    B, H, L, d = x.shape
+    if out is None:
+        out = torch.empty(x.shape, dtype=torch.int8, device=x.device)
+    _check_tensor(out, "out")
+    if out.shape != x.shape:
+        raise ValueError("out must match x")
+    n = H if per_head else 1
+    if scales is None:
+        scales = torch.empty(n, dtype=torch.float32, device=x.device)
+    if scales.dtype != torch.float32 or not scales.is_cuda or scales.numel() < n:
+        raise ValueError(f"scales must be a CUDA float32 tensor of at least {n} entries")
+    dt = DTYPE_BF16 if x.dtype == torch.bfloat16 else DTYPE_FP16
+    _check(lib().intattn_quantize(x.data_ptr(), dt, B, H, L, d, int(bool(per_head)), out.data_ptr(),
+                                  scales.data_ptr(), _stream_handle(stream, x.device)), "intattn_quantize")
+    return out, scales
 
 
 def device_error(stream=None) -> int:

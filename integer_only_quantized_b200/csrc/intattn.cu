@@ -16,6 +16,7 @@
 #include "intattn.h"
 
 #include "decode_kernel.cuh"
+#include "quantize_kernel.cuh"
 #include "prefill_kernel.cuh"
 
 using intattn::DecodeArgs;
@@ -418,6 +419,49 @@ int intattn_decode_static_scratch(const int8_t* q, const int8_t* k_cache, const 
   decode_scratch(&a, L, static_cast<char*>(scratch));
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   return d == 64 ? decode_launch<64>(a, st) : decode_launch<128>(a, st);
+}
+
+int intattn_quantize(const void* x, int dtype, int B, int H, int L, int d, int per_head, int8_t* out,
+                     float* scales, intattn_stream_t stream) {
+  if (B < 0 || H <= 0 || L < 0 || d <= 0) return INTATTN_ERR_INVALID_ARG;
+  if (dtype != INTATTN_DTYPE_FP16 && dtype != INTATTN_DTYPE_BF16) return INTATTN_ERR_UNSUPPORTED;
+  if (!scales) return INTATTN_ERR_INVALID_ARG;
+  const long long slice = static_cast<long long>(L) * d;
+  if (slice % intattn::quant::kVec) return INTATTN_ERR_UNSUPPORTED;  // whole 16-byte vectors per (b, h)
+  const long long BH = static_cast<long long>(B) * H;
+  if (BH > 65535) return INTATTN_ERR_UNSUPPORTED;  // grid y limit
+  if (reinterpret_cast<uintptr_t>(scales) & 3u) return INTATTN_ERR_UNSUPPORTED;
+  const int n_scales = per_head ? H : 1;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  if (BH == 0 || slice == 0) {
+    // no elements: amax 0 -> every scale is 1
+    if (note_launch(cudaMemsetAsync(scales, 0, n_scales * sizeof(float), st))) return INTATTN_ERR_CUDA;
+    intattn::quant::quant_scales_kernel<<<1, 128, 0, st>>>(reinterpret_cast<uint32_t*>(scales), n_scales);
+    return note_launch(cudaGetLastError());
+  }
+  if (!x || !out) return INTATTN_ERR_INVALID_ARG;
+  if (!aligned16(x) || !aligned16(out)) return INTATTN_ERR_UNSUPPORTED;
+  const long long chunks = (slice + intattn::quant::kChunkElems - 1) / intattn::quant::kChunkElems;
+  if (chunks > 0x7fffffffLL) return INTATTN_ERR_UNSUPPORTED;
+  intattn::QuantArgs a;
+  a.x = x;
+  a.out = out;
+  a.amax = reinterpret_cast<uint32_t*>(scales);
+  a.slice = slice;
+  a.H = H;
+  a.per_head = per_head ? 1 : 0;
+  a.bf16 = dtype == INTATTN_DTYPE_BF16 ? 1 : 0;
+  a.chunks = static_cast<int32_t>(chunks);
+  if (note_launch(cudaMemsetAsync(scales, 0, n_scales * sizeof(float), st))) return INTATTN_ERR_CUDA;
+  const dim3 grid(static_cast<unsigned>(chunks), static_cast<unsigned>(BH));
+  intattn::quant::quant_amax_kernel<<<grid, intattn::quant::kThreads, 0, st>>>(a);
+  int rc = note_launch(cudaGetLastError());
+  if (rc) return rc;
+  intattn::quant::quant_codes_kernel<<<grid, intattn::quant::kThreads, 0, st>>>(a);
+  rc = note_launch(cudaGetLastError());
+  if (rc) return rc;
+  intattn::quant::quant_scales_kernel<<<1, 128, 0, st>>>(a.amax, n_scales);
+  return note_launch(cudaGetLastError());
 }
 
 int intattn_selftest_timeout(intattn_stream_t stream) {
