@@ -138,9 +138,11 @@ enum { INTATTN_DTYPE_FP16 = 0, INTATTN_DTYPE_BF16 = 1 };
  *   scales: DEVICE float buffer of H entries (per_head) or 1, overwritten
  *   with the scales (real value = scale * code); used as scratch meanwhile.
  * Definition: amax = max |x| over the tensor (or over head h);
- *   s = amax / 127 in IEEE fp32 (s = 1 when amax = 0);
- *   code = clamp(rint(x / s), -127, 127), fp32 division rounded to nearest,
- *   rint half to even.  Symmetric: zero-point 0.  Inputs must be finite.
+ *   s = amax / 127 and inv = min(127 / amax, FLT_MAX) in IEEE fp32 (both 1
+ *   when amax = 0);
+ *   code = clamp(rint(x * inv), -127, 127), fp32 product rounded to
+ *   nearest, rint half to even.  Symmetric: zero-point 0.  Inputs must be
+ *   finite.
  * L * d must be a multiple of 8.  Asynchronous on `stream`; the scales are on
  * the device when the stream reaches the end of the call (a caller that
  * passes them to intattn_forward reads them back first).

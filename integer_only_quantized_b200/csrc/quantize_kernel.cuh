@@ -6,9 +6,10 @@
 // describes choosing the quantisation range of each layer (or head) from the
 // live activations.  Definition computed here (identical to the numpy
 // oracle): amax = max |x| over the tensor or over one head [B, L, d] slice;
-// s = amax / 127 (IEEE fp32 division), s = 1 if amax = 0; code =
-// clamp(rint(x / s), -127, 127) with the fp32 division rounded to nearest
-// and rint rounding half to even.  Zero-point 0 (symmetric).
+// s = amax / 127 and inv = min(127 / amax, FLT_MAX) (IEEE fp32 divisions),
+// s = inv = 1 if amax = 0; code = clamp(rint(x * inv), -127, 127) with the
+// fp32 product rounded to nearest and rint rounding half to even.
+// Zero-point 0.
 //
 // Three launches per tensor: quant_amax (per-CTA max |x| of a slice chunk,
 // atomicMax on the float bits, which order like the unsigned integers for
@@ -34,8 +35,8 @@ namespace quant {
 
 constexpr int kThreads = 256;
 constexpr int kVec = 8;                          // elements per 16-byte load
-constexpr int kIters = 4;                        // loads per thread and CTA
-constexpr int kChunkElems = kThreads * kVec * kIters;  // 8192 elements per CTA
+constexpr int kIters = 16;                       // loads per thread and CTA
+constexpr int kChunkElems = kThreads * kVec * kIters;  // 32768 elements per CTA
 
 __device__ __forceinline__ void to_float8(uint4 v, bool bf16, float (&f)[8]) {
   const uint32_t w[4] = {v.x, v.y, v.z, v.w};
@@ -54,6 +55,12 @@ __device__ __forceinline__ void to_float8(uint4 v, bool bf16, float (&f)[8]) {
 __device__ __forceinline__ float scale_of(uint32_t amax_bits) {
   const float s = __fdiv_rn(__uint_as_float(amax_bits), 127.0f);
   return s == 0.0f ? 1.0f : s;
+}
+// 127 / amax, capped at the largest float (an amax below 127 / FLT_MAX would
+// overflow it)
+__device__ __forceinline__ float inv_scale_of(uint32_t amax_bits) {
+  const float amax = __uint_as_float(amax_bits);
+  return amax == 0.0f ? 1.0f : fminf(__fdiv_rn(127.0f, amax), 3.402823466e38f);
 }
 
 // grid (chunks, B*H)
@@ -90,7 +97,7 @@ __global__ void __launch_bounds__(kThreads) quant_codes_kernel(const __grid_cons
   const int64_t e0 = static_cast<int64_t>(blockIdx.x) * kChunkElems;
   const uint4* src = reinterpret_cast<const uint4*>(static_cast<const uint16_t*>(a.x) + bh * a.slice);
   uint2* dst = reinterpret_cast<uint2*>(a.out + bh * a.slice);
-  const float s = scale_of(__ldcg(a.amax + (a.per_head ? bh % a.H : 0)));
+  const float inv = inv_scale_of(__ldcg(a.amax + (a.per_head ? bh % a.H : 0)));
 #pragma unroll
   for (int it = 0; it < kIters; ++it) {
     const int64_t e = e0 + (static_cast<int64_t>(it) * kThreads + threadIdx.x) * kVec;
@@ -100,7 +107,7 @@ __global__ void __launch_bounds__(kThreads) quant_codes_kernel(const __grid_cons
       uint32_t b[8];
 #pragma unroll
       for (int i = 0; i < 8; ++i) {
-        int q = __float2int_rn(__fdiv_rn(f[i], s));
+        int q = __float2int_rn(__fmul_rn(f[i], inv));
         q = q > 127 ? 127 : (q < -127 ? -127 : q);
         b[i] = static_cast<uint32_t>(q) & 0xFFu;
       }

@@ -8,8 +8,9 @@ section 动态量化策略 (the quantisation range of a layer, or of a head, is 
 from the live activations), with the readings: symmetric (zero-point 0),
 range = max |x|, 127 levels each side, round half to even.  Definition:
     amax = max |x| over the tensor, or over one head's [B, L, d] slice
-    s    = amax / 127 in IEEE fp32 (s = 1 when amax = 0)
-    code = clamp(rint(x / s), -127, 127), the fp32 division rounded to nearest
+    s    = amax / 127 and inv = min(127 / amax, FLT_MAX) in IEEE fp32 (both 1
+           when amax = 0)
+    code = clamp(rint(x * inv), -127, 127), the fp32 product rounded to nearest
 """
 import numpy as np
 
@@ -23,8 +24,13 @@ def quantize(x, per_head: bool):
         amax = np.abs(x).max(axis=(0, 2, 3)) if x.size else np.zeros(H, np.float32)
     else:
         amax = np.array([np.abs(x).max() if x.size else 0.0], dtype=np.float32)
-    s = (amax.astype(np.float32) / np.float32(127.0)).astype(np.float32)
-    s[s == 0] = np.float32(1.0)
-    per = s if per_head else np.repeat(s, H)
-    q = np.rint(x / per[None, :, None, None].astype(np.float32))  # float32 division, half-even
+    amax = amax.astype(np.float32)
+    s = (amax / np.float32(127.0)).astype(np.float32)
+    s[amax == 0] = np.float32(1.0)
+    inv = np.ones_like(amax)
+    nz = amax != 0
+    with np.errstate(over="ignore", divide="ignore"):
+        inv[nz] = np.minimum(np.float32(127.0) / amax[nz], np.finfo(np.float32).max).astype(np.float32)
+    per = inv if per_head else np.repeat(inv, H)
+    q = np.rint(x * per[None, :, None, None].astype(np.float32))  # float32 product, half-even
     return np.clip(q, -127, 127).astype(np.int8), s
