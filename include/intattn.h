@@ -66,14 +66,22 @@ enum {
 #define INTATTN_MAX_HEADS 128
 
 /* Quantisation scales (real value = scale * int8 code).  per_head = 0: each
- * array holds one entry shared by all heads; per_head = 1: H entries. */
+ * array holds one entry shared by all heads; per_head = 1: H entries.
+ * clip_c (optional): per-head clip thresholds in the same layout (the
+ * authors name a learned / adaptive clip as future work: this is where a
+ * calibrated threshold per head goes in); NULL: the clip_c argument of the
+ * call applies to every head.  At most INTATTN_MAX_CLIPS distinct values per
+ * call (each needs its own exp table), else INTATTN_ERR_UNSUPPORTED. */
 typedef struct intattn_scales {
     int32_t per_head;
     const float *s_q;
     const float *s_k;
     const float *s_v;
     const float *s_o;
+    const float *clip_c;
 } intattn_scales_t;
+
+#define INTATTN_MAX_CLIPS 8
 
 /* Derived integer parameters of one head (see the definition above). */
 typedef struct intattn_head_params {
@@ -85,7 +93,8 @@ typedef struct intattn_head_params {
 } intattn_head_params_t;
 
 /* Host-only: derive the LUT and the per-head parameters exactly as the
- * kernels use them.  lut: 32 entries; out: H entries.  No GPU needed. */
+ * kernels use them.  lut: 32 entries (the table of head 0's clip threshold);
+ * out: H entries.  No GPU needed. */
 int intattn_derive_params(const intattn_scales_t *scales, int H, int d, float clip_c,
                           int32_t lut[32], intattn_head_params_t *out);
 

@@ -19,6 +19,7 @@ LIB_PATH = os.path.join(_HERE, "libintattn.so")
 
 OK, ERR_INVALID_ARG, ERR_UNSUPPORTED, ERR_PARAM_RANGE, ERR_CUDA, ERR_WORKSPACE, ERR_TIMEOUT = range(7)
 MAX_HEADS = 128
+MAX_CLIPS = 8
 
 # every function declared in include/intattn.h
 EXPORTED = ("intattn_derive_params", "intattn_forward", "intattn_decode_workspace_size",
@@ -38,7 +39,8 @@ class _Scales(ctypes.Structure):
                 ("s_q", ctypes.POINTER(ctypes.c_float)),
                 ("s_k", ctypes.POINTER(ctypes.c_float)),
                 ("s_v", ctypes.POINTER(ctypes.c_float)),
-                ("s_o", ctypes.POINTER(ctypes.c_float))]
+                ("s_o", ctypes.POINTER(ctypes.c_float)),
+                ("clip_c", ctypes.POINTER(ctypes.c_float))]
 
 
 class _HeadParams(ctypes.Structure):
@@ -51,18 +53,26 @@ FloatArg = Union[float, Sequence[float], np.ndarray]
 
 @dataclasses.dataclass
 class Scales:
-    """Quantisation scales (real = scale * code).  per_head: arrays of H."""
+    """Quantisation scales (real = scale * code).  per_head: arrays of H.
+    clip: optional per-head clip thresholds (same layout as the scales);
+    None: the call's clip_c applies to every head."""
     s_q: FloatArg
     s_k: FloatArg
     s_v: FloatArg
     s_o: FloatArg
     per_head: bool = False
+    clip: Optional[FloatArg] = None
 
     def _c(self):
         arrs = [np.ascontiguousarray(np.atleast_1d(np.asarray(x, dtype=np.float32)))
                 for x in (self.s_q, self.s_k, self.s_v, self.s_o)]
         fp = ctypes.POINTER(ctypes.c_float)
-        s = _Scales(int(bool(self.per_head)), *[a.ctypes.data_as(fp) for a in arrs])
+        clip = None
+        if self.clip is not None:
+            clip = np.ascontiguousarray(np.atleast_1d(np.asarray(self.clip, dtype=np.float32)))
+            arrs.append(clip)
+        s = _Scales(int(bool(self.per_head)), *[a.ctypes.data_as(fp) for a in arrs[:4]],
+                    clip.ctypes.data_as(fp) if clip is not None else fp())
         return s, arrs  # keep the arrays alive for the duration of the call
 
 

@@ -41,7 +41,7 @@ struct DecodeArgs {
   uint32_t* ws_cnt;  // [BH]              arrival tickets
   int32_t* ws_mr;    // [BH, 2]           row max and reciprocal R
   int32_t BH, H, Lk, Lmax, nsplit, chunk, per_head, ld_s;
-  uint32_t lut[32];
+  uint32_t lut[INTATTN_MAX_CLIPS][32];  // one exp table per distinct clip threshold
   HeadParamsDev hp[INTATTN_MAX_HEADS];
 };
 
@@ -201,7 +201,7 @@ __global__ void __launch_bounds__(kThreads) decode_z_kernel(const __grid_constan
   const HeadParamsDev hp = a.hp[a.per_head ? h : 0];
   __shared__ uint32_t lut_s[32];
   __shared__ int32_t red[kThreads / 32];
-  if (tid < 32) lut_s[tid] = a.lut[tid];
+  if (tid < 32) lut_s[tid] = a.lut[hp.lut][tid];
   int32_t m = INT_MIN;
   for (int i = 0; i < a.nsplit; ++i) m = imax32(m, __ldcg(a.ws_max + static_cast<size_t>(bh) * a.nsplit + i));
   const long long lo64 = static_cast<long long>(m) - hp.D;
@@ -260,7 +260,7 @@ __global__ void __launch_bounds__(kThreads) decode_pv_kernel(const __grid_consta
   const int32_t m = __ldcg(a.ws_mr + 2 * bh);
   const unsigned long long R = static_cast<uint32_t>(__ldcg(a.ws_mr + 2 * bh + 1));
   if (tid < 32)
-    ptab_s[tid] = static_cast<uint32_t>((static_cast<unsigned long long>(a.lut[tid]) * R + (1ull << 31)) >> 32);
+    ptab_s[tid] = static_cast<uint32_t>((static_cast<unsigned long long>(a.lut[hp.lut][tid]) * R + (1ull << 31)) >> 32);
   const long long lo64 = static_cast<long long>(m) - hp.D;
   const int32_t lo = lo64 < INT_MIN ? INT_MIN : static_cast<int32_t>(lo64);
   const uint32_t Mu = static_cast<uint32_t>(hp.M);
@@ -502,7 +502,7 @@ __global__ void __launch_bounds__(kThreads, 3) decode4_pv_kernel(const __grid_co
   const int32_t m = __ldcg(a.ws_mr + 2 * bh);
   const unsigned long long R = static_cast<uint32_t>(__ldcg(a.ws_mr + 2 * bh + 1));
   if (tid < 32)
-    ptab_s[tid] = static_cast<uint32_t>((static_cast<unsigned long long>(a.lut[tid]) * R + (1ull << 31)) >> 32);
+    ptab_s[tid] = static_cast<uint32_t>((static_cast<unsigned long long>(a.lut[hp.lut][tid]) * R + (1ull << 31)) >> 32);
   const long long lo64 = static_cast<long long>(m) - hp.D;
   const int32_t lo = lo64 < INT_MIN ? INT_MIN : static_cast<int32_t>(lo64);
   const uint32_t Mu = static_cast<uint32_t>(hp.M);

@@ -74,21 +74,33 @@ int make_lut(double c, uint32_t lut[32]) {
   return INTATTN_OK;
 }
 
-// LUT and head parameters; per-tensor scales fill hp[0] only.
-int derive(const intattn_scales_t* sc, int H, int d, float clip_c, uint32_t lut[32],
-           HeadParamsDev* hp, int max_heads) {
+// LUTs and head parameters; per-tensor scales fill hp[0] only.  Each
+// distinct clip threshold gets its own table (at most INTATTN_MAX_CLIPS).
+int derive(const intattn_scales_t* sc, int H, int d, float clip_c, uint32_t lut[INTATTN_MAX_CLIPS][32],
+           HeadParamsDev* hp, int max_heads, int* n_luts = nullptr) {
   if (!sc || !sc->s_q || !sc->s_k || !sc->s_v || !sc->s_o) return INTATTN_ERR_INVALID_ARG;
   if (H <= 0) return INTATTN_ERR_INVALID_ARG;
   const int n = sc->per_head ? H : 1;
   if (n > max_heads) return INTATTN_ERR_UNSUPPORTED;
-  int rc = make_lut(static_cast<double>(clip_c), lut);
-  if (rc) return rc;
+  float clips[INTATTN_MAX_CLIPS];
+  int nclips = 0;
   for (int i = 0; i < n; ++i) {
-    rc = index_params(sc->s_q[i], sc->s_k[i], d, static_cast<double>(clip_c), &hp[i]);
+    const float c = sc->clip_c ? sc->clip_c[i] : clip_c;
+    int id = 0;
+    while (id < nclips && !(clips[id] == c)) ++id;
+    if (id == nclips) {
+      if (nclips == INTATTN_MAX_CLIPS) return INTATTN_ERR_UNSUPPORTED;
+      const int rc = make_lut(static_cast<double>(c), lut[nclips]);
+      if (rc) return rc;
+      clips[nclips++] = c;
+    }
+    int rc = index_params(sc->s_q[i], sc->s_k[i], d, static_cast<double>(c), &hp[i]);
     if (rc) return rc;
     rc = requant_params(sc->s_v[i], sc->s_o[i], &hp[i]);
     if (rc) return rc;
+    hp[i].lut = id;
   }
+  if (n_luts) *n_luts = nclips;
   return INTATTN_OK;
 }
 
@@ -263,7 +275,8 @@ int decode_setup(const int8_t* q, const int8_t* k_cache, const int8_t* v_cache, 
   if (B < 0 || H <= 0 || Lk < 1 || Lk > 65535 || Lmax < Lk) return INTATTN_ERR_INVALID_ARG;
   if (d != 64 && d != 128) return INTATTN_ERR_UNSUPPORTED;
   if (!scales) return INTATTN_ERR_INVALID_ARG;
-  static_assert(sizeof(DecodeArgs) <= 4096, "kernel argument block too large");
+  // kernel parameters up to 32764 bytes need CUDA 12.1 or later
+  static_assert(sizeof(DecodeArgs) <= 8192, "kernel argument block too large");
   std::memset(a, 0, sizeof(*a));
   int rc = derive(scales, H, d, clip_c, a->lut, a->hp, INTATTN_MAX_HEADS);
   if (rc) return rc;
@@ -307,7 +320,7 @@ int intattn_derive_params(const intattn_scales_t* scales, int H, int d, float cl
                           intattn_head_params_t* out) {
   if (!lut || !out) return INTATTN_ERR_INVALID_ARG;
   if (d != 64 && d != 128) return INTATTN_ERR_UNSUPPORTED;
-  uint32_t l[32];
+  uint32_t l[INTATTN_MAX_CLIPS][32];
   HeadParamsDev hp[INTATTN_MAX_HEADS];
   if (scales && !scales->per_head && H > 0) {
     // per-tensor: every head shares entry 0; any H is accepted
@@ -319,7 +332,7 @@ int intattn_derive_params(const intattn_scales_t* scales, int H, int d, float cl
     if (rc) return rc;
     for (int h = 0; h < H; ++h) out[h] = {hp[h].M, hp[h].s, hp[h].D, hp[h].Mo, hp[h].so};
   }
-  for (int i = 0; i < 32; ++i) lut[i] = static_cast<int32_t>(l[i]);
+  for (int i = 0; i < 32; ++i) lut[i] = static_cast<int32_t>(l[hp[0].lut][i]);
   return INTATTN_OK;
 }
 
@@ -330,10 +343,10 @@ int intattn_forward(const int8_t* q, const int8_t* k, const int8_t* v, const int
   if (causal && Lq > Lk) return INTATTN_ERR_INVALID_ARG;
   if (d != 64 && d != 128) return INTATTN_ERR_UNSUPPORTED;
   if (!scales) return INTATTN_ERR_INVALID_ARG;
-  static_assert(sizeof(PrefillArgs) <= 4096, "kernel argument block too large");
+  static_assert(sizeof(PrefillArgs) <= 8192, "kernel argument block too large");
   PrefillArgs args;
   std::memset(&args, 0, sizeof(args));
-  int rc = derive(scales, H, d, clip_c, args.lut, args.hp, INTATTN_MAX_HEADS);
+  int rc = derive(scales, H, d, clip_c, args.lut, args.hp, INTATTN_MAX_HEADS, &args.n_luts);
   if (rc) return rc;
   const long long BH = static_cast<long long>(B) * H;
   if (BH == 0 || Lq == 0) return INTATTN_OK;

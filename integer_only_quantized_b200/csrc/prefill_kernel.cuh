@@ -55,8 +55,8 @@ struct PrefillArgs {
   CUtensorMap tm_k;  // [B*H, Lk, d]
   CUtensorMap tm_v;  // [B*H, Lk, d]
   int8_t* out;       // [B, H, Lq, d]
-  int32_t BH, H, Lq, Lk, causal, n_qtiles, per_head, n_tiles;
-  uint32_t lut[32];
+  int32_t BH, H, Lq, Lk, causal, n_qtiles, per_head, n_tiles, n_luts;
+  uint32_t lut[INTATTN_MAX_CLIPS][32];  // one exp table per distinct clip threshold
   HeadParamsDev hp[INTATTN_MAX_HEADS];
 };
 
@@ -116,7 +116,7 @@ struct Cfg {
   static constexpr uint32_t kOffPtab = kOffKV + kStages * kTileBytes;    // [33][kBM] u32
   static constexpr uint32_t kOffRed = kOffPtab + 33 * kBM * 4;          // [2][kGroups][kBM] int32
   static constexpr uint32_t kOffLut = kOffRed + 2 * kGroups * kBM * 4;
-  static constexpr uint32_t kOffBars = kOffLut + 32 * 4;
+  static constexpr uint32_t kOffBars = kOffLut + INTATTN_MAX_CLIPS * 32 * 4;
   static constexpr uint32_t kOffTmem = kOffBars + kNumBars * 8;
   static constexpr uint32_t kUsed = kOffTmem + 16;
   // One CTA per SM: every CTA allocates all 512 TMEM columns, so the
@@ -215,7 +215,7 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_kernel(const __grid_const
     }
     mbar_fence_init();
   }
-  if (tid < 32) lut_s[tid] = args.lut[tid];
+  for (int i = tid; i < args.n_luts * 32; i += blockDim.x) lut_s[i] = args.lut[i >> 5][i & 31];
   if (warp == kMmaWarp) {
     tmem_alloc(smem_u32(tmem_slot), kTmemCols);
     tmem_relinquish();
@@ -242,8 +242,7 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_kernel(const __grid_const
     // for a masked / clipped key.  Lane k holds LUT[k-1] as a float (lane 0:
     // 0); a shuffle whose source lane is the low 5 bits of the code looks it
     // up.  Per tile a thread sums 32 values below 2^15: the float sums are exact.
-    const int32_t lut_lane =
-        __float_as_int(lane == 0 ? 0.f : __int2float_rn(static_cast<int32_t>(lut_s[lane - 1])));
+    int32_t lut_lane = 0;  // set per tile: the table of the tile's head
     if (sw < 4) ptab[r] = 0u;  // table row 0 (masked keys) stays 0
     bool ok = true;
     uint32_t sc = 0;  // S tiles of the CTA so far (both teams, all passes and tiles)
@@ -288,6 +287,8 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_kernel(const __grid_const
       if (L >= args.n_tiles) break;
       const Tile T = tile_of(args, L);
       const HeadParamsDev hp = args.hp[args.per_head ? T.h : 0];
+      const uint32_t* lut_h = lut_s + 32 * hp.lut;
+      lut_lane = __float_as_int(lane == 0 ? 0.f : __int2float_rn(static_cast<int32_t>(lut_h[lane - 1])));
       const int off = args.Lk - args.Lq;
       const int row_limit = T.q0 + r + off;  // causal: last visible key of this row
       auto tile_full = [&](int j) {
@@ -397,7 +398,7 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_kernel(const __grid_const
 #pragma unroll
         for (int i = grp * 8; i < grp * 8 + 8; ++i)
           ptab[(i + 1) * kBM + r] =
-              static_cast<uint32_t>((static_cast<unsigned long long>(lut_s[i]) * R + (1ull << 31)) >> 32);
+              static_cast<uint32_t>((static_cast<unsigned long long>(lut_h[i]) * R + (1ull << 31)) >> 32);
       }
       all_sync(true);  // the table is complete
 
