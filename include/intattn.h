@@ -143,9 +143,10 @@ enum { INTATTN_DTYPE_FP16 = 0, INTATTN_DTYPE_BF16 = 1 };
  * forum page "IntAttention：面向边缘设备的纯整数注意力推理加速方案", section
  * 动态量化策略, sets each layer's or head's range from the live activations).
  *   x   [B, H, L, d] fp16 or bf16 (dtype), device, 16-byte aligned
- *   out [B, H, L, d] int8 codes, device, 16-byte aligned
+ *   out [B, H, L, d] int8 codes, device, 16-byte aligned, not overlapping
+ *   x; its first 8 bytes hold two grid-barrier counters until the call ends
  *   scales: DEVICE float buffer of H entries (per_head) or 1, overwritten
- *   with the scales (real value = scale * code); used as scratch meanwhile.
+ *   with the scales (real value = scale * code); holds amax meanwhile.
  * Definition: amax = max |x| over the tensor (or over head h);
  *   s = amax / 127 and inv = min(127 / amax, FLT_MAX) in IEEE fp32 (both 1
  *   when amax = 0);
@@ -155,7 +156,10 @@ enum { INTATTN_DTYPE_FP16 = 0, INTATTN_DTYPE_BF16 = 1 };
  * L * d must be a multiple of 8.  Asynchronous on `stream`; the scales are on
  * the device when the stream reaches the end of the call (a caller that
  * passes them to intattn_forward reads them back first).
- * B*H*L*d == 0 only sets the scales to 1. */
+ * B*H*L*d == 0 only sets the scales to 1.
+ * Two launches: a zeroing kernel and one cooperative single-pass kernel
+ * (max |x|, a bounded grid barrier, codes); a barrier that times out is
+ * reported by intattn_device_error. */
 int intattn_quantize(const void *x, int dtype, int B, int H, int L, int d, int per_head, int8_t *out,
                      float *scales, intattn_stream_t stream);
 

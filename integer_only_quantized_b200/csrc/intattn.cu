@@ -8,6 +8,7 @@
 #include <cuda.h>
 #include <cuda_runtime.h>
 
+#include <algorithm>
 #include <cmath>
 #include <cstdint>
 #include <cstring>
@@ -441,9 +442,8 @@ int intattn_quantize(const void* x, int dtype, int B, int H, int L, int d, int p
   if (!scales) return INTATTN_ERR_INVALID_ARG;
   const long long slice = static_cast<long long>(L) * d;
   if (slice % intattn::quant::kVec) return INTATTN_ERR_UNSUPPORTED;  // whole 16-byte vectors per (b, h)
-  const long long BH = static_cast<long long>(B) * H;
-  if (BH > 65535) return INTATTN_ERR_UNSUPPORTED;  // grid y limit
   if (reinterpret_cast<uintptr_t>(scales) & 3u) return INTATTN_ERR_UNSUPPORTED;
+  const long long BH = static_cast<long long>(B) * H;
   const int n_scales = per_head ? H : 1;
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   if (BH == 0 || slice == 0) {
@@ -454,27 +454,43 @@ int intattn_quantize(const void* x, int dtype, int B, int H, int L, int d, int p
   }
   if (!x || !out) return INTATTN_ERR_INVALID_ARG;
   if (!aligned16(x) || !aligned16(out)) return INTATTN_ERR_UNSUPPORTED;
-  const long long chunks = (slice + intattn::quant::kChunkElems - 1) / intattn::quant::kChunkElems;
-  if (chunks > 0x7fffffffLL) return INTATTN_ERR_UNSUPPORTED;
   intattn::QuantArgs a;
   a.x = x;
   a.out = out;
   a.amax = reinterpret_cast<uint32_t*>(scales);
-  a.slice = slice;
+  a.nvec = BH * (slice / intattn::quant::kVec);
+  a.seg = per_head ? slice / intattn::quant::kVec : a.nvec;
   a.H = H;
   a.per_head = per_head ? 1 : 0;
   a.bf16 = dtype == INTATTN_DTYPE_BF16 ? 1 : 0;
-  a.chunks = static_cast<int32_t>(chunks);
-  if (note_launch(cudaMemsetAsync(scales, 0, n_scales * sizeof(float), st))) return INTATTN_ERR_CUDA;
-  const dim3 grid(static_cast<unsigned>(chunks), static_cast<unsigned>(BH));
-  intattn::quant::quant_amax_kernel<<<grid, intattn::quant::kThreads, 0, st>>>(a);
-  int rc = note_launch(cudaGetLastError());
+  a.n_scales = n_scales;
+  int sms = 0;
+  if (sm_count(&sms) != INTATTN_OK) return INTATTN_ERR_CUDA;
+  // one CTA per resident slot (the grid barrier needs them all resident),
+  // each CTA >= one vector per thread
+  int occ = 0;
+  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, intattn::quant::quant_fused_kernel,
+                                                    intattn::quant::kThreads, 0) != cudaSuccess || occ < 1)
+    return note_launch(cudaGetLastError());
+  const long long want = (a.nvec + intattn::quant::kThreads - 1) / intattn::quant::kThreads;
+  const unsigned grid = static_cast<unsigned>(std::min<long long>(want, static_cast<long long>(sms) * occ));
+  intattn::quant::quant_zero_kernel<<<1, 128, 0, st>>>(a.amax, n_scales, reinterpret_cast<uint32_t*>(out));
+  const int rc = note_launch(cudaGetLastError());
   if (rc) return rc;
-  intattn::quant::quant_codes_kernel<<<grid, intattn::quant::kThreads, 0, st>>>(a);
-  rc = note_launch(cudaGetLastError());
-  if (rc) return rc;
-  intattn::quant::quant_scales_kernel<<<1, 128, 0, st>>>(a.amax, n_scales);
-  return note_launch(cudaGetLastError());
+  // cooperative: all CTAs resident (the grid barrier); programmatic
+  // serialisation: the loads of pass 1 overlap quant_zero
+  cudaLaunchAttribute attrs[2];
+  attrs[0].id = cudaLaunchAttributeCooperative;
+  attrs[0].val.cooperative = 1;
+  attrs[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attrs[1].val.programmaticStreamSerializationAllowed = 1;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(grid);
+  cfg.blockDim = dim3(intattn::quant::kThreads);
+  cfg.stream = st;
+  cfg.attrs = attrs;
+  cfg.numAttrs = 2;
+  return note_launch(cudaLaunchKernelEx(&cfg, intattn::quant::quant_fused_kernel, a));
 }
 
 int intattn_selftest_timeout(intattn_stream_t stream) {

@@ -11,15 +11,24 @@
 // fp32 product rounded to nearest and rint rounding half to even.
 // Zero-point 0.
 //
-// Three launches per tensor: quant_amax (per-CTA max |x| of a slice chunk,
-// atomicMax on the float bits, which order like the unsigned integers for
-// values >= 0), quant_codes (each CTA derives s from amax and writes the
-// codes), quant_scales (amax -> s in place).  The caller's scale buffer
-// holds amax between the launches; it is zeroed by a memset first.
+// Two launches per tensor.  quant_zero clears the caller's scale buffer
+// (which holds amax as float bits until the end) and the first 8 bytes of
+// the code buffer (two grid-barrier counters until the end).  quant_fused
+// runs one CTA per resident slot (cooperative launch, so all are resident)
+// over balanced ranges of 16-byte vectors: pass 1 takes max |x| of each
+// range (split at head boundaries) and merges it with atomicMax on the float
+// bits, which order like the unsigned integers for values >= 0; a grid
+// barrier; pass 2 re-reads the range (from L2 when the tensor fits there),
+// derives inv from amax and writes the codes.  After every CTA has finished
+// pass 2, CTA 0 turns amax into s in place and writes code vector 0 over the
+// counters.  Each wait is bounded in time and records a timeout in
+// g_device_error.
 #pragma once
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
 #include <cstdint>
+
+#include "sm100.cuh"
 
 namespace intattn {
 
@@ -27,16 +36,51 @@ struct QuantArgs {
   const void* x;     // [B, H, L, d] fp16 or bf16
   int8_t* out;       // [B, H, L, d]
   uint32_t* amax;    // [H] or [1]: the caller's float scale buffer, used as bits
-  int64_t slice;     // L * d elements of one (b, h)
-  int32_t H, per_head, bf16, chunks;  // chunks: CTAs per (b, h) slice
+  int64_t nvec;      // B * H * L * d / 8: 16-byte input vectors in all
+  int64_t seg;       // vectors sharing one scale: L * d / 8 per head, or nvec
+  int32_t H, per_head, bf16, n_scales;
 };
 
 namespace quant {
 
 constexpr int kThreads = 256;
 constexpr int kVec = 8;                          // elements per 16-byte load
-constexpr int kIters = 16;                       // loads per thread and CTA
-constexpr int kChunkElems = kThreads * kVec * kIters;  // 32768 elements per CTA
+constexpr int kBatch = 8;                        // loads in flight per thread
+constexpr int kStep = kThreads * kBatch;         // vectors per CTA and batch
+
+constexpr unsigned kRoleGridBarrier = 4;  // role bits of a quant_fused timeout
+
+// Programmatic dependent launch: a grid launched with programmatic stream
+// serialisation may start once its predecessor has triggered (or exited);
+// griddep_wait returns when the predecessor has completed and its writes
+// are visible.
+__device__ __forceinline__ void griddep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void griddep_trigger() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
+// Waits until *ctr >= target (acquire, gpu scope).  Returns false and records
+// the error after kWaitTimeoutNs.
+__device__ __forceinline__ bool wait_count(const uint32_t* ctr, uint32_t target) {
+  uint32_t v;
+  asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(ctr) : "memory");
+  if (v >= target) return true;
+  const unsigned long long t0 = globaltimer_ns();
+  while (true) {
+    __nanosleep(20);
+    asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(ctr) : "memory");
+    if (v >= target) return true;
+    if (globaltimer_ns() - t0 > kWaitTimeoutNs) {
+      atomicOr(&g_device_error, kErrTimeout | (kRoleGridBarrier << 8));
+      return false;
+    }
+  }
+}
+
+// Vector range [lo, hi) of CTA `b` of `g`: equal shares, +-1.
+__device__ __forceinline__ void cta_range(int64_t n, int64_t& lo, int64_t& hi) {
+  const int64_t b = blockIdx.x, g = gridDim.x;
+  lo = n / g * b + min(b, n % g);
+  hi = lo + n / g + (b < n % g ? 1 : 0);
+}
 
 __device__ __forceinline__ void to_float8(uint4 v, bool bf16, float (&f)[8]) {
   const uint32_t w[4] = {v.x, v.y, v.z, v.w};
@@ -63,61 +107,150 @@ __device__ __forceinline__ float inv_scale_of(uint32_t amax_bits) {
   return amax == 0.0f ? 1.0f : fminf(__fdiv_rn(127.0f, amax), 3.402823466e38f);
 }
 
-// grid (chunks, B*H)
-__global__ void __launch_bounds__(kThreads) quant_amax_kernel(const __grid_constant__ QuantArgs a) {
-  const int bh = blockIdx.y;
-  const int64_t e0 = static_cast<int64_t>(blockIdx.x) * kChunkElems;
-  const uint4* src = reinterpret_cast<const uint4*>(static_cast<const uint16_t*>(a.x) + bh * a.slice);
-  float m = 0.0f;
+// Codes of 8 elements.  p = x * inv (fp32, rounded to nearest); adding
+// 1.5 * 2^23 rounds p to an integer q with ties to even (|p| < 2^22) and
+// leaves 0x400000 + q in the mantissa, so the low byte of the sum's bits is q
+// as a two's complement byte.  The clamp to [-127, 127] of the definition
+// never binds here: |x| <= amax gives |p| <= RN(amax * RN(127 / amax)) <=
+// 127 * (1 + 2^-24), which rounds to at most 127, and with inv capped at
+// FLT_MAX (amax < 127 / FLT_MAX) |p| <= amax * FLT_MAX < 127.
+// RN(x * m) on a pair of floats (one packed multiply).
+__device__ __forceinline__ float2 mul_rn2(float x0, float x1, float m) {
+  float2 r;
+  asm("{\n\t.reg .b64 xa, ma, pa;\n\t"
+      "mov.b64 xa, {%2, %3};\n\t"
+      "mov.b64 ma, {%4, %4};\n\t"
+      "mul.rn.f32x2 pa, xa, ma;\n\t"
+      "mov.b64 {%0, %1}, pa;\n\t}"
+      : "=f"(r.x), "=f"(r.y)
+      : "f"(x0), "f"(x1), "f"(m));
+  return r;
+}
+
+__device__ __forceinline__ uint2 codes8(uint4 v, bool bf16, float inv) {
+  constexpr float kRound = 12582912.0f;  // 1.5 * 2^23
+  float f[8];
+  to_float8(v, bf16, f);
+  uint32_t t[8];
 #pragma unroll
-  for (int it = 0; it < kIters; ++it) {
-    const int64_t e = e0 + (static_cast<int64_t>(it) * kThreads + threadIdx.x) * kVec;
-    if (e < a.slice) {
-      float f[8];
-      to_float8(__ldg(src + e / kVec), a.bf16, f);
-#pragma unroll
-      for (int i = 0; i < 8; ++i) m = fmaxf(m, fabsf(f[i]));
-    }
+  for (int i = 0; i < 4; ++i) {
+    // the adds are scalar with explicit rounding: a packed add after the
+    // packed multiply was contracted into one fused operation
+    const float2 p = mul_rn2(f[2 * i], f[2 * i + 1], inv);
+    t[2 * i] = __float_as_uint(__fadd_rn(p.x, kRound));
+    t[2 * i + 1] = __float_as_uint(__fadd_rn(p.y, kRound));
   }
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+  return make_uint2(__byte_perm(__byte_perm(t[0], t[1], 0x0040), __byte_perm(t[2], t[3], 0x0040), 0x5410),
+                    __byte_perm(__byte_perm(t[4], t[5], 0x0040), __byte_perm(t[6], t[7], 0x0040), 0x5410));
+}
+
+// 1-D cooperative grid of at most one CTA per resident slot
+__global__ void __launch_bounds__(kThreads) quant_fused_kernel(const __grid_constant__ QuantArgs a) {
+  const uint4* src = static_cast<const uint4*>(a.x);
+  uint2* dst = reinterpret_cast<uint2*>(a.out);
+  uint32_t* arrive = reinterpret_cast<uint32_t*>(a.out);  // code bytes 0-3 until the end
+  uint32_t* depart = arrive + 1;                           // code bytes 4-7
   __shared__ float red[kThreads / 32];
-  if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = m;
+  __shared__ int ok;
+  int64_t lo0, hi;
+  cta_range(a.nvec, lo0, hi);
+
+  // pass 1: max |x| per head segment of the range (the loads start while
+  // quant_zero may still run)
+  bool zeroed = false;
+  for (int64_t lo = lo0; lo < hi;) {
+    const int64_t seg_id = lo / a.seg;
+    const int64_t end = min(hi, (seg_id + 1) * a.seg);
+    float m = 0.0f;
+    for (int64_t base = lo; base < end; base += kStep) {
+      // all of a batch's loads are issued before any is used
+      uint4 v[kBatch];
+#pragma unroll
+      for (int it = 0; it < kBatch; ++it) {
+        const int64_t e = base + it * kThreads + threadIdx.x;
+        v[it] = e < end ? __ldg(src + e) : make_uint4(0, 0, 0, 0);  // 0 = +0.0 in both types
+      }
+#pragma unroll
+      for (int it = 0; it < kBatch; ++it) {
+        float f[8];
+        to_float8(v[it], a.bf16, f);
+#pragma unroll
+        for (int i = 0; i < 8; ++i) m = fmaxf(m, fabsf(f[i]));
+      }
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+    if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = m;
+    __syncthreads();
+    if (threadIdx.x == 0) {
+      for (int w = 1; w < kThreads / 32; ++w) m = fmaxf(m, red[w]);
+      if (!zeroed) griddep_wait();  // quant_zero has completed
+      zeroed = true;
+      atomicMax(a.amax + (a.per_head ? static_cast<int>(seg_id % a.H) : 0), __float_as_uint(m));
+    }
+    __syncthreads();  // red is reused by the next segment
+    lo = end;
+  }
+
+  // grid barrier: every amax merged
+  if (threadIdx.x == 0) {
+    if (!zeroed) griddep_wait();
+    __threadfence();
+    atomicAdd(arrive, 1u);
+    ok = wait_count(arrive, gridDim.x);
+  }
+  __syncthreads();
+  if (!ok) return;
+
+  // pass 2: codes, batches in the reverse order of pass 1 (the last ones
+  // read are still in L1); vector 0 (the counters) is kept for the end
+  uint2 first = make_uint2(0, 0);
+  for (int64_t top = hi; top > lo0;) {
+    const int64_t seg_id = (top - 1) / a.seg;
+    const int64_t start = max(lo0, seg_id * a.seg);
+    const float inv = inv_scale_of(__ldcg(a.amax + (a.per_head ? static_cast<int>(seg_id % a.H) : 0)));
+    for (int64_t base = start + (top - 1 - start) / kStep * kStep; base >= start; base -= kStep) {
+      uint4 v[kBatch];
+#pragma unroll
+      for (int it = 0; it < kBatch; ++it) {
+        const int64_t e = base + it * kThreads + threadIdx.x;
+        v[it] = e < top ? __ldg(src + e) : make_uint4(0, 0, 0, 0);
+      }
+#pragma unroll
+      for (int it = 0; it < kBatch; ++it) {
+        const int64_t e = base + it * kThreads + threadIdx.x;
+        if (e < top) {
+          const uint2 c = codes8(v[it], a.bf16, inv);
+          if (e == 0) first = c;
+          else dst[e] = c;
+        }
+      }
+    }
+    top = start;
+  }
+
+  // every CTA is past its last read of amax and of the arrival counter
   __syncthreads();
   if (threadIdx.x == 0) {
-    for (int w = 1; w < kThreads / 32; ++w) m = fmaxf(m, red[w]);
-    const int slot = a.per_head ? bh % a.H : 0;
-    atomicMax(a.amax + slot, __float_as_uint(m));
+    __threadfence();
+    atomicAdd(depart, 1u);
   }
+  if (blockIdx.x != 0) return;
+  if (threadIdx.x == 0) ok = wait_count(depart, gridDim.x);
+  __syncthreads();
+  if (!ok) return;
+  for (int i = threadIdx.x; i < a.n_scales; i += kThreads) a.amax[i] = __float_as_uint(scale_of(__ldcg(a.amax + i)));
+  if (threadIdx.x == 0) dst[0] = first;  // thread 0 of CTA 0 owns vector 0
 }
 
-// grid (chunks, B*H)
-__global__ void __launch_bounds__(kThreads) quant_codes_kernel(const __grid_constant__ QuantArgs a) {
-  const int bh = blockIdx.y;
-  const int64_t e0 = static_cast<int64_t>(blockIdx.x) * kChunkElems;
-  const uint4* src = reinterpret_cast<const uint4*>(static_cast<const uint16_t*>(a.x) + bh * a.slice);
-  uint2* dst = reinterpret_cast<uint2*>(a.out + bh * a.slice);
-  const float inv = inv_scale_of(__ldcg(a.amax + (a.per_head ? bh % a.H : 0)));
-#pragma unroll
-  for (int it = 0; it < kIters; ++it) {
-    const int64_t e = e0 + (static_cast<int64_t>(it) * kThreads + threadIdx.x) * kVec;
-    if (e < a.slice) {
-      float f[8];
-      to_float8(__ldg(src + e / kVec), a.bf16, f);
-      uint32_t b[8];
-#pragma unroll
-      for (int i = 0; i < 8; ++i) {
-        int q = __float2int_rn(__fmul_rn(f[i], inv));
-        q = q > 127 ? 127 : (q < -127 ? -127 : q);
-        b[i] = static_cast<uint32_t>(q) & 0xFFu;
-      }
-      dst[e / kVec] = make_uint2(b[0] | (b[1] << 8) | (b[2] << 16) | (b[3] << 24),
-                                 b[4] | (b[5] << 8) | (b[6] << 16) | (b[7] << 24));
-    }
-  }
+// one CTA: zero the amax slots and the two barrier counters
+__global__ void quant_zero_kernel(uint32_t* amax, int n, uint32_t* counters) {
+  griddep_trigger();  // quant_fused waits for completion before it uses these
+  for (int i = threadIdx.x; i < n; i += blockDim.x) amax[i] = 0u;
+  if (threadIdx.x < 2) counters[threadIdx.x] = 0u;
 }
 
-// one CTA: amax bits -> the float scale, in place
+// one CTA: amax bits -> the float scale, in place (the empty tensor: s = 1)
 __global__ void quant_scales_kernel(uint32_t* amax, int n) {
   for (int i = threadIdx.x; i < n; i += blockDim.x) amax[i] = __float_as_uint(scale_of(amax[i]));
 }

@@ -35,7 +35,9 @@ def _inputs(shape, seed, dtype, spread=(0.01, 30.0), outlier=40.0):
 
 
 CASES = [((1, 1, 1, 8), False), ((2, 3, 37, 64), True), ((2, 3, 37, 64), False), ((1, 4, 512, 128), True),
-         ((3, 2, 1000, 64), True), ((8, 12, 512, 64), False)]
+         ((3, 2, 1000, 64), True), ((8, 12, 512, 64), False),
+         # one CTA over 256 one-vector heads; a full grid over 32 heads of 256K elements
+         ((4, 64, 1, 8), True), ((1, 32, 2048, 128), True)]
 
 
 @pytest.mark.parametrize("dtype_name", ["bfloat16", "float16"])
@@ -62,6 +64,36 @@ def test_quantize_ties_round_half_to_even(ia):
     codes, scales = ia.quantize(x.cuda(), True)
     assert scales.cpu().tolist() == [1.0]
     assert codes.cpu().numpy().ravel()[:10].tolist() == [127, -127, 0, 2, 2, 0, -2, -2, 62, -64]
+
+
+def test_quantize_product_rounded_before_rint(ia):
+    """amax 4.84375, x 2.421875: the exact x * inv lies just below 63.5 but
+    the fp32 product is 63.5, a tie that goes to 64; a fused multiply-add
+    would give 63."""
+    import torch
+    x = torch.tensor([4.84375, 2.421875, -2.421875] + [0.0] * 5, dtype=torch.bfloat16).reshape(1, 1, 1, 8)
+    inv = np.float32(127.0) / np.float32(4.84375)
+    assert np.float32(2.421875) * inv == np.float32(63.5)
+    assert 2.421875 * float(inv) < 63.5
+    codes, _ = ia.quantize(x.cuda(), True)
+    assert codes.cpu().numpy().ravel()[:3].tolist() == [127, 64, -64]
+    want, _ = oq.quantize(x.float().numpy(), True)
+    assert want.ravel()[:3].tolist() == [127, 64, -64]
+
+
+def test_quantize_reuses_buffers(ia):
+    """Second call into the same code and scale buffers (whose first bytes
+    the call uses as scratch) gives the oracle's result again."""
+    import torch
+    shape = (2, 8, 300, 64)
+    out = torch.full(shape, 77, dtype=torch.int8, device="cuda")
+    sc = torch.full((8,), 5.0, dtype=torch.float32, device="cuda")
+    for seed in (1, 2):
+        t, x32 = _inputs(shape, seed, torch.bfloat16)
+        ia.quantize(t.cuda(), True, out=out, scales=sc)
+        want_codes, want_scales = oq.quantize(x32, True)
+        assert np.array_equal(sc.cpu().numpy(), want_scales)
+        assert np.array_equal(out.cpu().numpy(), want_codes)
 
 
 def test_quantize_empty_and_zero(ia):
