@@ -302,6 +302,7 @@ def run_ours(args):
         line["decode_int4"] = run_decode(args, dev, stream, world, peaks, peak_src,
                                          "llama7b_decode_int4_b64_lk4096")
         line["quantize"] = run_quantize(args, dev, stream, world, peaks, peak_src)
+        line["gelu"] = run_gelu(args, dev, stream, world, peaks, peak_src)
     if not args.no_cpu_baseline and rank == 0 and world == 1:
         line["cpu_baseline"] = cpu_baseline(w, x, args.cpu_seconds)
     if rank == 0:
@@ -347,6 +348,43 @@ def run_quantize(args, dev, stream, world, peaks, peak_src):
                          "frac": round(gbs / peaks["hbm_gbs"], 4), "peak_source": f"{peak_src} hbm_gbs",
                          "traffic": None},
             "l2": "inputs rotate over 3 copies (201 MB > 126 MB L2)"}
+
+
+def run_gelu(args, dev, stream, world, peaks, peak_src):
+    """Integer GELU over GPT-2-small MLP activations (int8 [16*1024, 3072]):
+    GB/s of the int8 read + int8 write."""
+    import torch
+
+    import integer_only_quantized_b200 as ia
+    from integer_only_quantized_b200 import workloads as wl
+    name = "gpt2_small_mlp_gelu_b16_l1024_f3072"
+    spec = wl.GELU_WORKLOADS[name]
+    ins = [wl.gelu_inputs_torch(spec["tokens"], spec["features"], 20251126 + i, dev) for i in range(4)]
+    xs = [c for c, _ in ins]
+    s_x = ins[0][1]
+    n = xs[0].numel()
+    out = torch.empty_like(xs[0])
+    steps = max(10, min(args.steps, 100))
+    for i in range(max(3, args.warmup)):
+        ia.gelu(xs[i % 4], s_x, s_x, spec["c"], out=out, stream=stream)
+    torch.cuda.synchronize(dev)
+    barrier(world, dev)
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    t0.record(stream)
+    for i in range(steps):
+        ia.gelu(xs[i % 4], s_x, s_x, spec["c"], out=out, stream=stream)
+    t1.record(stream)
+    torch.cuda.synchronize(dev)
+    barrier(world, dev)
+    ms = max_over_ranks(t0.elapsed_time(t1) / steps, world, dev)
+    algo = 2 * n  # 1 byte read + 1 byte written per element
+    gbs = algo / (ms * 1e-3) / 1e9
+    return {"workload": name, "value": round(aggregate_value(algo, world, ms * 1e-3) / 1e9, 1), "unit": "GB/s",
+            "ms_per_call": round(ms, 5), "launches_per_call": 1, "bytes_per_call": algo,
+            "roofline": {"bound": "hbm", "achieved": round(gbs, 1), "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                         "frac": round(gbs / peaks["hbm_gbs"], 4), "peak_source": f"{peak_src} hbm_gbs",
+                         "traffic": kernel_traffic("gelu_kernel", name)},
+            "l2": "inputs rotate over 4 copies (201 MB > 126 MB L2)"}
 
 
 def run_decode(args, dev, stream, world, peaks, peak_src, name):

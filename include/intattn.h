@@ -163,6 +163,36 @@ enum { INTATTN_DTYPE_FP16 = 0, INTATTN_DTYPE_BF16 = 1 };
 int intattn_quantize(const void *x, int dtype, int B, int H, int L, int d, int per_head, int8_t *out,
                      float *scales, intattn_stream_t stream);
 
+/* Integer GELU (the summary page "[Paper] IntAttention：全整数注意力流水线用于
+ * 高效边缘推理", section 局限性与未来工作, names GELU as the next operator for the
+ * method; this definition is the library's reading of "the same machinery":
+ * an index by integer multiply and shift, a 32-entry integer gate table, a
+ * requantising multiply and shift).  Real values: x = s_x * q, y = s_y * out.
+ *   r = (s_x * 31) / (2c); s = 26, lowered while llround(r 2^s) > 2^24;
+ *   M = llround(r 2^s) in [1, 2^24]
+ *   gate[i] = llround(32768 * (0.5 * erfc(-t_i / sqrt 2))), t_i = ((2i - 31) c) / 31,
+ *   i = 1..30; gate[0] = 0, gate[31] = 32768
+ *   m = s_x / (32768 s_y) = f 2^e; Mo = llround(f 2^31) (2^31 -> 2^30, e+1);
+ *   so = 31 - e in [1, 62]
+ *   per element: idx = clamp(16 + floor(q M / 2^s), 0, 31); y = q * gate[idx];
+ *   out = clamp(floor((y Mo + 2^(so-1)) / 2^so), -127, 127)
+ * (IEEE double in that order; llround rounds half away from zero.) */
+typedef struct {
+    int32_t M, s;       /* index multiplier and shift */
+    int32_t Mo, so;     /* requant multiplier and shift */
+    int32_t gate[32];   /* 2^15 * Phi at the 32 table points */
+} intattn_gelu_params_t;
+
+/* Host only: the parameters above.  PARAM_RANGE for a scale or c that is not
+ * finite and > 0, or M / so out of range; INVALID_ARG for out == NULL. */
+int intattn_gelu_derive_params(float s_x, float s_y, float c, intattn_gelu_params_t *out);
+
+/* y[i] = integer GELU of x[i], i < n.  x, y: device, 16-byte aligned; y == x
+ * (in place) is allowed, any other overlap is INVALID_ARG.  n == 0 launches
+ * nothing.  One launch, asynchronous on `stream`. */
+int intattn_gelu(const int8_t *x, int8_t *y, long long n, float s_x, float s_y, float c,
+                 intattn_stream_t stream);
+
 /* Capacity in bytes of the library's static decode scratch (48 MiB). */
 #define INTATTN_STATIC_SCRATCH_BYTES (48u * 1024u * 1024u)
 

@@ -24,8 +24,14 @@ MAX_CLIPS = 8
 # every function declared in include/intattn.h
 EXPORTED = ("intattn_derive_params", "intattn_forward", "intattn_decode_workspace_size",
             "intattn_decode", "intattn_decode_int4", "intattn_decode_static_scratch", "intattn_quantize",
-            "intattn_selftest_timeout", "intattn_device_error", "intattn_strerror")
+            "intattn_gelu_derive_params", "intattn_gelu", "intattn_selftest_timeout", "intattn_device_error",
+            "intattn_strerror")
 DTYPE_FP16, DTYPE_BF16 = 0, 1
+
+
+class _GeluParams(ctypes.Structure):
+    _fields_ = [("M", ctypes.c_int32), ("s", ctypes.c_int32), ("Mo", ctypes.c_int32), ("so", ctypes.c_int32),
+                ("gate", ctypes.c_int32 * 32)]
 
 
 class IntAttnError(RuntimeError):
@@ -101,6 +107,8 @@ def lib() -> ctypes.CDLL:
         L.intattn_decode_static_scratch.argtypes = [vp, vp, vp, ctypes.POINTER(_Scales), i32, i32, i32,
                                                     i32, i32, f32, vp, vp]
         L.intattn_quantize.argtypes = [vp, i32, i32, i32, i32, i32, i32, vp, vp, vp]
+        L.intattn_gelu_derive_params.argtypes = [f32, f32, f32, ctypes.POINTER(_GeluParams)]
+        L.intattn_gelu.argtypes = [vp, vp, ctypes.c_longlong, f32, f32, f32, vp]
         L.intattn_selftest_timeout.argtypes = [vp]
         L.intattn_device_error.argtypes = [vp]
         L.intattn_strerror.argtypes = [i32]
@@ -262,6 +270,30 @@ def quantize(x, per_head: bool, out=None, scales=None, stream=None):
     _check(lib().intattn_quantize(x.data_ptr(), dt, B, H, L, d, int(bool(per_head)), out.data_ptr(),
                                   scales.data_ptr(), _stream_handle(stream, x.device)), "intattn_quantize")
     return out, scales
+
+
+def gelu_params(s_x: float, s_y: float, c: float):
+    """(M, s, gate[32], Mo, so) of the integer GELU, as the kernel uses them."""
+    p = _GeluParams()
+    _check(lib().intattn_gelu_derive_params(float(s_x), float(s_y), float(c), ctypes.byref(p)),
+           "intattn_gelu_derive_params")
+    return p.M, p.s, list(p.gate), p.Mo, p.so
+
+
+def gelu(x, s_x: float, s_y: float, c: float, out=None, stream=None):
+    """Integer GELU of a contiguous CUDA int8 tensor (any shape): int8 codes
+    of scale s_y for codes x of scale s_x; gate tabulated on [-c, c].
+    out may be x itself (in place)."""
+    _check_tensor(x, "x")
+    if out is None:
+        import torch
+        out = torch.empty_like(x)
+    _check_tensor(out, "out")
+    if out.numel() != x.numel():
+        raise ValueError("out must have as many elements as x")
+    _check(lib().intattn_gelu(x.data_ptr(), out.data_ptr(), x.numel(), float(s_x), float(s_y), float(c),
+                              _stream_handle(stream, x.device)), "intattn_gelu")
+    return out
 
 
 def device_error(stream=None) -> int:

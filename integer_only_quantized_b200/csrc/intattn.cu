@@ -17,6 +17,7 @@
 #include "intattn.h"
 
 #include "decode_kernel.cuh"
+#include "gelu_kernel.cuh"
 #include "quantize_kernel.cuh"
 #include "prefill_kernel.cuh"
 
@@ -491,6 +492,86 @@ int intattn_quantize(const void* x, int dtype, int B, int H, int L, int d, int p
   cfg.attrs = attrs;
   cfg.numAttrs = 2;
   return note_launch(cudaLaunchKernelEx(&cfg, intattn::quant::quant_fused_kernel, a));
+}
+
+namespace {
+
+// Integer GELU parameters, IEEE double in the definition's order: index
+// r = s_x 31 / (2c) as M / 2^s (M <= 2^24, s <= 26), the gate table
+// G[i] = llround(2^15 Phi((2i - 31) c / 31)) with G[0] = 0 and G[31] = 2^15,
+// and the requant m = s_x / (2^15 s_y) as Mo / 2^so.
+int gelu_derive(float s_x_f, float s_y_f, float c_f, intattn_gelu_params_t* p) {
+  const double s_x = s_x_f, s_y = s_y_f, c = c_f;
+  if (!(std::isfinite(s_x) && s_x > 0.0 && std::isfinite(s_y) && s_y > 0.0 && std::isfinite(c) && c > 0.0))
+    return INTATTN_ERR_PARAM_RANGE;
+  const double r = (s_x * 31.0) / (2.0 * c);
+  if (!(r < 1e15)) return INTATTN_ERR_PARAM_RANGE;  // M > 2^24 at every shift
+  int sh = 26;
+  while (sh > 1 && std::llround(std::ldexp(r, sh)) > (1LL << 24)) --sh;
+  const long long M = std::llround(std::ldexp(r, sh));
+  if (M < 1 || M > (1LL << 24)) return INTATTN_ERR_PARAM_RANGE;
+  p->M = static_cast<int32_t>(M);
+  p->s = sh;
+  p->gate[0] = 0;
+  p->gate[31] = 32768;
+  for (int i = 1; i < 31; ++i) {
+    const double t = (static_cast<double>(2 * i - 31) * c) / 31.0;
+    p->gate[i] = static_cast<int32_t>(std::llround(32768.0 * (0.5 * std::erfc(-t / std::sqrt(2.0)))));
+  }
+  const double m = s_x / (32768.0 * s_y);
+  int e = 0;
+  const double f = std::frexp(m, &e);
+  long long Mo = std::llround(f * 2147483648.0);
+  if (Mo == (1LL << 31)) {
+    Mo = 1LL << 30;
+    ++e;
+  }
+  const int so = 31 - e;
+  if (so < 1 || so > 62) return INTATTN_ERR_PARAM_RANGE;
+  p->Mo = static_cast<int32_t>(Mo);
+  p->so = so;
+  return INTATTN_OK;
+}
+
+}  // namespace
+
+int intattn_gelu_derive_params(float s_x, float s_y, float c, intattn_gelu_params_t* out) {
+  if (!out) return INTATTN_ERR_INVALID_ARG;
+  return gelu_derive(s_x, s_y, c, out);
+}
+
+int intattn_gelu(const int8_t* x, int8_t* y, long long n, float s_x, float s_y, float c, intattn_stream_t stream) {
+  if (n < 0) return INTATTN_ERR_INVALID_ARG;
+  intattn_gelu_params_t p;
+  int rc = gelu_derive(s_x, s_y, c, &p);
+  if (rc) return rc;
+  if (n == 0) return INTATTN_OK;
+  if (!x || !y) return INTATTN_ERR_INVALID_ARG;
+  if (!aligned16(x) || !aligned16(y)) return INTATTN_ERR_UNSUPPORTED;
+  const uintptr_t xa = reinterpret_cast<uintptr_t>(x), ya = reinterpret_cast<uintptr_t>(y);
+  if (xa != ya && xa < ya + static_cast<uintptr_t>(n) && ya < xa + static_cast<uintptr_t>(n))
+    return INTATTN_ERR_INVALID_ARG;  // partial overlap (in place is fine)
+  intattn::GeluArgs a;
+  a.x = x;
+  a.y = y;
+  a.n = n;
+  a.M = p.M;
+  a.s = p.s;
+  a.Mo = p.Mo;
+  a.so = p.so;
+  for (int i = 0; i < 32; ++i) a.gate[i] = p.gate[i];
+  int sms = 0;
+  if (sm_count(&sms) != INTATTN_OK) return INTATTN_ERR_CUDA;
+  int occ = 0;
+  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, intattn::gelu::gelu_kernel, intattn::gelu::kThreads, 0) !=
+          cudaSuccess ||
+      occ < 1)
+    return note_launch(cudaGetLastError());
+  const long long per_cta = static_cast<long long>(intattn::gelu::kThreads) * intattn::gelu::kBatch;
+  const long long want = std::max(1LL, ((n >> 4) + per_cta - 1) / per_cta);
+  const unsigned grid = static_cast<unsigned>(std::min<long long>(want, static_cast<long long>(sms) * occ));
+  intattn::gelu::gelu_kernel<<<grid, intattn::gelu::kThreads, 0, reinterpret_cast<cudaStream_t>(stream)>>>(a);
+  return note_launch(cudaGetLastError());
 }
 
 int intattn_selftest_timeout(intattn_stream_t stream) {

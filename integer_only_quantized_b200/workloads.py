@@ -311,3 +311,29 @@ def pack_int4_torch(x):
     import torch
     u = (x.to(torch.int16) & 0x0F).to(torch.uint8)
     return (u[..., 0::2] | (u[..., 1::2] << 4)).contiguous()
+
+
+# ------------------------------------------------------------- integer GELU
+# GELU input: the pre-activation of a transformer MLP (GPT-2 small: hidden
+# 768 -> 3072).  Recipe: N(0, 1.5) draws, 1 % of the 3072 channels scaled by
+# 4 (outlier channels), per-tensor symmetric int8 with s_x = max|x| / 127,
+# s_y = s_x (GELU(x) <= max(x, 0)), gate range c = 4.
+GELU_WORKLOADS = {
+    "gpt2_small_mlp_gelu_b16_l1024_f3072": dict(tokens=16 * 1024, features=3072, c=4.0),
+    "gelu_small_t512_f768": dict(tokens=512, features=768, c=4.0),
+}
+
+
+def gelu_inputs_torch(tokens: int, features: int, seed: int, device):
+    """(codes int8 [tokens, features], s_x) drawn on `device`."""
+    import torch
+    g = torch.Generator(device=device)
+    g.manual_seed(seed)
+    x = torch.randn((tokens, features), generator=g, device=device, dtype=torch.float32) * 1.5
+    n_out = max(1, round(0.01 * features))
+    ch = torch.randperm(features, generator=g, device=device)[:n_out]
+    x[:, ch] *= 4.0
+    amax = float(x.abs().max())
+    s_x = float(np.float32(amax / 127.0)) if amax > 0 else 1.0
+    codes = torch.clamp(torch.round(x / s_x), -127, 127).to(torch.int8)
+    return codes, s_x
