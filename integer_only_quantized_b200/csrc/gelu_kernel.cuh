@@ -32,7 +32,7 @@ struct GeluArgs {
 namespace gelu {
 
 constexpr int kThreads = 256;
-constexpr int kBatch = 4;  // 16-byte loads in flight per thread
+constexpr int kBatch = 8;  // 16-byte loads in flight per thread
 
 // The definition for one code.
 __device__ __forceinline__ uint32_t code_of(int q, const GeluArgs& a) {
@@ -46,7 +46,7 @@ __device__ __forceinline__ uint32_t code_of(int q, const GeluArgs& a) {
 
 __device__ __forceinline__ uint4 ld_stream16(const uint4* p) {
   uint4 r;
-  asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0, %1, %2, %3}, [%4];"
+  asm volatile("ld.global.nc.L1::no_allocate.L2::256B.v4.u32 {%0, %1, %2, %3}, [%4];"
                : "=r"(r.x), "=r"(r.y), "=r"(r.z), "=r"(r.w)
                : "l"(p));
   return r;
