@@ -45,6 +45,8 @@ def parse_args(argv=None):
     p.add_argument("--no-decode", action="store_true")
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--cpu-seconds", type=float, default=12.0)
+    p.add_argument("--leg", choices=["decode", "decode_int4", "quantize", "gelu"], default=None,
+                   help="run only this secondary leg and print its object (for profiler captures)")
     return p.parse_args(argv)
 
 
@@ -187,6 +189,30 @@ class ClockSampler:
 def _int8_peak(peaks, sustained: bool):
     key = "bf16_tflops_sustained" if sustained and "bf16_tflops_sustained" in peaks else "bf16_tflops"
     return peaks[key] * INT8_OVER_BF16, key
+
+
+def run_leg(args):
+    """One secondary leg alone: its device footprint is its own inputs only."""
+    import torch
+    rank, local_rank, world = dist_env()
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    init_dist(world, "nccl")
+    stream = torch.cuda.current_stream(dev)
+    peaks, peak_src = load_peaks()
+    if args.leg == "decode":
+        out = run_decode(args, dev, stream, world, peaks, peak_src, args.decode_workload)
+    elif args.leg == "decode_int4":
+        out = run_decode(args, dev, stream, world, peaks, peak_src, "llama7b_decode_int4_b64_lk4096")
+    elif args.leg == "quantize":
+        out = run_quantize(args, dev, stream, world, peaks, peak_src)
+    else:
+        out = run_gelu(args, dev, stream, world, peaks, peak_src)
+    if rank == 0:
+        print(json.dumps({"leg": args.leg, **out}), flush=True)
+    if world > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
 
 
 def run_ours(args):
@@ -501,6 +527,8 @@ def main(argv=None):
     args = parse_args(argv)
     if args.impl == "reference":
         run_reference(args)
+    elif args.leg:
+        run_leg(args)
     else:
         run_ours(args)
 
