@@ -31,7 +31,7 @@ struct GeluArgs {
 
 namespace gelu {
 
-constexpr int kThreads = 256;
+constexpr int kThreads = 256;  // the table build assumes 256 (one code per thread)
 constexpr int kBatch = 8;  // 16-byte loads in flight per thread
 
 // The definition for one code.
@@ -77,12 +77,17 @@ __global__ void __launch_bounds__(kThreads) gelu_kernel(const __grid_constant__ 
     const int64_t e = base + it * kThreads + threadIdx.x;
     v[it] = e < nvec ? ld_stream16(src + e) : make_uint4(0, 0, 0, 0);
   }
-  // table: thread t evaluates code (int8)(t) once and writes its 32 copies
-  {
-    const uint32_t out = code_of(static_cast<int8_t>(threadIdx.x), a);
-    uint4* row = reinterpret_cast<uint4*>(tab + threadIdx.x * 32);
+  // table: thread t evaluates code (int8)(t) once; then each warp writes 512
+  // contiguous bytes per store (16-byte stores of one entry's copies), which
+  // touches every bank once
+  __shared__ uint32_t codes[256];
+  codes[threadIdx.x] = code_of(static_cast<int8_t>(threadIdx.x), a);
+  __syncthreads();
 #pragma unroll
-    for (int i = 0; i < 8; ++i) row[i] = make_uint4(out, out, out, out);
+  for (int k = 0; k < 8; ++k) {
+    const uint32_t w = 4u * threadIdx.x + 1024u * k;  // first of 4 words, all of entry w / 32
+    const uint32_t out = codes[w >> 5];
+    *reinterpret_cast<uint4*>(tab + w) = make_uint4(out, out, out, out);
   }
   __syncthreads();
 
