@@ -161,23 +161,31 @@ __global__ void __launch_bounds__(kThreads) quant_fused_kernel(const __grid_cons
   for (int64_t lo = lo0; lo < hi;) {
     const int64_t seg_id = lo / a.seg;
     const int64_t end = min(hi, (seg_id + 1) * a.seg);
-    float m = 0.0f;
+    // max |x| as 16-bit patterns, two per word: with the sign bit cleared,
+    // finite fp16 / bf16 values order like their unsigned bit patterns
+    uint32_t mh = 0;
     for (int64_t base = lo; base < end; base += kStep) {
       // all of a batch's loads are issued before any is used
       uint4 v[kBatch];
+      const uint4* p = src + base + threadIdx.x;
+      if (base + kStep <= end) {
 #pragma unroll
-      for (int it = 0; it < kBatch; ++it) {
-        const int64_t e = base + it * kThreads + threadIdx.x;
-        v[it] = e < end ? __ldg(src + e) : make_uint4(0, 0, 0, 0);  // 0 = +0.0 in both types
+        for (int it = 0; it < kBatch; ++it) v[it] = __ldg(p + it * kThreads);
+      } else {
+#pragma unroll
+        for (int it = 0; it < kBatch; ++it)
+          v[it] = base + it * kThreads + threadIdx.x < end ? __ldg(p + it * kThreads) : make_uint4(0, 0, 0, 0);
       }
 #pragma unroll
       for (int it = 0; it < kBatch; ++it) {
-        float f[8];
-        to_float8(v[it], a.bf16, f);
-#pragma unroll
-        for (int i = 0; i < 8; ++i) m = fmaxf(m, fabsf(f[i]));
+        mh = __vmaxu2(mh, v[it].x & 0x7FFF7FFFu);
+        mh = __vmaxu2(mh, v[it].y & 0x7FFF7FFFu);
+        mh = __vmaxu2(mh, v[it].z & 0x7FFF7FFFu);
+        mh = __vmaxu2(mh, v[it].w & 0x7FFF7FFFu);
       }
     }
+    const uint32_t m16 = max(mh & 0xFFFFu, mh >> 16);
+    float m = a.bf16 ? __uint_as_float(m16 << 16) : __half2float(__ushort_as_half(static_cast<unsigned short>(m16)));
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
     if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = m;
@@ -211,18 +219,25 @@ __global__ void __launch_bounds__(kThreads) quant_fused_kernel(const __grid_cons
     const float inv = inv_scale_of(__ldcg(a.amax + (a.per_head ? static_cast<int>(seg_id % a.H) : 0)));
     for (int64_t base = start + (top - 1 - start) / kStep * kStep; base >= start; base -= kStep) {
       uint4 v[kBatch];
+      const uint4* p = src + base + threadIdx.x;
+      uint2* q = dst + base + threadIdx.x;
+      if (base + kStep <= top && base != 0) {  // a full batch without vector 0
 #pragma unroll
-      for (int it = 0; it < kBatch; ++it) {
-        const int64_t e = base + it * kThreads + threadIdx.x;
-        v[it] = e < top ? __ldg(src + e) : make_uint4(0, 0, 0, 0);
-      }
+        for (int it = 0; it < kBatch; ++it) v[it] = __ldg(p + it * kThreads);
 #pragma unroll
-      for (int it = 0; it < kBatch; ++it) {
-        const int64_t e = base + it * kThreads + threadIdx.x;
-        if (e < top) {
-          const uint2 c = codes8(v[it], a.bf16, inv);
-          if (e == 0) first = c;
-          else dst[e] = c;
+        for (int it = 0; it < kBatch; ++it) q[it * kThreads] = codes8(v[it], a.bf16, inv);
+      } else {
+#pragma unroll
+        for (int it = 0; it < kBatch; ++it)
+          v[it] = base + it * kThreads + threadIdx.x < top ? __ldg(p + it * kThreads) : make_uint4(0, 0, 0, 0);
+#pragma unroll
+        for (int it = 0; it < kBatch; ++it) {
+          const int64_t e = base + it * kThreads + threadIdx.x;
+          if (e < top) {
+            const uint2 c = codes8(v[it], a.bf16, inv);
+            if (e == 0) first = c;
+            else q[it * kThreads] = c;
+          }
         }
       }
     }
