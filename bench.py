@@ -372,7 +372,7 @@ def run_quantize(args, dev, stream, world, peaks, peak_src):
             "unit": "GB/s", "ms_per_call": round(ms, 5), "launches_per_call": 2, "bytes_per_call": algo,
             "roofline": {"bound": "hbm", "achieved": round(gbs, 1), "peak": peaks["hbm_gbs"], "unit": "GB/s",
                          "frac": round(gbs / peaks["hbm_gbs"], 4), "peak_source": f"{peak_src} hbm_gbs",
-                         "traffic": None},
+                         "traffic": kernel_traffic("quant_fused_kernel", "llama7b_layer_bf16_b1h32l8192d128")},
             "l2": "inputs rotate over 3 copies (201 MB > 126 MB L2)"}
 
 
