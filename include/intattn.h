@@ -107,6 +107,34 @@ int intattn_forward(const int8_t *q, const int8_t *k, const int8_t *v,
                     const intattn_scales_t *scales, int B, int H, int Lq, int Lk, int d,
                     int causal, float clip_c, int8_t *out, intattn_stream_t stream);
 
+/* Bytes of device workspace intattn_forward_host needs for these sizes
+ * (0 for invalid sizes). */
+size_t intattn_forward_host_workspace_size(int B, int H, int Lq, int Lk, int d);
+
+/* intattn_forward on HOST tensors: q, k, v and out are host pointers in the
+ * layout of intattn_forward; page-locked (pinned) memory lets the copies run
+ * asynchronously, pageable memory works but the copies then serialise with
+ * the host.  The inputs are copied in on a library copy stream, the forward
+ * runs on `stream`, the output is copied out on a second copy stream.  The
+ * workspace has two slots that consecutive calls with the same workspace
+ * from one host thread alternate between, so the copies in of one call
+ * overlap the forward and the copy out of the previous one: a sequence of
+ * calls costs about the host-to-device copy time per call.
+ *   workspace: device, 256-byte aligned, at least
+ *   intattn_forward_host_workspace_size(B, H, Lq, Lk, d) bytes (two slots of
+ *   q, k, v and out); contents need no initialisation.  Calls that share a
+ *   workspace must come from one host thread.
+ * The library keeps two copy streams per device (created on first use, kept
+ * for the process) and seven events per host thread and device.  The result
+ * is in `out` when `stream` reaches the end of the call; q, k, v and out must
+ * stay valid and unmodified until then.  Under stream capture the copy
+ * streams fork from and join `stream`, and calls do not overlap.  Return
+ * codes as intattn_forward, plus INTATTN_ERR_WORKSPACE. */
+int intattn_forward_host(const int8_t *q, const int8_t *k, const int8_t *v,
+                         const intattn_scales_t *scales, int B, int H, int Lq, int Lk, int d,
+                         int causal, float clip_c, int8_t *out, void *workspace,
+                         size_t workspace_bytes, intattn_stream_t stream);
+
 /* Bytes of device workspace intattn_decode needs for these sizes. */
 size_t intattn_decode_workspace_size(int B, int H, int Lk, int d);
 

@@ -22,7 +22,8 @@ MAX_HEADS = 128
 MAX_CLIPS = 8
 
 # every function declared in include/intattn.h
-EXPORTED = ("intattn_derive_params", "intattn_forward", "intattn_decode_workspace_size",
+EXPORTED = ("intattn_derive_params", "intattn_forward", "intattn_forward_host_workspace_size",
+            "intattn_forward_host", "intattn_decode_workspace_size",
             "intattn_decode", "intattn_decode_int4", "intattn_decode_static_scratch", "intattn_quantize",
             "intattn_gelu_derive_params", "intattn_gelu", "intattn_selftest_timeout", "intattn_device_error",
             "intattn_strerror")
@@ -98,6 +99,10 @@ def lib() -> ctypes.CDLL:
                                             ctypes.POINTER(ctypes.c_int32), ctypes.POINTER(_HeadParams)]
         L.intattn_forward.argtypes = [vp, vp, vp, ctypes.POINTER(_Scales), i32, i32, i32, i32, i32,
                                       i32, f32, vp, vp]
+        L.intattn_forward_host_workspace_size.argtypes = [i32, i32, i32, i32, i32]
+        L.intattn_forward_host_workspace_size.restype = ctypes.c_size_t
+        L.intattn_forward_host.argtypes = [vp, vp, vp, ctypes.POINTER(_Scales), i32, i32, i32, i32, i32,
+                                           i32, f32, vp, vp, ctypes.c_size_t, vp]
         L.intattn_decode_workspace_size.argtypes = [i32, i32, i32, i32]
         L.intattn_decode_workspace_size.restype = ctypes.c_size_t
         L.intattn_decode.argtypes = [vp, vp, vp, ctypes.POINTER(_Scales), i32, i32, i32, i32, i32,
@@ -173,6 +178,41 @@ def forward(q, k, v, scales: Scales, causal: bool, clip_c: float, out=None, stre
                                _stream_handle(stream, q.device))
     del keep
     _check(rc, "intattn_forward")
+    return out
+
+
+def forward_host_workspace_size(B: int, H: int, Lq: int, Lk: int, d: int) -> int:
+    return int(lib().intattn_forward_host_workspace_size(B, H, Lq, Lk, d))
+
+
+def forward_host(q, k, v, scales: Scales, causal: bool, clip_c: float, out=None, workspace=None, stream=None,
+                 device=None):
+    """forward on CPU int8 tensors (pinned for asynchronous copies): the
+    library copies them in, runs the forward and copies the result out;
+    consecutive calls with one workspace overlap.  Returns out (a CPU tensor,
+    valid once `stream` has reached the end of the call)."""
+    import torch
+    for t, name in ((q, "q"), (k, "k"), (v, "v")):
+        if not isinstance(t, torch.Tensor) or t.dtype != torch.int8 or t.is_cuda or not t.is_contiguous():
+            raise TypeError(f"{name} must be a contiguous CPU int8 tensor")
+    B, H, Lq, d = q.shape
+    Lk = k.shape[2]
+    if k.shape != (B, H, Lk, d) or v.shape != k.shape:
+        raise ValueError("k and v must be [B, H, Lk, d]")
+    dev = torch.device("cuda") if device is None else torch.device(device)
+    if out is None:
+        out = torch.empty(q.shape, dtype=torch.int8, pin_memory=True)
+    if out.is_cuda or out.dtype != torch.int8 or out.shape != q.shape or not out.is_contiguous():
+        raise ValueError("out must be a contiguous CPU int8 tensor shaped like q")
+    need = forward_host_workspace_size(B, H, Lq, Lk, d)
+    if workspace is None:
+        workspace = torch.empty(max(need, 1), dtype=torch.uint8, device=dev)
+    sc, keep = scales._c()
+    rc = lib().intattn_forward_host(q.data_ptr(), k.data_ptr(), v.data_ptr(), ctypes.byref(sc), B, H, Lq, Lk, d,
+                                    int(bool(causal)), float(clip_c), out.data_ptr(), workspace.data_ptr(),
+                                    workspace.numel(), _stream_handle(stream, dev))
+    del keep
+    _check(rc, "intattn_forward_host")
     return out
 
 

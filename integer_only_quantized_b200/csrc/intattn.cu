@@ -377,6 +377,146 @@ int intattn_forward(const int8_t* q, const int8_t* k, const int8_t* v, const int
   return d == 64 ? prefill_launch<64>(args, grid, st) : prefill_launch<128>(args, grid, st);
 }
 
+// ------------------------------------------------ forward from host buffers
+namespace {
+
+size_t align256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
+
+// One workspace slot: device copies of q, k, v and out.
+size_t host_slot_bytes(int B, int H, int Lq, int Lk, int d) {
+  const size_t bh = static_cast<size_t>(B) * H;
+  const size_t q = bh * Lq * d, kv = bh * Lk * d;
+  return 2 * align256(q) + 2 * align256(kv);
+}
+
+// Two copy streams per device (host to device, device to host), created on
+// first use and kept for the life of the process.
+int copy_streams(cudaStream_t* h2d, cudaStream_t* d2h) {
+  static std::mutex mu;
+  static cudaStream_t streams[64][2] = {};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return INTATTN_ERR_CUDA;
+  std::lock_guard<std::mutex> lock(mu);
+  if (!streams[dev][0]) {
+    cudaStream_t a = nullptr, b = nullptr;
+    if (cudaStreamCreateWithFlags(&a, cudaStreamNonBlocking) != cudaSuccess) return INTATTN_ERR_CUDA;
+    if (cudaStreamCreateWithFlags(&b, cudaStreamNonBlocking) != cudaSuccess) {
+      cudaStreamDestroy(a);
+      return INTATTN_ERR_CUDA;
+    }
+    streams[dev][0] = a;
+    streams[dev][1] = b;
+  }
+  *h2d = streams[dev][0];
+  *d2h = streams[dev][1];
+  return INTATTN_OK;
+}
+
+// Per host thread and device: the events that order the two slots of the
+// workspaces this thread uses (copied in, computed, copied out, per slot,
+// plus one fork event), and which slot each recent workspace takes next.
+struct HostPipe {
+  cudaEvent_t ev[7] = {};
+  const void* ws[16] = {};
+  int next[16] = {};
+  int clock = 0;
+};
+
+int host_pipe(HostPipe** out) {
+  thread_local HostPipe pipes[64];
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return INTATTN_ERR_CUDA;
+  HostPipe& p = pipes[dev];
+  if (!p.ev[0])
+    for (int i = 0; i < 7; ++i)
+      if (cudaEventCreateWithFlags(&p.ev[i], cudaEventDisableTiming) != cudaSuccess) return INTATTN_ERR_CUDA;
+  *out = &p;
+  return INTATTN_OK;
+}
+
+// Slot this call uses in `ws` (alternates per workspace; a workspace not
+// seen recently starts at slot 0).
+int take_slot(HostPipe* p, const void* ws) {
+  for (int i = 0; i < 16; ++i)
+    if (p->ws[i] == ws) {
+      const int s = p->next[i];
+      p->next[i] = s ^ 1;
+      return s;
+    }
+  const int i = p->clock++ & 15;
+  p->ws[i] = ws;
+  p->next[i] = 1;
+  return 0;
+}
+
+}  // namespace
+
+size_t intattn_forward_host_workspace_size(int B, int H, int Lq, int Lk, int d) {
+  if (B < 0 || H <= 0 || Lq < 0 || Lk < 1 || (d != 64 && d != 128)) return 0;
+  return 2 * host_slot_bytes(B, H, Lq, Lk, d);
+}
+
+int intattn_forward_host(const int8_t* q, const int8_t* k, const int8_t* v, const intattn_scales_t* scales, int B,
+                         int H, int Lq, int Lk, int d, int causal, float clip_c, int8_t* out, void* workspace,
+                         size_t workspace_bytes, intattn_stream_t stream) {
+  if (B < 0 || H <= 0 || Lq < 0 || Lk < 1 || Lk > 65535) return INTATTN_ERR_INVALID_ARG;
+  if (causal && Lq > Lk) return INTATTN_ERR_INVALID_ARG;
+  if (d != 64 && d != 128) return INTATTN_ERR_UNSUPPORTED;
+  if (!scales) return INTATTN_ERR_INVALID_ARG;
+  {
+    // every parameter check of the forward, before anything is queued
+    HeadParamsDev hp[INTATTN_MAX_HEADS];
+    uint32_t l[INTATTN_MAX_CLIPS][32];
+    const int rc = derive(scales, H, d, clip_c, l, hp, INTATTN_MAX_HEADS);
+    if (rc) return rc;
+  }
+  if (static_cast<long long>(B) * H == 0 || Lq == 0) return INTATTN_OK;
+  if (!q || !k || !v || !out) return INTATTN_ERR_INVALID_ARG;
+  const size_t slot_bytes = host_slot_bytes(B, H, Lq, Lk, d);
+  if (!workspace || workspace_bytes < 2 * slot_bytes) return INTATTN_ERR_WORKSPACE;
+  if (reinterpret_cast<uintptr_t>(workspace) & 255u) return INTATTN_ERR_WORKSPACE;
+
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream), h2d = nullptr, d2h = nullptr;
+  HostPipe* pipe = nullptr;
+  if (copy_streams(&h2d, &d2h) || host_pipe(&pipe)) return INTATTN_ERR_CUDA;
+  cudaEvent_t e_fork = pipe->ev[0];
+  const int sl = take_slot(pipe, workspace);
+  cudaEvent_t e_in = pipe->ev[1 + sl], e_done = pipe->ev[3 + sl], e_out = pipe->ev[5 + sl];
+  cudaStreamCaptureStatus cap = cudaStreamCaptureStatusNone;
+  if (note_launch(cudaStreamIsCapturing(st, &cap))) return INTATTN_ERR_CUDA;
+  if (cap != cudaStreamCaptureStatusNone) {
+    // under stream capture the copy streams join the capture through `stream`
+    if (note_launch(cudaEventRecord(e_fork, st)) || note_launch(cudaStreamWaitEvent(h2d, e_fork, 0)) ||
+        note_launch(cudaStreamWaitEvent(d2h, e_fork, 0)))
+      return INTATTN_ERR_CUDA;
+  }
+  const size_t bh = static_cast<size_t>(B) * H;
+  const size_t qn = bh * Lq * d, kvn = bh * Lk * d;
+  char* base = static_cast<char*>(workspace) + sl * slot_bytes;
+  int8_t* dq = reinterpret_cast<int8_t*>(base);
+  int8_t* dk = reinterpret_cast<int8_t*>(base + align256(qn));
+  int8_t* dv = reinterpret_cast<int8_t*>(base + align256(qn) + align256(kvn));
+  int8_t* dout = reinterpret_cast<int8_t*>(base + align256(qn) + 2 * align256(kvn));
+  // copies in once this slot's previous forward has read its inputs; the
+  // forward once they have landed and the slot's previous output has been
+  // copied out; the copy out once the forward is done.  The copies of the
+  // next call (other slot) overlap this call's forward and copy out.
+  if (note_launch(cudaStreamWaitEvent(h2d, e_done, 0)) ||
+      note_launch(cudaMemcpyAsync(dq, q, qn, cudaMemcpyHostToDevice, h2d)) ||
+      note_launch(cudaMemcpyAsync(dk, k, kvn, cudaMemcpyHostToDevice, h2d)) ||
+      note_launch(cudaMemcpyAsync(dv, v, kvn, cudaMemcpyHostToDevice, h2d)) ||
+      note_launch(cudaEventRecord(e_in, h2d)) || note_launch(cudaStreamWaitEvent(st, e_in, 0)) ||
+      note_launch(cudaStreamWaitEvent(st, e_out, 0)))
+    return INTATTN_ERR_CUDA;
+  const int rc = intattn_forward(dq, dk, dv, scales, B, H, Lq, Lk, d, causal, clip_c, dout, stream);
+  if (rc) return rc;
+  if (note_launch(cudaEventRecord(e_done, st)) || note_launch(cudaStreamWaitEvent(d2h, e_done, 0)) ||
+      note_launch(cudaMemcpyAsync(out, dout, qn, cudaMemcpyDeviceToHost, d2h)) ||
+      note_launch(cudaEventRecord(e_out, d2h)) || note_launch(cudaStreamWaitEvent(st, e_out, 0)))
+    return INTATTN_ERR_CUDA;
+  return INTATTN_OK;
+}
+
 size_t intattn_decode_workspace_size(int B, int H, int Lk, int d) {
   if (B < 0 || H <= 0 || Lk < 1 || (d != 64 && d != 128)) return 0;
   return decode_layout(static_cast<long long>(B) * H, Lk, d).total;

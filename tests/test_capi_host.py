@@ -153,3 +153,24 @@ def test_binding_fails_loudly_without_library(tmp_path, monkeypatch, ia):
     monkeypatch.setattr(mod, "LIB_PATH", str(tmp_path / "missing.so"))
     with pytest.raises(ImportError):
         mod.lib()
+
+
+def test_forward_host_checks_without_gpu():
+    """Argument checks of intattn_forward_host return before any CUDA call."""
+    import ctypes
+    import integer_only_quantized_b200 as ia
+    L = ia.lib()
+    one = np.ones(1, dtype=np.float32)
+    sc = ia.Scales(one, one, one, one)
+    c, keep = sc._c()
+    f = L.intattn_forward_host
+    need = L.intattn_forward_host_workspace_size(2, 3, 64, 64, 64)
+    assert need > 0 and need % 256 == 0
+    assert L.intattn_forward_host_workspace_size(2, 3, 64, 64, 96) == 0
+    args = lambda B, ws, nbytes: (16, 16, 16, ctypes.byref(c), B, 3, 64, 64, 64, 0, 8.0, 16, ws, nbytes, None)
+    assert f(*args(-1, 256, need)) == ia.ERR_INVALID_ARG
+    assert f(*args(0, 256, need)) == ia.OK                 # nothing to do
+    assert f(*args(2, 256, need - 1)) == ia.ERR_WORKSPACE
+    assert f(*args(2, 0, need)) == ia.ERR_WORKSPACE
+    assert f(*args(2, 256 + 16, need)) == ia.ERR_WORKSPACE  # not 256-byte aligned
+    del keep
