@@ -49,6 +49,9 @@ namespace decode {
 
 constexpr int kThreads = 256;
 constexpr int kChunk = 512;    // keys per CTA, int8 cache (multiple of the rows one step covers)
+// Partial-sum rows of the P.V reductions: one word of padding per row keeps
+// both the per-thread writes and the per-channel reads free of bank conflicts.
+constexpr int kPartStride = kThreads + 1;
 constexpr int kChunk4 = 4096;  // keys per CTA, int4 cache (measured best for the 4096-key rows)
 
 __device__ __forceinline__ uint4 ld_stream(const void* p) {
@@ -86,7 +89,10 @@ __device__ __forceinline__ int32_t dp4a_uu(uint32_t a, uint32_t b, int32_t c) {
 // 8 packed int4 channels (one word) -> biased bytes u = x + 8 of the even
 // channels (lo) and of the odd channels (hi)
 __device__ __forceinline__ uint32_t nib_lo(uint32_t w) { return (w & 0x0F0F0F0Fu) ^ 0x08080808u; }
-__device__ __forceinline__ uint32_t nib_hi(uint32_t w) { return ((w >> 4) & 0x0F0F0F0Fu) ^ 0x08080808u; }
+// The high nibbles in place, biased: byte t holds 16 * (x_hi + 8).  Products
+// with it are 16 times the biased ones (one op fewer than shifting down);
+// their sums are divided by 16 exactly at the end.
+__device__ __forceinline__ uint32_t nib_hi16(uint32_t w) { return (w & 0xF0F0F0F0u) ^ 0x80808080u; }
 
 __device__ __forceinline__ int32_t imax32(int32_t a, int32_t b) { return a > b ? a : b; }
 
@@ -254,7 +260,7 @@ __global__ void __launch_bounds__(kThreads) decode_pv_kernel(const __grid_consta
 
   __shared__ uint32_t ptab_s[32];
   __shared__ uint32_t pk[kChunk / 4];              // u8 probabilities of this chunk
-  __shared__ int32_t part[kThreads * 16];          // per-thread partial sums
+  __shared__ int32_t part[16 * kPartStride];       // per-thread partial sums, [channel][thread]
   __shared__ int last_flag;
 
   const int32_t m = __ldcg(a.ws_mr + 2 * bh);
@@ -332,13 +338,13 @@ __global__ void __launch_bounds__(kThreads) decode_pv_kernel(const __grid_consta
   }
   // reduce over the row groups: column piece*16 + c
 #pragma unroll
-  for (int c = 0; c < 16; ++c) part[tid * 16 + c] = acc[c];
+  for (int c = 0; c < 16; ++c) part[c * kPartStride + tid] = acc[c];
   __syncthreads();
   int32_t* gpart = a.ws_part + (static_cast<size_t>(bh) * a.nsplit + sp) * D;
   if (tid < D) {
     const int pc = tid / 16, c = tid % 16;
     int32_t sum = 0;
-    for (int g = 0; g < Lt::kGroups; ++g) sum += part[(g * Lt::kCPR + pc) * 16 + c];
+    for (int g = 0; g < Lt::kGroups; ++g) sum += part[c * kPartStride + g * Lt::kCPR + pc];
     gpart[tid] = sum;
   }
   // the last CTA of this (b, h) adds the partials and requantises
@@ -418,13 +424,13 @@ __global__ void __launch_bounds__(kThreads) decode4_qk_kernel(const __grid_const
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
       const uint32_t w[4] = {kv[i].x, kv[i].y, kv[i].z, kv[i].w};
-      int32_t acc = -qbias;
+      int32_t acc = -qbias, acc16 = 0;  // even channels; odd channels x 16
 #pragma unroll
       for (int g = 0; g < 4; ++g) {
         acc = dp4a_su(qw[2 * g], nib_lo(w[g]), acc);
-        acc = dp4a_su(qw[2 * g + 1], nib_hi(w[g]), acc);
+        acc16 = dp4a_su(qw[2 * g + 1], nib_hi16(w[g]), acc16);
       }
-      s[i] = acc;
+      s[i] = acc + (acc16 >> 4);  // acc16 is a multiple of 16
     }
     // reduce the CPR partial sums of each of the 4 rows (transpose-reduce)
     if constexpr (Lt::kCPR == 4) {
@@ -496,7 +502,7 @@ __global__ void __launch_bounds__(kThreads, 3) decode4_pv_kernel(const __grid_co
 
   __shared__ uint32_t ptab_s[32];
   __shared__ uint32_t pk[kChunk4 / 4];             // u8 probabilities of this chunk
-  __shared__ int32_t part[kThreads * 16];          // per-thread partial sums
+  __shared__ int32_t part[16 * kPartStride];       // per-thread partial sums, [channel][thread]
   __shared__ int last_flag;
 
   const int32_t m = __ldcg(a.ws_mr + 2 * bh);
@@ -561,10 +567,11 @@ __global__ void __launch_bounds__(kThreads, 3) decode4_pv_kernel(const __grid_co
         const uint32_t y3 = g ? cur[4 * hq + 3].y : cur[4 * hq + 3].x;
 #pragma unroll
         for (int e = 0; e < 2; ++e) {
-          const uint32_t x0 = e ? nib_hi(y0) : nib_lo(y0);
-          const uint32_t x1 = e ? nib_hi(y1) : nib_lo(y1);
-          const uint32_t x2 = e ? nib_hi(y2) : nib_lo(y2);
-          const uint32_t x3 = e ? nib_hi(y3) : nib_lo(y3);
+          // e = 1: the odd channels, 16 x biased (accumulators divided by 16 at the end)
+          const uint32_t x0 = e ? nib_hi16(y0) : nib_lo(y0);
+          const uint32_t x1 = e ? nib_hi16(y1) : nib_lo(y1);
+          const uint32_t x2 = e ? nib_hi16(y2) : nib_lo(y2);
+          const uint32_t x3 = e ? nib_hi16(y3) : nib_lo(y3);
           // bytes (row i, column c) -> word c holds the 4 rows of column c
           const uint32_t ab_lo = __byte_perm(x0, x1, 0x5140);
           const uint32_t ab_hi = __byte_perm(x0, x1, 0x7362);
@@ -587,14 +594,14 @@ __global__ void __launch_bounds__(kThreads, 3) decode4_pv_kernel(const __grid_co
 #pragma unroll
   for (int s = 0; s < 16; ++s) {
     const int g = s >> 3, e = (s >> 2) & 1, c = s & 3;
-    part[tid * 16 + 8 * g + 2 * c + e] = acc[s] - 8 * psum;
+    part[(8 * g + 2 * c + e) * kPartStride + tid] = (e ? (acc[s] >> 4) : acc[s]) - 8 * psum;  // acc >= 0
   }
   __syncthreads();
   int32_t* gpart = a.ws_part + (static_cast<size_t>(bh) * a.nsplit + sp) * D;
   if (tid < D) {
     const int pc = tid / 16, c = tid % 16;
     int32_t sum = 0;
-    for (int g = 0; g < Lt::kGroups; ++g) sum += part[(g * Lt::kCPR + pc) * 16 + c];
+    for (int g = 0; g < Lt::kGroups; ++g) sum += part[c * kPartStride + g * Lt::kCPR + pc];
     gpart[tid] = sum;
   }
   // the last CTA of this (b, h) adds the partials and requantises
