@@ -517,19 +517,23 @@ __global__ void __launch_bounds__(kThreads, 3) decode4_pv_kernel(const __grid_co
   const int32_t* srow = a.ws_s + static_cast<size_t>(bh) * a.ld_s;
   __syncthreads();
 
-  // V rows streamed with 8-byte loads, one step ahead of the math
+  // V rows streamed with 8-byte loads, one step ahead of the math (two
+  // register buffers in turn)
   const int piece = tid % Lt::kCPR;
   const int grp = tid / Lt::kCPR;
   const int8_t* vbase = a.v + static_cast<size_t>(bh) * a.Lmax * kRowBytes + piece * 8;
   auto load8 = [&](int r0, uint2 (&vv)[8]) {
+    const int8_t* p = vbase + static_cast<size_t>(r0) * kRowBytes;
+    if (r0 + 8 <= j1) {
 #pragma unroll
-    for (int i = 0; i < 8; ++i) {
-      const int j = r0 + i;
-      vv[i] = (j < j1) ? ld_stream8(vbase + static_cast<size_t>(j) * kRowBytes) : make_uint2(0, 0);
+      for (int i = 0; i < 8; ++i) vv[i] = ld_stream8(p + i * kRowBytes);
+    } else {
+#pragma unroll
+      for (int i = 0; i < 8; ++i) vv[i] = (r0 + i < j1) ? ld_stream8(p + i * kRowBytes) : make_uint2(0, 0);
     }
   };
-  uint2 cur[8];
-  load8(j0 + 8 * grp, cur);
+  uint2 buf0[8], buf1[8];
+  load8(j0 + 8 * grp, buf0);  // in flight while the probabilities are built
 
   for (int w = tid; w < a.chunk / 4; w += kThreads) {
     uint32_t word = 0;
@@ -550,11 +554,7 @@ __global__ void __launch_bounds__(kThreads, 3) decode4_pv_kernel(const __grid_co
 #pragma unroll
   for (int c = 0; c < 16; ++c) acc[c] = 0;
   int32_t psum = 0;  // sum of this thread's P: the bias correction
-  for (int base = j0; base < j1; base += Lt::kRowsPerStep) {
-    const int r0 = base + 8 * grp;
-    const bool more = base + Lt::kRowsPerStep < j1;
-    uint2 nxt[8];
-    if (more) load8(r0 + Lt::kRowsPerStep, nxt);
+  auto octet = [&](int r0, const uint2 (&cur)[8]) {
 #pragma unroll
     for (int hq = 0; hq < 2; ++hq) {  // the two row quads of the octet
       const uint32_t p4 = pk[((r0 - j0) >> 2) + hq];  // P of 4 rows, one byte each (0 past j1)
@@ -585,10 +585,14 @@ __global__ void __launch_bounds__(kThreads, 3) decode4_pv_kernel(const __grid_co
         }
       }
     }
-    if (more) {
-#pragma unroll
-      for (int i = 0; i < 8; ++i) cur[i] = nxt[i];
-    }
+  };
+  for (int base = j0; base < j1; base += 2 * Lt::kRowsPerStep) {
+    const int r0 = base + 8 * grp;
+    if (base + Lt::kRowsPerStep < j1) load8(r0 + Lt::kRowsPerStep, buf1);
+    octet(r0, buf0);
+    if (base + Lt::kRowsPerStep >= j1) break;
+    if (base + 2 * Lt::kRowsPerStep < j1) load8(r0 + 2 * Lt::kRowsPerStep, buf0);
+    octet(r0 + Lt::kRowsPerStep, buf1);
   }
   // per-thread sums by channel, bias removed; then reduce over the row groups
 #pragma unroll
