@@ -415,10 +415,13 @@ __global__ void __launch_bounds__(kThreads) decode4_qk_kernel(const __grid_const
   for (int base = j0; base < j1; base += Lt::kRowsPerStep) {
     const int r0 = base + 4 * grp;
     uint4 kv[4];
+    const int8_t* kp = kbase + static_cast<size_t>(r0) * kRowBytes;
+    if (r0 + 4 <= j1) {
 #pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      const int j = r0 + i;
-      kv[i] = (j < j1) ? ld_stream(kbase + static_cast<size_t>(j) * kRowBytes) : make_uint4(0, 0, 0, 0);
+      for (int i = 0; i < 4; ++i) kv[i] = ld_stream(kp + i * kRowBytes);
+    } else {
+#pragma unroll
+      for (int i = 0; i < 4; ++i) kv[i] = (r0 + i < j1) ? ld_stream(kp + i * kRowBytes) : make_uint4(0, 0, 0, 0);
     }
     int32_t s[4];
 #pragma unroll
