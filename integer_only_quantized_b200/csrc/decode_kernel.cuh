@@ -412,9 +412,9 @@ __global__ void __launch_bounds__(kThreads) decode4_qk_kernel(const __grid_const
   int32_t* srow = a.ws_s + static_cast<size_t>(bh) * a.ld_s;
   int32_t mx = INT_MIN;
 
-  for (int base = j0; base < j1; base += Lt::kRowsPerStep) {
-    const int r0 = base + 4 * grp;
-    uint4 kv[4];
+  // K rows with 16-byte loads, one step ahead of the math (two register
+  // buffers in turn)
+  auto load4 = [&](int r0, uint4 (&kv)[4]) {
     const int8_t* kp = kbase + static_cast<size_t>(r0) * kRowBytes;
     if (r0 + 4 <= j1) {
 #pragma unroll
@@ -423,6 +423,8 @@ __global__ void __launch_bounds__(kThreads) decode4_qk_kernel(const __grid_const
 #pragma unroll
       for (int i = 0; i < 4; ++i) kv[i] = (r0 + i < j1) ? ld_stream(kp + i * kRowBytes) : make_uint4(0, 0, 0, 0);
     }
+  };
+  auto quad = [&](int r0, const uint4 (&kv)[4]) {
     int32_t s[4];
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
@@ -466,6 +468,16 @@ __global__ void __launch_bounds__(kThreads) decode4_qk_kernel(const __grid_const
         mx = imax32(mx, u1);
       }
     }
+  };
+  uint4 buf0[4], buf1[4];
+  load4(j0 + 4 * grp, buf0);
+  for (int base = j0; base < j1; base += 2 * Lt::kRowsPerStep) {
+    const int r0 = base + 4 * grp;
+    if (base + Lt::kRowsPerStep < j1) load4(r0 + Lt::kRowsPerStep, buf1);
+    quad(r0, buf0);
+    if (base + Lt::kRowsPerStep >= j1) break;
+    if (base + 2 * Lt::kRowsPerStep < j1) load4(r0 + 2 * Lt::kRowsPerStep, buf0);
+    quad(r0 + Lt::kRowsPerStep, buf1);
   }
   // chunk max
 #pragma unroll
