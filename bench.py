@@ -447,13 +447,15 @@ def run_decode(args, dev, stream, world, peaks, peak_src, name):
         raise RuntimeError("a kernel wait timed out in decode")
     gbs = w.decode_bytes / (ms * 1e-3) / 1e9
     return {"workload": w.name, "value": round(aggregate_value(w.decode_bytes, world, ms * 1e-3) / 1e9, 1),
-            "unit": "GB/s", "ms_per_call": round(ms, 5), "launches_per_call": 3,
+            "unit": "GB/s", "ms_per_call": round(ms, 5),
+            # int4 rows of at most 4096 keys: Q.K^T and P.V (which also finds Z)
+            "launches_per_call": 2 if (w.kv_bits == 4 and w.Lk <= 4096) else 3,
             "bytes_per_call": int(w.decode_bytes),
             "roofline": {"bound": "hbm", "achieved": round(gbs, 1), "peak": peaks["hbm_gbs"],
                          "unit": "GB/s", "frac": round(gbs / peaks["hbm_gbs"], 4),
                          "peak_source": f"{peak_src} hbm_gbs",
                          "traffic": kernel_traffic("decode", w.name, "bytes_per_call"),
-                         "traffic_unit": "DRAM bytes per call (decode_qk + decode_z + decode_pv)"},
+                         "traffic_unit": "DRAM bytes per call (all launches of one call)"},
             "kv_bits": w.kv_bits,
             "l2": f"K/V caches {2 * w.B * w.H * w.Lmax * w.d * w.kv_bits / 8 / 2**30:.0f} GiB > 126 MiB L2"}
 

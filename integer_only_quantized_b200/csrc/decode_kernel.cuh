@@ -503,7 +503,10 @@ struct LayoutPv4 {
   static_assert(kChunk4 % kRowsPerStep == 0, "chunk must be whole steps");
 };
 
-template <int D>
+// kOwnZ: the chunk is the whole row (nsplit == 1), so this CTA also takes
+// the role of decode_z: m from the chunk maximum, Z and R from the scores it
+// reads anyway to build P.  Same arithmetic as decode_z, bit for bit.
+template <int D, bool kOwnZ>
 __global__ void __launch_bounds__(kThreads, 3) decode4_pv_kernel(const __grid_constant__ DecodeArgs a) {
   using Lt = LayoutPv4<D>;
   constexpr int kRowBytes = D / 2;
@@ -519,11 +522,18 @@ __global__ void __launch_bounds__(kThreads, 3) decode4_pv_kernel(const __grid_co
   __shared__ uint32_t pk[kChunk4 / 4];             // u8 probabilities of this chunk
   __shared__ int32_t part[16 * kPartStride];       // per-thread partial sums, [channel][thread]
   __shared__ int last_flag;
+  __shared__ int32_t zred[kThreads / 32];
 
-  const int32_t m = __ldcg(a.ws_mr + 2 * bh);
-  const unsigned long long R = static_cast<uint32_t>(__ldcg(a.ws_mr + 2 * bh + 1));
-  if (tid < 32)
-    ptab_s[tid] = static_cast<uint32_t>((static_cast<unsigned long long>(a.lut[hp.lut][tid]) * R + (1ull << 31)) >> 32);
+  int32_t m;
+  if constexpr (kOwnZ) {
+    m = __ldcg(a.ws_max + bh);  // the only chunk's maximum
+    if (tid < 32) ptab_s[tid] = a.lut[hp.lut][tid];  // the exp table until R is known
+  } else {
+    m = __ldcg(a.ws_mr + 2 * bh);
+    const unsigned long long R = static_cast<uint32_t>(__ldcg(a.ws_mr + 2 * bh + 1));
+    if (tid < 32)
+      ptab_s[tid] = static_cast<uint32_t>((static_cast<unsigned long long>(a.lut[hp.lut][tid]) * R + (1ull << 31)) >> 32);
+  }
   const long long lo64 = static_cast<long long>(m) - hp.D;
   const int32_t lo = lo64 < INT_MIN ? INT_MIN : static_cast<int32_t>(lo64);
   const uint32_t Mu = static_cast<uint32_t>(hp.M);
@@ -550,17 +560,60 @@ __global__ void __launch_bounds__(kThreads, 3) decode4_pv_kernel(const __grid_co
   uint2 buf0[8], buf1[8];
   load8(j0 + 8 * grp, buf0);  // in flight while the probabilities are built
 
-  for (int w = tid; w < a.chunk / 4; w += kThreads) {
-    uint32_t word = 0;
+  if constexpr (kOwnZ) {
+    // indices first (bytes of pk) and Z = sum of their table entries; then R,
+    // the probability table, and the indices turned into probabilities
+    int32_t z = 0;
+    for (int w = tid; w < a.chunk / 4; w += kThreads) {
+      uint32_t word = 0;
 #pragma unroll
-    for (int b = 0; b < 4; ++b) {
-      const int j = j0 + 4 * w + b;
-      if (j < j1) {
-        const int32_t t = imax32(__ldcg(srow + j), lo);
-        word |= ptab_s[(Cm - static_cast<uint32_t>(t) * Mu) >> sh] << (8 * b);
+      for (int b = 0; b < 4; ++b) {
+        const int j = j0 + 4 * w + b;
+        if (j < j1) {
+          const uint32_t idx = (Cm - static_cast<uint32_t>(imax32(__ldcg(srow + j), lo)) * Mu) >> sh;
+          z += static_cast<int32_t>(ptab_s[idx]);
+          word |= idx << (8 * b);
+        } else {
+          word |= 32u << (8 * b);  // past the row: probability 0 (entry 32 below)
+        }
       }
+      pk[w] = word;
     }
-    pk[w] = word;
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) z += __shfl_xor_sync(0xffffffffu, z, o);
+    if ((tid & 31) == 0) zred[tid >> 5] = z;
+    __syncthreads();
+    if (tid < 32) {  // each lane turns its own table entry into a probability
+      int32_t Z = 0;
+      for (int i = 0; i < kThreads / 32; ++i) Z += zred[i];
+      const unsigned long long R =
+          ((255ull << 32) + static_cast<unsigned long long>(Z >> 1)) / static_cast<unsigned long long>(Z);
+      ptab_s[tid] = static_cast<uint32_t>((static_cast<unsigned long long>(ptab_s[tid]) * R + (1ull << 31)) >> 32);
+    }
+    __syncthreads();
+    for (int w = tid; w < a.chunk / 4; w += kThreads) {
+      const uint32_t x = pk[w];
+      uint32_t word = 0;
+#pragma unroll
+      for (int b = 0; b < 4; ++b) {
+        const uint32_t idx = (x >> (8 * b)) & 0xFFu;
+        word |= (idx < 32u ? ptab_s[idx] : 0u) << (8 * b);
+      }
+      pk[w] = word;
+    }
+  } else {
+    for (int w = tid; w < a.chunk / 4; w += kThreads) {
+      uint32_t word = 0;
+#pragma unroll
+      for (int b = 0; b < 4; ++b) {
+        const int j = j0 + 4 * w + b;
+        if (j < j1) {
+          const int32_t t = imax32(__ldcg(srow + j), lo);
+          word |= ptab_s[(Cm - static_cast<uint32_t>(t) * Mu) >> sh] << (8 * b);
+        }
+      }
+      pk[w] = word;
+    }
   }
   __syncthreads();
 

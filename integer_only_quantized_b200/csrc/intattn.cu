@@ -215,11 +215,16 @@ int decode_launch(const DecodeArgs& a, cudaStream_t stream) {
   }
   const int rc = note_launch(cudaGetLastError());
   if (rc != INTATTN_OK) return rc;
+  if (kInt4 && a.nsplit == 1) {
+    // one chunk per row: the P.V kernel computes m, Z and R itself
+    intattn::decode::decode4_pv_kernel<D, true><<<grid, intattn::decode::kThreads, 0, stream>>>(a);
+    return note_launch(cudaGetLastError());
+  }
   intattn::decode::decode_z_kernel<D><<<a.BH, intattn::decode::kThreads, 0, stream>>>(a);
   const int rz = note_launch(cudaGetLastError());
   if (rz != INTATTN_OK) return rz;
   if constexpr (kInt4) {
-    intattn::decode::decode4_pv_kernel<D><<<grid, intattn::decode::kThreads, 0, stream>>>(a);
+    intattn::decode::decode4_pv_kernel<D, false><<<grid, intattn::decode::kThreads, 0, stream>>>(a);
   } else {
     intattn::decode::decode_pv_kernel<D><<<grid, intattn::decode::kThreads, 0, stream>>>(a);
   }

@@ -35,7 +35,8 @@ def _assert_equal(got, want, what):
 
 SWEEP = [
     (1, 1, 1, 1, 64), (2, 3, 100, 160, 128), (1, 2, 511, 511, 64), (1, 2, 512, 512, 128),
-    (2, 2, 513, 600, 64), (3, 2, 1500, 2048, 128), (1, 4, 4096, 4100, 64), (2, 1, 9000, 9000, 128),
+    (2, 2, 513, 600, 64), (3, 2, 1500, 2048, 128), (1, 4, 4096, 4100, 64), (1, 2, 4097, 4097, 128),
+    (2, 1, 9000, 9000, 128),
 ]
 
 
