@@ -125,7 +125,9 @@ size_t intattn_forward_host_workspace_size(int B, int H, int Lq, int Lk, int d);
  *   q, k, v and out); contents need no initialisation.  Calls that share a
  *   workspace must come from one host thread.
  * The library keeps two copy streams per device (created on first use, kept
- * for the process) and seven events per host thread and device.  The result
+ * for the process) and, per host thread and device, six events for each of
+ * up to 64 workspaces (a 65th workspace waits on the host for the least
+ * recently used one's copies to finish and takes its events).  The result
  * is in `out` when `stream` reaches the end of the call; q, k, v and out must
  * stay valid and unmodified until then.  Under stream capture the copy
  * streams fork from and join `stream`, and calls do not overlap.  Return

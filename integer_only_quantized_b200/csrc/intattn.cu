@@ -13,6 +13,7 @@
 #include <cstdint>
 #include <cstring>
 #include <mutex>
+#include <unordered_map>
 
 #include "intattn.h"
 
@@ -417,41 +418,62 @@ int copy_streams(cudaStream_t* h2d, cudaStream_t* d2h) {
   return INTATTN_OK;
 }
 
-// Per host thread and device: the events that order the two slots of the
-// workspaces this thread uses (copied in, computed, copied out, per slot,
-// plus one fork event), and which slot each recent workspace takes next.
-struct HostPipe {
-  cudaEvent_t ev[7] = {};
-  const void* ws[16] = {};
-  int next[16] = {};
-  int clock = 0;
+// Per host thread and device, per workspace: which slot the next call takes
+// and the events that order each slot's reuse (copied in, computed, copied
+// out).  At most kMaxPipes workspaces are tracked; the least recently used
+// one is retired once its events have completed (a host wait that only a
+// thread cycling through more workspaces than that ever meets).
+struct SlotEvents {
+  cudaEvent_t in[2] = {}, done[2] = {}, out[2] = {};
+  int next = 0;
+  unsigned long long used = 0;
 };
 
-int host_pipe(HostPipe** out) {
-  thread_local HostPipe pipes[64];
-  int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return INTATTN_ERR_CUDA;
-  HostPipe& p = pipes[dev];
-  if (!p.ev[0])
-    for (int i = 0; i < 7; ++i)
-      if (cudaEventCreateWithFlags(&p.ev[i], cudaEventDisableTiming) != cudaSuccess) return INTATTN_ERR_CUDA;
-  *out = &p;
+struct HostPipes {
+  cudaEvent_t fork = nullptr;
+  std::unordered_map<const void*, SlotEvents> by_ws;
+  unsigned long long clock = 0;
+};
+
+constexpr size_t kMaxPipes = 64;
+
+int make_events(SlotEvents* e) {
+  cudaEvent_t* all[6] = {&e->in[0], &e->in[1], &e->done[0], &e->done[1], &e->out[0], &e->out[1]};
+  for (cudaEvent_t* ev : all)
+    if (cudaEventCreateWithFlags(ev, cudaEventDisableTiming) != cudaSuccess) return INTATTN_ERR_CUDA;
   return INTATTN_OK;
 }
 
-// Slot this call uses in `ws` (alternates per workspace; a workspace not
-// seen recently starts at slot 0).
-int take_slot(HostPipe* p, const void* ws) {
-  for (int i = 0; i < 16; ++i)
-    if (p->ws[i] == ws) {
-      const int s = p->next[i];
-      p->next[i] = s ^ 1;
-      return s;
+// The events of workspace `ws` for this thread and device (created on first use).
+int pipe_of(const void* ws, cudaEvent_t* fork, SlotEvents** out) {
+  thread_local HostPipes pipes[64];
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return INTATTN_ERR_CUDA;
+  HostPipes& p = pipes[dev];
+  if (!p.fork && cudaEventCreateWithFlags(&p.fork, cudaEventDisableTiming) != cudaSuccess) return INTATTN_ERR_CUDA;
+  auto it = p.by_ws.find(ws);
+  if (it == p.by_ws.end()) {
+    SlotEvents fresh;
+    if (p.by_ws.size() >= kMaxPipes) {
+      auto lru = p.by_ws.begin();
+      for (auto i = p.by_ws.begin(); i != p.by_ws.end(); ++i)
+        if (i->second.used < lru->second.used) lru = i;
+      for (int sl = 0; sl < 2; ++sl)
+        if (cudaEventSynchronize(lru->second.done[sl]) != cudaSuccess ||
+            cudaEventSynchronize(lru->second.out[sl]) != cudaSuccess)
+          return INTATTN_ERR_CUDA;
+      fresh = lru->second;  // its events, now complete, serve the new workspace
+      fresh.next = 0;
+      p.by_ws.erase(lru);
+    } else if (make_events(&fresh) != INTATTN_OK) {
+      return INTATTN_ERR_CUDA;
     }
-  const int i = p->clock++ & 15;
-  p->ws[i] = ws;
-  p->next[i] = 1;
-  return 0;
+    it = p.by_ws.emplace(ws, fresh).first;
+  }
+  it->second.used = ++p.clock;
+  *fork = p.fork;
+  *out = &it->second;
+  return INTATTN_OK;
 }
 
 }  // namespace
@@ -482,11 +504,12 @@ int intattn_forward_host(const int8_t* q, const int8_t* k, const int8_t* v, cons
   if (reinterpret_cast<uintptr_t>(workspace) & 255u) return INTATTN_ERR_WORKSPACE;
 
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream), h2d = nullptr, d2h = nullptr;
-  HostPipe* pipe = nullptr;
-  if (copy_streams(&h2d, &d2h) || host_pipe(&pipe)) return INTATTN_ERR_CUDA;
-  cudaEvent_t e_fork = pipe->ev[0];
-  const int sl = take_slot(pipe, workspace);
-  cudaEvent_t e_in = pipe->ev[1 + sl], e_done = pipe->ev[3 + sl], e_out = pipe->ev[5 + sl];
+  cudaEvent_t e_fork = nullptr;
+  SlotEvents* pipe = nullptr;
+  if (copy_streams(&h2d, &d2h) || pipe_of(workspace, &e_fork, &pipe)) return INTATTN_ERR_CUDA;
+  const int sl = pipe->next;
+  pipe->next = sl ^ 1;
+  cudaEvent_t e_in = pipe->in[sl], e_done = pipe->done[sl], e_out = pipe->out[sl];
   cudaStreamCaptureStatus cap = cudaStreamCaptureStatusNone;
   if (note_launch(cudaStreamIsCapturing(st, &cap))) return INTATTN_ERR_CUDA;
   if (cap != cudaStreamCaptureStatusNone) {

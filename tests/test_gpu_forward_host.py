@@ -99,6 +99,30 @@ def test_forward_host_overlapping_calls(ia, oracle_mod):
         assert np.array_equal(out.numpy(), want)
 
 
+def test_forward_host_two_workspaces_two_streams(ia, oracle_mod):
+    """Calls alternating between two workspaces, each on its own stream:
+    every workspace keeps its own slot order, so no call overwrites a slot
+    that the other stream's forward still reads."""
+    import torch
+    streams = [torch.cuda.Stream(), torch.cuda.Stream()]
+    wss = [torch.empty(ia.forward_host_workspace_size(2, 4, 192, 192, 64), dtype=torch.uint8, device="cuda")
+           for _ in range(2)]
+    runs = []
+    for i in range(8):
+        w = wl.custom_workload("host_two", 2, 4, 192, 192, 64, bool(i % 3 == 0), per_head=bool(i % 2),
+                               index=1400 + i)
+        x = wl.make_inputs(w)
+        runs.append((w, x, [_host(a, True) for a in (x.q, x.k, x.v)],
+                     torch.empty(x.q.shape, dtype=torch.int8).pin_memory()))
+    for i, (w, x, (q, k, v), out) in enumerate(runs):
+        ia.forward_host(q, k, v, ia.Scales(x.s_q, x.s_k, x.s_v, x.s_o, per_head=w.per_head), w.causal,
+                        w.clip_c, out=out, workspace=wss[i % 2], stream=streams[i % 2])
+    torch.cuda.synchronize()
+    for w, x, _, out in runs:
+        want = oracle_mod.forward(x.q, x.k, x.v, w.per_head, x.s_q, x.s_k, x.s_v, x.s_o, w.causal, w.clip_c)
+        assert np.array_equal(out.numpy(), want)
+
+
 def test_forward_host_matches_device_forward_on_bench_workload(ia):
     """BERT-base B8 H12 L512: host path == device path, byte for byte."""
     import torch
