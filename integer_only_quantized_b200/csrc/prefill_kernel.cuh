@@ -8,8 +8,9 @@
 // Work unit: one (batch, head, 128-query tile).  The kernel is persistent:
 // one CTA per SM takes a tile in each round, in snake order over the tiles
 // sorted longest first (causal), so the loads and MMAs of a tile overlap the
-// reductions and the epilogue of the previous one.  Warp roles:
-//   warps 0-15  IndexSoftmax + epilogue, in two teams of eight.  Team t
+// reductions of the previous one, and its epilogue the next tile's passes.
+// Warp roles:
+//   warps 0-15  IndexSoftmax, in two teams of eight.  Team t
 //               (warps 8t .. 8t+7) takes the S tiles whose running index is
 //               t mod 2, so one team computes while the other waits for its
 //               next tile.  Warp w reads TMEM lane quadrant w % 4 (query rows
@@ -23,6 +24,10 @@
 //   warp 17     TMEM allocator and MMA issuer (one thread): tcgen05.mma
 //               kind::i8 for S = Q.K^T (both operands in shared memory) and
 //               O += P.V (P from TMEM, V from shared memory, N-major).
+//   warps 20-23 epilogue: O of a finished tile (TMEM lane quadrant
+//               warp % 4, one query row per thread) -> requantised int8 rows,
+//               while the softmax warps already work on the next tile.
+//   warps 18-19 none (they complete the fifth warpgroup).
 //
 // The LUT index of a score depends on the final row max and P depends on
 // the final row sum Z, so a bit-exact result needs three sweeps over the
@@ -37,7 +42,7 @@
 // Every mbarrier wait is bounded (polls with a time limit).  Each softmax
 // warp polls its own barriers (one vote per poll).  A warp whose wait runs
 // out leaves its pass loop; every softmax warp still reaches the same
-// sequence of all-warp named barriers (one per pass and per epilogue), which
+// sequence of all-warp named barriers (one per pass), which
 // AND the warps' verdicts (bar.red.and), so all warps then leave together
 // and none is left waiting.
 #pragma once
@@ -76,10 +81,14 @@ constexpr int kGroups = kTeams * kColGroups;  // partial results per query row (
 constexpr int kSoftBase = 0;               // first softmax warp
 constexpr int kProducerWarp = kSoftWarps;
 constexpr int kMmaWarp = kSoftWarps + 1;
-constexpr int kThreads = 32 * (kSoftWarps + 2);  // 576
+// Epilogue warps 20-23 (TMEM lane quadrants 0-3); warps 18-19 only fill the
+// fifth warpgroup.
+constexpr int kEpiWarp0 = kSoftWarps + 4;
+constexpr int kEpiWarps = 4;
+constexpr int kThreads = 32 * (kEpiWarp0 + kEpiWarps);  // 768: six whole warpgroups
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kColS = 0;    // two S buffers: [0,128) and [128,256)
-constexpr uint32_t kColO = 256;  // O accumulator: d columns
+constexpr uint32_t kColO = 256;  // O accumulators: d columns each (two for d = 64)
 constexpr uint32_t kColP = 384;  // four P buffers of 32 columns (128 u8 keys each)
 constexpr int kPBufs = 4;
 // named barriers (id 0 is __syncthreads)
@@ -87,7 +96,7 @@ constexpr uint32_t kNbAll = 1;   // all softmax warps
 
 static_assert(kGroups == 4 && kCols % 32 == 0, "4 partials per row, whole 32-column TMEM loads");
 
-enum Role : unsigned { kRoleSoftmax = 1, kRoleProducer = 2, kRoleMma = 3 };
+enum Role : unsigned { kRoleSoftmax = 1, kRoleProducer = 2, kRoleMma = 3, kRoleEpilogue = 4 };
 
 // Shared-memory barriers, by index.
 enum Bar : int {
@@ -97,15 +106,19 @@ enum Bar : int {
   kBarSEmpty = 6,       // [2]  S tile loaded by all softmax warps
   kBarPFull = 8,        // [4]  P tile written to TMEM
   kBarPEmpty = 12,      // [4]  P.V MMA that read it is done
-  kBarOFull = 16,       //      all P.V MMAs of a tile done
-  kBarOEmpty = 17,      //      epilogue has read O
-  kBarDrain = 18,       //      final MMA drain
-  kBarKvFull = 19,      // [stages], then kv_empty[stages]
+  kBarOFull = 16,       // [2]  all P.V MMAs of a tile done (per O buffer)
+  kBarOEmpty = 18,      // [2]  epilogue has read that O buffer
+  kBarDrain = 20,       //      final MMA drain
+  kBarKvFull = 21,      // [stages], then kv_empty[stages]
 };
 
 template <int D>
 struct Cfg {
   static constexpr int kStages = (D == 64) ? 8 : 6;
+  // O accumulators in TMEM: with d = 64 two fit below the P buffers, so a
+  // tile accumulates into one while the epilogue drains the other
+  static constexpr int kOBufs = (D == 64) ? 2 : 1;
+  static_assert(kColO + kOBufs * D <= kColP, "O buffers overlap the P buffers");
   static constexpr uint32_t kTileBytes = kBN * D;  // one K or V tile
   static constexpr uint32_t kQBytes = kBM * D;
   static constexpr uint32_t kSwizzle = (D == 128) ? 2u : 4u;  // 128B / 64B swizzle
@@ -206,8 +219,10 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_kernel(const __grid_const
       mbar_init(bar(kBarPFull + i), kTeamWarps);
       mbar_init(bar(kBarPEmpty + i), 1);
     }
-    mbar_init(bar(kBarOFull), 1);
-    mbar_init(bar(kBarOEmpty), kSoftWarps);
+    for (int i = 0; i < C::kOBufs; ++i) {
+      mbar_init(bar(kBarOFull + i), 1);
+      mbar_init(bar(kBarOEmpty + i), kEpiWarps);
+    }
     mbar_init(bar(kBarDrain), 1);
     for (int i = 0; i < C::kStages; ++i) {
       mbar_init(bar_kv_full(i), 1);
@@ -443,34 +458,42 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_kernel(const __grid_const
       sc += T.nkt;
       pc += T.nkt;
 
-      // ---- epilogue: O (int32, TMEM) -> requantised int8 rows ----
-      {
-        const bool got = (ok && sw == 0) ? mbar_wait(bar(kBarOFull), it & 1, kRoleSoftmax) : ok;
-        if (!all_sync(got)) { ok = false; break; }
-      }
+    }
+  } else if (warp >= kEpiWarp0) {
+    // ============================ epilogue ============================
+    // O (int32, TMEM) of each tile -> requantised int8 rows, while the
+    // softmax warps go on with the next tile.  Thread = query row (TMEM lane).
+    const int quad = warp & 3;
+    const int r = quad * 32 + lane;
+    const uint32_t tlane = tmem + (static_cast<uint32_t>(quad * 32) << 16);
+    for (int it = 0;; ++it) {
+      const int L = tile_index(it, blockIdx.x, gridDim.x);
+      if (L >= args.n_tiles) break;
+      const Tile T = tile_of(args, L);
+      const HeadParamsDev hp = args.hp[args.per_head ? T.h : 0];
+      const int ob = it % C::kOBufs;
+      if (!mbar_wait_warp(bar(kBarOFull + ob), (it / C::kOBufs) & 1, kRoleEpilogue)) break;
       tc_fence_after();
-      constexpr int kOC = D / kGroups;  // output columns per thread: 16 or 32
-      uint32_t v[32];
-      if constexpr (kOC == 32) {
-        tmem_ld32(tlane + kColO + grp * kOC, v);
-      } else {
-        tmem_ld16(tlane + kColO + grp * kOC, v);
-      }
-      tmem_wait_ld();
-      tc_fence_before();
-      arrive_warp(bar(kBarOEmpty));  // O may now be overwritten by the next tile
-      uint32_t w[8];
-#pragma unroll
-      for (int q = 0; q < kOC / 4; ++q)
-        w[q] = pack4(requant_byte(static_cast<int32_t>(v[4 * q + 0]), hp.Mo, hp.so),
-                     requant_byte(static_cast<int32_t>(v[4 * q + 1]), hp.Mo, hp.so),
-                     requant_byte(static_cast<int32_t>(v[4 * q + 2]), hp.Mo, hp.so),
-                     requant_byte(static_cast<int32_t>(v[4 * q + 3]), hp.Mo, hp.so));
       const int row = T.q0 + r;
-      if (row < args.Lq) {
-        uint4* o = reinterpret_cast<uint4*>(args.out + (static_cast<size_t>(T.bh) * args.Lq + row) * D + grp * kOC);
-        o[0] = make_uint4(w[0], w[1], w[2], w[3]);
-        if constexpr (kOC == 32) o[1] = make_uint4(w[4], w[5], w[6], w[7]);
+      uint4* o = reinterpret_cast<uint4*>(args.out + (static_cast<size_t>(T.bh) * args.Lq + row) * D);
+#pragma unroll
+      for (int c = 0; c < D / 16; ++c) {
+        uint32_t v[16];
+        tmem_ld16(tlane + kColO + ob * D + 16 * c, v);
+        tmem_wait_ld();
+        if (c == D / 16 - 1) {  // O may now be overwritten by the next tile
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(bar(kBarOEmpty + ob));
+        }
+        uint32_t w[4];
+#pragma unroll
+        for (int q = 0; q < 4; ++q)
+          w[q] = pack4(requant_byte(static_cast<int32_t>(v[4 * q + 0]), hp.Mo, hp.so),
+                       requant_byte(static_cast<int32_t>(v[4 * q + 1]), hp.Mo, hp.so),
+                       requant_byte(static_cast<int32_t>(v[4 * q + 2]), hp.Mo, hp.so),
+                       requant_byte(static_cast<int32_t>(v[4 * q + 3]), hp.Mo, hp.so));
+        if (row < args.Lq) o[c] = make_uint4(w[0], w[1], w[2], w[3]);
       }
     }
   } else if (warp == kProducerWarp) {
@@ -595,7 +618,11 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_kernel(const __grid_const
         if (j + 2 < T.nkt) issue_qk();
         if (!ok) break;
         // O of the previous tile must have been read before it is overwritten
-        if (j == 0 && !mbar_wait_warp(bar(kBarOEmpty), (it & 1) ^ 1, kRoleMma)) { ok = false; break; }
+        // (with two O buffers: the tile before the previous one)
+        if (j == 0 && !mbar_wait_warp(bar(kBarOEmpty + it % C::kOBufs), ((it / C::kOBufs) & 1) ^ 1, kRoleMma)) {
+          ok = false;
+          break;
+        }
         const uint32_t pb = pc & (kPBufs - 1);
         if (!mbar_wait2_warp(bar(kBarPFull + pb), (pc / kPBufs) & 1, bar_kv_full(slot), kv_par, kRoleMma)) {
           ok = false;
@@ -606,7 +633,8 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_kernel(const __grid_const
         if (elect_one()) {
 #pragma unroll
           for (int kk = 0; kk < kBN / 32; ++kk)  // 32 keys per MMA: 8 TMEM columns of P, 32 V rows
-            mma_i8_ts(tmem + kColO, tmem + kColP + pb * 32 + kk * 8, v_desc + ((32u * D * kk) >> 4), idesc_pv,
+            mma_i8_ts(tmem + kColO + (it % C::kOBufs) * D, tmem + kColP + pb * 32 + kk * 8,
+                      v_desc + ((32u * D * kk) >> 4), idesc_pv,
                       (j > 0 || kk > 0) ? 1u : 0u);
           mma_commit(bar_kv_empty(slot));
           mma_commit(bar(kBarPEmpty + pb));
@@ -616,7 +644,7 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_kernel(const __grid_const
       }
       if (!ok) break;
       mma_commit_elect(bar(kBarQEmpty + qb));  // every MMA that read this Q buffer
-      mma_commit_elect(bar(kBarOFull));
+      mma_commit_elect(bar(kBarOFull + it % C::kOBufs));
     }
     // every MMA this warp issued is complete before TMEM is released
     mma_commit_elect(bar(kBarDrain));
