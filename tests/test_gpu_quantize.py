@@ -36,8 +36,9 @@ def _inputs(shape, seed, dtype, spread=(0.01, 30.0), outlier=40.0):
 
 CASES = [((1, 1, 1, 8), False), ((2, 3, 37, 64), True), ((2, 3, 37, 64), False), ((1, 4, 512, 128), True),
          ((3, 2, 1000, 64), True), ((8, 12, 512, 64), False),
-         # one CTA over 256 one-vector heads; a full grid over 32 heads of 256K elements
-         ((4, 64, 1, 8), True), ((1, 32, 2048, 128), True)]
+         # one CTA over 256 one-vector heads; a full grid over 32 heads of 256K elements;
+         # two heads of 2M elements
+         ((4, 64, 1, 8), True), ((1, 32, 2048, 128), True), ((1, 2, 16384, 128), True)]
 
 
 @pytest.mark.parametrize("dtype_name", ["bfloat16", "float16"])
