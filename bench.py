@@ -3,7 +3,10 @@
 
 One step = one IntAttention forward (int8 Q.K^T -> IndexSoftmax -> u8 x s8
 P.V -> int8) over one batch of the workload, through the C ABI.  Default
-workload: BERT-base batch, B=8 H=12 L=512 d=64, non-causal.
+workload: the largest one, a LLaMA-7B-shaped causal prefill, B=1 H=32
+L=8192 d=128.  The other prefill workloads (BERT-base L128 and B8 L512,
+ViT-B/16 L197, GPT-2-small causal L2048) are timed the same way and reported
+in the "prefill_configs" object of the same line.
 
   python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME]
   python bench.py --impl reference ...   # the CPU oracle, timed on host cores
@@ -40,7 +43,8 @@ def parse_args(argv=None):
     p.add_argument("--steps", type=int, default=200)
     p.add_argument("--warmup", type=int, default=10)
     p.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    p.add_argument("--workload", default="bert_base_b8_l512")
+    p.add_argument("--workload", default="llama7b_causal_l8192")
+    p.add_argument("--no-configs", action="store_true", help="skip the other prefill workloads")
     p.add_argument("--decode-workload", default="llama7b_decode_b64_lk4096")
     p.add_argument("--no-decode", action="store_true")
     p.add_argument("--no-cpu-baseline", action="store_true")
@@ -186,6 +190,74 @@ class ClockSampler:
 
 
 # ------------------------------------------------------------- our arm
+PREFILL_WORKLOADS = ["bert_base_l128", "bert_base_b8_l512", "vit_b16_l197", "gpt2_small_causal_l2048",
+                     "llama7b_causal_l8192"]
+
+
+def rotation(w):
+    """Number of input copies the timed steps rotate over (q, k, v, out of
+    one step: their total exceeds the 126 MB L2 at least twice) and the bytes
+    of one copy."""
+    set_bytes = 2 * w.B * w.H * w.Lq * w.d + 2 * w.B * w.H * w.Lk * w.d
+    return max(2, min(1024, math.ceil(2 * L2_BYTES / set_bytes))), set_bytes
+
+
+def workload_config(w, world: int) -> dict:
+    """The `config` object of the JSON line (the same for both arms)."""
+    nsets, set_bytes = rotation(w)
+    return {"workload": w.name, "B": w.B, "H": w.H, "Lq": w.Lq, "Lk": w.Lk, "d": w.d,
+            "causal": w.causal, "clip_c": w.clip_c,
+            "quant": "per_head" if w.per_head else "per_tensor",
+            "l2": f"inputs rotate over {nsets} copies ({nsets * set_bytes / 2**20:.0f} MiB > 126 MiB L2)",
+            "timing": "K steps captured as one CUDA graph, replayed once between CUDA events",
+            "parallelism": f"dp{world} (independent problems)"}
+
+
+def time_prefill(ia, w, x, dev, stream, steps: int, warmup: int, clocks=None, world: int = 1):
+    """ms per forward of workload w: `steps` calls over rotating copies of the
+    inputs, captured as one CUDA graph and replayed between CUDA events on
+    `stream`; max over ranks."""
+    import torch
+    sc = ia.Scales(x.s_q, x.s_k, x.s_v, x.s_o, per_head=w.per_head)
+    nsets, _ = rotation(w)
+    q0, k0, v0 = (torch.from_numpy(a).to(dev) for a in (x.q, x.k, x.v))
+    sets = [(q0.clone(), k0.clone(), v0.clone(), torch.empty_like(q0)) for _ in range(nsets)]
+    del q0, k0, v0
+
+    def step(i):
+        q, k, v, o = sets[i % nsets]
+        ia.forward(q, k, v, sc, w.causal, w.clip_c, out=o, stream=stream)
+
+    for i in range(warmup):
+        step(i)
+    torch.cuda.synchronize(dev)
+    if ia.device_error(stream) != ia.OK:
+        raise RuntimeError("a kernel wait timed out during warm-up")
+    # the timed steps are captured once as a CUDA graph and replayed: the
+    # device time then excludes the host's per-call launch latency
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph, stream=stream):
+        for i in range(steps):
+            step(i)
+    torch.cuda.synchronize(dev)
+    barrier(world, dev)
+    torch.cuda.synchronize(dev)
+    if clocks is not None:
+        clocks.start()
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    t0.record(stream)
+    graph.replay()
+    t1.record(stream)
+    torch.cuda.synchronize(dev)
+    barrier(world, dev)
+    clk = clocks.stop() if clocks is not None else None
+    ms = max_over_ranks(t0.elapsed_time(t1) / steps, world, dev)
+    if ia.device_error(stream) != ia.OK:
+        raise RuntimeError("a kernel wait timed out during the timed steps")
+    del graph, sets
+    return ms, clk
+
+
 def _int8_peak(peaks, sustained: bool):
     key = "bf16_tflops_sustained" if sustained and "bf16_tflops_sustained" in peaks else "bf16_tflops"
     return peaks[key] * INT8_OVER_BF16, key
@@ -230,44 +302,9 @@ def run_ours(args):
     assert not w.decode, "the headline workload is a prefill workload"
     x = wl.make_inputs(w)
     sc = ia.Scales(x.s_q, x.s_k, x.s_v, x.s_o, per_head=w.per_head)
-    set_bytes = x.q.nbytes + x.k.nbytes + x.v.nbytes + x.q.nbytes
-    nsets = max(2, min(64, math.ceil(2 * L2_BYTES / set_bytes)))
-    q0, k0, v0 = (torch.from_numpy(a).to(dev) for a in (x.q, x.k, x.v))
-    sets = [(q0.clone(), k0.clone(), v0.clone(), torch.empty_like(q0)) for _ in range(nsets)]
-    stream = torch.cuda.current_stream(dev)
-
-    def step(i):
-        q, k, v, o = sets[i % nsets]
-        ia.forward(q, k, v, sc, w.causal, w.clip_c, out=o, stream=torch.cuda.current_stream(dev))
-
-    for i in range(args.warmup):
-        step(i)
-    torch.cuda.synchronize(dev)
-    if ia.device_error(stream) != ia.OK:
-        raise RuntimeError("a kernel wait timed out during warm-up")
-    # the K timed steps are captured once as a CUDA graph and replayed: the
-    # device time then excludes the host's per-call launch latency
-    graph = torch.cuda.CUDAGraph()
-    with torch.cuda.graph(graph):
-        for i in range(args.steps):
-            step(i)
-    torch.cuda.synchronize(dev)
+    stream = torch.cuda.Stream(dev)
     clocks = ClockSampler(local_rank)
-    barrier(world, dev)
-    torch.cuda.synchronize(dev)
-    clocks.start()
-    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    t0.record(stream)
-    graph.replay()
-    t1.record(stream)
-    torch.cuda.synchronize(dev)
-    barrier(world, dev)
-    clk = clocks.stop()
-    ms = t0.elapsed_time(t1) / args.steps
-    ms = max_over_ranks(ms, world, dev)
-    if ia.device_error(stream) != ia.OK:
-        raise RuntimeError("a kernel wait timed out during the timed steps")
-    del graph
+    ms, clk = time_prefill(ia, w, x, dev, stream, args.steps, args.warmup, clocks, world)
     ops = w.effective_ops
     value = aggregate_value(ops, world, ms * 1e-3) / 1e12
 
@@ -304,12 +341,7 @@ def run_ours(args):
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms, 5),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
         "dtype": "int8", "data": "synthetic",
-        "config": {"workload": w.name, "B": w.B, "H": w.H, "Lq": w.Lq, "Lk": w.Lk, "d": w.d,
-                   "causal": w.causal, "clip_c": w.clip_c,
-                   "quant": "per_head" if w.per_head else "per_tensor",
-                   "l2": f"inputs rotate over {nsets} copies ({nsets * set_bytes / 2**20:.0f} MiB > 126 MiB L2)",
-                   "timing": "K steps captured as one CUDA graph, replayed once between CUDA events",
-                   "parallelism": f"dp{world} (independent problems)"},
+        "config": workload_config(w, world),
         "roofline": {"bound": "tensor", "kernel": "prefill_kernel", "achieved": round(achieved, 3),
                      "peak": round(peak_int8, 1), "unit": "TOPS", "frac": round(achieved / peak_int8, 4),
                      "peak_source": f"{peak_src} {peak_key} x {INT8_OVER_BF16} (dense int8/bf16)",
@@ -322,6 +354,8 @@ def run_ours(args):
         "clocks": clk,
     }
 
+    if not args.no_configs:
+        line["prefill_configs"] = run_prefill_configs(args, ia, dev, stream, world, peak_int8, w.name)
     if not args.no_decode:
         line["decode"] = run_decode(args, dev, stream, world, peaks, peak_src, args.decode_workload)
         line["decode_int4"] = run_decode(args, dev, stream, world, peaks, peak_src,
@@ -335,6 +369,30 @@ def run_ours(args):
     if world > 1:
         import torch.distributed as dist
         dist.destroy_process_group()
+
+
+def run_prefill_configs(args, ia, dev, stream, world, peak_int8, skip):
+    """Every other prefill workload, timed like the headline (rotating
+    inputs, one CUDA graph of calls between CUDA events)."""
+    from integer_only_quantized_b200 import workloads as wl
+    res = {}
+    for name in PREFILL_WORKLOADS:
+        if name == skip:
+            continue
+        w = wl.WORKLOADS[name]
+        x = wl.make_inputs(w)
+        nsets, set_bytes = rotation(w)
+        steps = max(args.steps, 100, nsets)  # every copy is used at least once
+        ms, _ = time_prefill(ia, w, x, dev, stream, steps, max(3, args.warmup), None, world)
+        tops = w.effective_ops / (ms * 1e-3) / 1e12
+        res[name] = {"value": round(aggregate_value(w.effective_ops, world, ms * 1e-3) / 1e12, 3), "unit": "TOPS",
+                     "ms_per_call": round(ms, 5), "calls": steps, "launches_per_call": 1,
+                     "effective_ops": w.effective_ops,
+                     "roofline": {"bound": "tensor", "achieved": round(tops, 3), "peak": round(peak_int8, 1),
+                                  "unit": "TOPS", "frac": round(tops / peak_int8, 4),
+                                  "traffic": kernel_traffic("prefill_kernel", name)},
+                     "l2": f"inputs rotate over {nsets} copies ({nsets * set_bytes / 2**20:.0f} MiB > 126 MiB L2)"}
+    return res
 
 
 def run_quantize(args, dev, stream, world, peaks, peak_src):
@@ -514,9 +572,7 @@ def run_reference(args):
             "ms_per_step": round(1e3 * total_t / args.steps, 3), "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "int8", "data": "synthetic",
             "impl": "reference",
-            "config": {"workload": w.name, "B": w.B, "H": w.H, "Lq": w.Lq, "Lk": w.Lk, "d": w.d,
-                       "causal": w.causal, "clip_c": w.clip_c,
-                       "quant": "per_head" if w.per_head else "per_tensor"},
+            "config": workload_config(w, world),
             "cpu_baseline": {"value": round(value, 6), "unit": "TOPS", "cores": threads,
                              "kind": "oracle", "sample": f"each step: {sample}"},
             "e2e": {"value": round(value, 6), "unit": "TOPS", "h2d_bytes_per_step": 0,

@@ -33,6 +33,10 @@
  *   - The library allocates and frees nothing, never synchronises the stream
  *     (except intattn_device_error), and launches only on the given stream.
  *     Calls are asynchronous: a 0 return means the work was enqueued.
+ *     One exception: intattn_forward_host (host buffers) creates two copy
+ *     streams per device and events per workspace on first use, runs its
+ *     copies on those streams, and can wait on the host when a host thread
+ *     cycles through more than 64 workspaces (see its comment).
  *   - Scale arrays are HOST pointers, read during the call only.
  *   - d must be 64 or 128; 1 <= Lk <= 65535 (keeps Z < 2^31).
  *   - Return codes are the INTATTN_* values below; on any non-zero return
@@ -129,9 +133,18 @@ size_t intattn_forward_host_workspace_size(int B, int H, int Lq, int Lk, int d);
  * up to 64 workspaces (a 65th workspace waits on the host for the least
  * recently used one's copies to finish and takes its events).  The result
  * is in `out` when `stream` reaches the end of the call; q, k, v and out must
- * stay valid and unmodified until then.  Under stream capture the copy
- * streams fork from and join `stream`, and calls do not overlap.  Return
- * codes as intattn_forward, plus INTATTN_ERR_WORKSPACE. */
+ * stay valid and unmodified until then.
+ * Stream capture: a captured call forks its copy streams from `stream` and
+ * joins them back; it records its own set of events and waits on no event
+ * recorded outside the capture, so captured calls are ordered by `stream`
+ * alone and do not overlap each other.  Replays of the graph must be
+ * ordered on `stream` with other calls on the same workspace.  After a
+ * workspace has been used in a capture, later uncaptured calls on it also
+ * start their copies after the work already on `stream` (a replay may be
+ * there), so they no longer overlap each other: give captured and uncaptured
+ * calls separate workspaces to keep the uncaptured ones overlapped.  A capture that would
+ * need a 65th workspace returns INTATTN_ERR_UNSUPPORTED.  Return codes as
+ * intattn_forward, plus INTATTN_ERR_WORKSPACE. */
 int intattn_forward_host(const int8_t *q, const int8_t *k, const int8_t *v,
                          const intattn_scales_t *scales, int B, int H, int Lq, int Lk, int d,
                          int causal, float clip_c, int8_t *out, void *workspace,

@@ -423,14 +423,27 @@ int copy_streams(cudaStream_t* h2d, cudaStream_t* d2h) {
 // out).  At most kMaxPipes workspaces are tracked; the least recently used
 // one is retired once its events have completed (a host wait that only a
 // thread cycling through more workspaces than that ever meets).
+//
+// Stream capture: a capture may not wait on an event recorded outside it
+// (the dependency would cross the capture boundary), and an uncaptured call
+// may not wait on an event recorded inside one.  Captured calls therefore
+// record a separate set of events (cap_*) and wait on none recorded before
+// the capture: each captured call forks its copy streams from `stream` and
+// joins them back, so captured calls are ordered by `stream` alone.  Once a
+// workspace has been used in a capture, the graph may be replayed on
+// `stream` at any later point, so every later uncaptured call on that
+// workspace also starts its copies after the work already on `stream`.
 struct SlotEvents {
   cudaEvent_t in[2] = {}, done[2] = {}, out[2] = {};
+  cudaEvent_t cap_in[2] = {}, cap_done[2] = {}, cap_out[2] = {};
+  bool cap_events = false;  // cap_* created
+  bool captured = false;    // used in a capture at least once
   int next = 0;
   unsigned long long used = 0;
 };
 
 struct HostPipes {
-  cudaEvent_t fork = nullptr;
+  cudaEvent_t fork = nullptr, cap_fork = nullptr;  // fork events outside and inside captures
   std::unordered_map<const void*, SlotEvents> by_ws;
   unsigned long long clock = 0;
 };
@@ -444,17 +457,31 @@ int make_events(SlotEvents* e) {
   return INTATTN_OK;
 }
 
-// The events of workspace `ws` for this thread and device (created on first use).
-int pipe_of(const void* ws, cudaEvent_t* fork, SlotEvents** out) {
+int make_capture_events(SlotEvents* e) {
+  if (e->cap_events) return INTATTN_OK;
+  cudaEvent_t* all[6] = {&e->cap_in[0], &e->cap_in[1], &e->cap_done[0], &e->cap_done[1], &e->cap_out[0],
+                         &e->cap_out[1]};
+  for (cudaEvent_t* ev : all)
+    if (cudaEventCreateWithFlags(ev, cudaEventDisableTiming) != cudaSuccess) return INTATTN_ERR_CUDA;
+  e->cap_events = true;
+  return INTATTN_OK;
+}
+
+// The events of workspace `ws` for this thread and device (created on first
+// use), and the fork event for a call inside (capturing) or outside a capture.
+int pipe_of(const void* ws, bool capturing, cudaEvent_t* fork, SlotEvents** out) {
   thread_local HostPipes pipes[64];
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return INTATTN_ERR_CUDA;
   HostPipes& p = pipes[dev];
-  if (!p.fork && cudaEventCreateWithFlags(&p.fork, cudaEventDisableTiming) != cudaSuccess) return INTATTN_ERR_CUDA;
+  cudaEvent_t& f = capturing ? p.cap_fork : p.fork;
+  if (!f && cudaEventCreateWithFlags(&f, cudaEventDisableTiming) != cudaSuccess) return INTATTN_ERR_CUDA;
   auto it = p.by_ws.find(ws);
   if (it == p.by_ws.end()) {
     SlotEvents fresh;
     if (p.by_ws.size() >= kMaxPipes) {
+      // retiring a workspace waits on the host, which a capture forbids
+      if (capturing) return INTATTN_ERR_UNSUPPORTED;
       auto lru = p.by_ws.begin();
       for (auto i = p.by_ws.begin(); i != p.by_ws.end(); ++i)
         if (i->second.used < lru->second.used) lru = i;
@@ -464,6 +491,7 @@ int pipe_of(const void* ws, cudaEvent_t* fork, SlotEvents** out) {
           return INTATTN_ERR_CUDA;
       fresh = lru->second;  // its events, now complete, serve the new workspace
       fresh.next = 0;
+      fresh.captured = false;  // the new workspace has not been used in a capture
       p.by_ws.erase(lru);
     } else if (make_events(&fresh) != INTATTN_OK) {
       return INTATTN_ERR_CUDA;
@@ -471,7 +499,7 @@ int pipe_of(const void* ws, cudaEvent_t* fork, SlotEvents** out) {
     it = p.by_ws.emplace(ws, fresh).first;
   }
   it->second.used = ++p.clock;
-  *fork = p.fork;
+  *fork = f;
   *out = &it->second;
   return INTATTN_OK;
 }
@@ -506,18 +534,29 @@ int intattn_forward_host(const int8_t* q, const int8_t* k, const int8_t* v, cons
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream), h2d = nullptr, d2h = nullptr;
   cudaEvent_t e_fork = nullptr;
   SlotEvents* pipe = nullptr;
-  if (copy_streams(&h2d, &d2h) || pipe_of(workspace, &e_fork, &pipe)) return INTATTN_ERR_CUDA;
-  const int sl = pipe->next;
-  pipe->next = sl ^ 1;
-  cudaEvent_t e_in = pipe->in[sl], e_done = pipe->done[sl], e_out = pipe->out[sl];
   cudaStreamCaptureStatus cap = cudaStreamCaptureStatusNone;
   if (note_launch(cudaStreamIsCapturing(st, &cap))) return INTATTN_ERR_CUDA;
-  if (cap != cudaStreamCaptureStatusNone) {
-    // under stream capture the copy streams join the capture through `stream`
+  const bool capturing = cap != cudaStreamCaptureStatusNone;
+  if (copy_streams(&h2d, &d2h)) return INTATTN_ERR_CUDA;
+  if (const int prc = pipe_of(workspace, capturing, &e_fork, &pipe)) return prc;
+  if (capturing && make_capture_events(pipe) != INTATTN_OK) return INTATTN_ERR_CUDA;
+  const int sl = pipe->next;
+  pipe->next = sl ^ 1;
+  cudaEvent_t e_in = capturing ? pipe->cap_in[sl] : pipe->in[sl];
+  cudaEvent_t e_done = capturing ? pipe->cap_done[sl] : pipe->done[sl];
+  cudaEvent_t e_out = capturing ? pipe->cap_out[sl] : pipe->out[sl];
+  if (capturing || pipe->captured) {
+    // the copy streams start after the work already on `stream`: under
+    // capture this is how they join the capture; after a capture, how they
+    // wait for any replay of it
     if (note_launch(cudaEventRecord(e_fork, st)) || note_launch(cudaStreamWaitEvent(h2d, e_fork, 0)) ||
         note_launch(cudaStreamWaitEvent(d2h, e_fork, 0)))
       return INTATTN_ERR_CUDA;
   }
+  // the slot's previous use: ordered by `stream` under capture (each
+  // captured call ends joined to it), by the slot's events otherwise
+  const bool wait_prev = !capturing;
+  if (capturing) pipe->captured = true;
   const size_t bh = static_cast<size_t>(B) * H;
   const size_t qn = bh * Lq * d, kvn = bh * Lk * d;
   char* base = static_cast<char*>(workspace) + sl * slot_bytes;
@@ -529,12 +568,12 @@ int intattn_forward_host(const int8_t* q, const int8_t* k, const int8_t* v, cons
   // forward once they have landed and the slot's previous output has been
   // copied out; the copy out once the forward is done.  The copies of the
   // next call (other slot) overlap this call's forward and copy out.
-  if (note_launch(cudaStreamWaitEvent(h2d, e_done, 0)) ||
+  if ((wait_prev && note_launch(cudaStreamWaitEvent(h2d, e_done, 0))) ||
       note_launch(cudaMemcpyAsync(dq, q, qn, cudaMemcpyHostToDevice, h2d)) ||
       note_launch(cudaMemcpyAsync(dk, k, kvn, cudaMemcpyHostToDevice, h2d)) ||
       note_launch(cudaMemcpyAsync(dv, v, kvn, cudaMemcpyHostToDevice, h2d)) ||
       note_launch(cudaEventRecord(e_in, h2d)) || note_launch(cudaStreamWaitEvent(st, e_in, 0)) ||
-      note_launch(cudaStreamWaitEvent(st, e_out, 0)))
+      (wait_prev && note_launch(cudaStreamWaitEvent(st, e_out, 0))))
     return INTATTN_ERR_CUDA;
   const int rc = intattn_forward(dq, dk, dv, scales, B, H, Lq, Lk, d, causal, clip_c, dout, stream);
   if (rc) return rc;

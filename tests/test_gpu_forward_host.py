@@ -145,3 +145,48 @@ def test_forward_host_workspace_errors(ia):
     with pytest.raises(ia.IntAttnError) as e:
         ia.forward_host(q, k, v, sc, False, w.clip_c, workspace=small)
     assert e.value.code == ia.ERR_WORKSPACE
+
+
+def test_forward_host_under_stream_capture(ia, oracle_mod):
+    """Uncaptured calls first (their slot events are recorded outside any
+    capture), then two calls captured as a CUDA graph on the same workspace
+    and replayed twice, then uncaptured calls again: every output equals the
+    oracle's.  A captured call must not wait on events recorded outside the
+    capture, nor an uncaptured call on events recorded inside one."""
+    import torch
+    runs = []
+    for i in range(2):
+        w = wl.custom_workload("host_graph", 2, 3, 150, 150, 64, bool(i), per_head=True, index=1500 + i)
+        x = wl.make_inputs(w)
+        want = oracle_mod.forward(x.q, x.k, x.v, True, x.s_q, x.s_k, x.s_v, x.s_o, w.causal, w.clip_c)
+        runs.append((w, x, [_host(a, True) for a in (x.q, x.k, x.v)],
+                     torch.empty(x.q.shape, dtype=torch.int8).pin_memory(), want))
+    ws = torch.empty(ia.forward_host_workspace_size(2, 3, 150, 150, 64), dtype=torch.uint8, device="cuda")
+    s = torch.cuda.Stream()
+
+    def call_all():
+        for w, x, (q, k, v), out, _ in runs:
+            ia.forward_host(q, k, v, ia.Scales(x.s_q, x.s_k, x.s_v, x.s_o, per_head=True), w.causal, w.clip_c,
+                            out=out, workspace=ws, stream=s)
+
+    def check(what):
+        for i, (_, _, _, out, want) in enumerate(runs):
+            assert np.array_equal(out.numpy(), want), f"{what}: call {i} differs from the oracle"
+            out.fill_(0x5A)
+
+    with torch.cuda.stream(s):
+        call_all()
+        s.synchronize()
+        check("warm-up")
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=s):
+            call_all()
+        for rep in range(2):
+            g.replay()
+            s.synchronize()
+            check(f"replay {rep}")
+        call_all()  # uncaptured again, after the capture, on the same workspace
+        s.synchronize()
+        check("after capture")
+    del g
+    assert ia.device_error() == ia.OK

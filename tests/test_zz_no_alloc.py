@@ -4,8 +4,9 @@ It serves callers that cannot allocate device memory where they call us (a
 plugin living under another framework's caching allocator with no workspace
 to offer, or a latency-bound loop that must not call cudaMalloc): the split-K
 scratch comes from a fixed array inside the library instead of a caller
-workspace.  Its output must equal intattn_decode's, call after call, while
-the shared array keeps whatever the previous call left in it.
+workspace.  Its output must equal intattn_decode's (which is checked against the CPU
+oracle here too), call after call, while the shared array keeps whatever the
+previous call left in it.
 
 This file is collected last on purpose, so a stop-at-first-failure run has
 already run every other test; it also passes on its own in a fresh process.
@@ -50,7 +51,7 @@ def _static_call(ia, x, w, out):
 
 
 @pytest.mark.parametrize("case", CASES, ids=lambda c: "B{}H{}Lk{}d{}".format(c[0], c[1], c[2], c[4]))
-def test_static_scratch_matches_workspace_decode(ia, case):
+def test_static_scratch_matches_workspace_decode(ia, oracle_mod, case):
     import torch
     B, H, Lk, Lmax, d, per_head = case
     w = wl.custom_workload("noalloc", B, H, 1, Lk, d, False, per_head=per_head, clip_c=10.0,
@@ -60,6 +61,10 @@ def test_static_scratch_matches_workspace_decode(ia, case):
     ref = ia.decode(x.q, x.k, x.v, ia.Scales(x.s_q, x.s_k, x.s_v, x.s_o, per_head=per_head), Lk, w.clip_c)
     torch.cuda.synchronize()
     want = ref.cpu().numpy()
+    # the workspace decode itself against the CPU oracle, so this file stands on its own
+    oracle_out = oracle_mod.decode(x.q.cpu().numpy(), x.k.cpu().numpy(), x.v.cpu().numpy(), per_head,
+                                   x.s_q, x.s_k, x.s_v, x.s_o, Lk, w.clip_c)
+    assert np.array_equal(want, oracle_out), f"{int((want != oracle_out).sum())} bytes differ from the oracle"
     for call in range(2):  # the second call sees the first call's leftovers
         out = torch.full_like(x.q, 99)
         rc = _static_call(ia, x, w, out)
