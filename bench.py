@@ -228,27 +228,29 @@ def time_prefill(ia, w, x, dev, stream, steps: int, warmup: int, clocks=None, wo
         q, k, v, o = sets[i % nsets]
         ia.forward(q, k, v, sc, w.causal, w.clip_c, out=o, stream=stream)
 
-    for i in range(warmup):
-        step(i)
-    torch.cuda.synchronize(dev)
-    if ia.device_error(stream) != ia.OK:
-        raise RuntimeError("a kernel wait timed out during warm-up")
-    # the timed steps are captured once as a CUDA graph and replayed: the
-    # device time then excludes the host's per-call launch latency
-    graph = torch.cuda.CUDAGraph()
-    with torch.cuda.graph(graph, stream=stream):
-        for i in range(steps):
+    # everything on `stream`: the calls, the capture, the replay and the events
+    with torch.cuda.stream(stream):
+        for i in range(warmup):
             step(i)
-    torch.cuda.synchronize(dev)
-    barrier(world, dev)
-    torch.cuda.synchronize(dev)
-    if clocks is not None:
-        clocks.start()
-    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    t0.record(stream)
-    graph.replay()
-    t1.record(stream)
-    torch.cuda.synchronize(dev)
+        torch.cuda.synchronize(dev)
+        if ia.device_error(stream) != ia.OK:
+            raise RuntimeError("a kernel wait timed out during warm-up")
+        # the timed steps are captured once as a CUDA graph and replayed: the
+        # device time then excludes the host's per-call launch latency
+        graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(graph, stream=stream):
+            for i in range(steps):
+                step(i)
+        torch.cuda.synchronize(dev)
+        barrier(world, dev)
+        torch.cuda.synchronize(dev)
+        if clocks is not None:
+            clocks.start()
+        t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        t0.record(stream)
+        graph.replay()
+        t1.record(stream)
+        torch.cuda.synchronize(dev)
     barrier(world, dev)
     clk = clocks.stop() if clocks is not None else None
     ms = max_over_ranks(t0.elapsed_time(t1) / steps, world, dev)
@@ -335,6 +337,8 @@ def run_ours(args):
     peaks, peak_src = load_peaks()
     peak_int8, peak_key = _int8_peak(peaks, sustained=False)
     achieved = ops / (ms * 1e-3) / 1e12  # one launch per step: per-launch duration = ms
+    if achieved > 1.5 * peak_int8:
+        raise RuntimeError(f"{achieved:.0f} TOPS is far above the int8 peak: the timed region missed the work")
     traffic = kernel_traffic("prefill_kernel", w.name)
     line = {
         "metric": METRIC, "value": round(value, 3), "unit": "TOPS", "n_gpus": world,
@@ -385,6 +389,8 @@ def run_prefill_configs(args, ia, dev, stream, world, peak_int8, skip):
         steps = max(args.steps, 100, nsets)  # every copy is used at least once
         ms, _ = time_prefill(ia, w, x, dev, stream, steps, max(3, args.warmup), None, world)
         tops = w.effective_ops / (ms * 1e-3) / 1e12
+        if tops > 1.5 * peak_int8:
+            raise RuntimeError(f"{name}: {tops:.0f} TOPS is far above the int8 peak: the timed region missed the work")
         res[name] = {"value": round(aggregate_value(w.effective_ops, world, ms * 1e-3) / 1e12, 3), "unit": "TOPS",
                      "ms_per_call": round(ms, 5), "calls": steps, "launches_per_call": 1,
                      "effective_ops": w.effective_ops,

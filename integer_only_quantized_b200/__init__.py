@@ -22,12 +22,15 @@ MAX_HEADS = 128
 MAX_CLIPS = 8
 
 # every function declared in include/intattn.h
-EXPORTED = ("intattn_derive_params", "intattn_forward", "intattn_forward_host_workspace_size",
+EXPORTED = ("intattn_derive_params", "intattn_forward", "intattn_forward_variant",
+            "intattn_forward_host_workspace_size",
             "intattn_forward_host", "intattn_decode_workspace_size",
             "intattn_decode", "intattn_decode_int4", "intattn_decode_static_scratch", "intattn_quantize",
             "intattn_gelu_derive_params", "intattn_gelu", "intattn_selftest_timeout", "intattn_device_error",
             "intattn_strerror")
 DTYPE_FP16, DTYPE_BF16 = 0, 1
+VARIANT_AUTO, VARIANT_THREE_PASS, VARIANT_SHORT_ROWS = 0, 1, 2
+SHORT_ROWS_MAX_KEYS = 512
 
 
 class _GeluParams(ctypes.Structure):
@@ -99,6 +102,8 @@ def lib() -> ctypes.CDLL:
                                             ctypes.POINTER(ctypes.c_int32), ctypes.POINTER(_HeadParams)]
         L.intattn_forward.argtypes = [vp, vp, vp, ctypes.POINTER(_Scales), i32, i32, i32, i32, i32,
                                       i32, f32, vp, vp]
+        L.intattn_forward_variant.argtypes = [vp, vp, vp, ctypes.POINTER(_Scales), i32, i32, i32, i32, i32,
+                                              i32, f32, vp, i32, vp]
         L.intattn_forward_host_workspace_size.argtypes = [i32, i32, i32, i32, i32]
         L.intattn_forward_host_workspace_size.restype = ctypes.c_size_t
         L.intattn_forward_host.argtypes = [vp, vp, vp, ctypes.POINTER(_Scales), i32, i32, i32, i32, i32,
@@ -158,8 +163,10 @@ def _check_tensor(t, name: str):
         raise ValueError(f"{name} must be contiguous")
 
 
-def forward(q, k, v, scales: Scales, causal: bool, clip_c: float, out=None, stream=None):
-    """out[B,H,Lq,d] int8 = IntAttention forward of int8 q[B,H,Lq,d], k/v[B,H,Lk,d]."""
+def forward(q, k, v, scales: Scales, causal: bool, clip_c: float, out=None, stream=None, variant: int = 0):
+    """out[B,H,Lq,d] int8 = IntAttention forward of int8 q[B,H,Lq,d], k/v[B,H,Lk,d].
+    variant: VARIANT_AUTO (intattn_forward), VARIANT_THREE_PASS or
+    VARIANT_SHORT_ROWS (intattn_forward_variant); the bytes are the same."""
     import torch
     for t, n in ((q, "q"), (k, "k"), (v, "v")):
         _check_tensor(t, n)
@@ -173,9 +180,14 @@ def forward(q, k, v, scales: Scales, causal: bool, clip_c: float, out=None, stre
     if out.shape != q.shape:
         raise ValueError("out must match q")
     sc, keep = scales._c()
-    rc = lib().intattn_forward(q.data_ptr(), k.data_ptr(), v.data_ptr(), ctypes.byref(sc), B, H, Lq, Lk,
-                               d, int(bool(causal)), float(clip_c), out.data_ptr(),
-                               _stream_handle(stream, q.device))
+    if variant == VARIANT_AUTO:
+        rc = lib().intattn_forward(q.data_ptr(), k.data_ptr(), v.data_ptr(), ctypes.byref(sc), B, H, Lq, Lk,
+                                   d, int(bool(causal)), float(clip_c), out.data_ptr(),
+                                   _stream_handle(stream, q.device))
+    else:
+        rc = lib().intattn_forward_variant(q.data_ptr(), k.data_ptr(), v.data_ptr(), ctypes.byref(sc), B, H,
+                                           Lq, Lk, d, int(bool(causal)), float(clip_c), out.data_ptr(),
+                                           int(variant), _stream_handle(stream, q.device))
     del keep
     _check(rc, "intattn_forward")
     return out

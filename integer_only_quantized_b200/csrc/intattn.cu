@@ -21,6 +21,7 @@
 #include "gelu_kernel.cuh"
 #include "quantize_kernel.cuh"
 #include "prefill_kernel.cuh"
+#include "prefill_short_kernel.cuh"
 
 using intattn::DecodeArgs;
 using intattn::HeadParamsDev;
@@ -182,6 +183,23 @@ int prefill_launch(const PrefillArgs& args, int grid, cudaStream_t stream) {
     attr_set[dev] = true;
   }
   intattn::prefill::prefill_kernel<D><<<grid, intattn::prefill::kThreads, C::kSmemBytes, stream>>>(args);
+  return note_launch(cudaGetLastError());
+}
+
+template <int D>
+int prefill_short_launch(const PrefillArgs& args, int grid, cudaStream_t stream) {
+  using C = intattn::shortrow::Cfg<D>;
+  static bool attr_set[64] = {};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return INTATTN_ERR_CUDA;
+  if (dev < 0 || dev >= 64) return INTATTN_ERR_CUDA;
+  if (!attr_set[dev]) {
+    if (cudaFuncSetAttribute(intattn::shortrow::prefill_short_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             static_cast<int>(C::kSmemBytes)) != cudaSuccess)
+      return INTATTN_ERR_CUDA;
+    attr_set[dev] = true;
+  }
+  intattn::shortrow::prefill_short_kernel<D><<<grid, intattn::shortrow::kThreads, C::kSmemBytes, stream>>>(args);
   return note_launch(cudaGetLastError());
 }
 
@@ -347,6 +365,17 @@ int intattn_derive_params(const intattn_scales_t* scales, int H, int d, float cl
 int intattn_forward(const int8_t* q, const int8_t* k, const int8_t* v, const intattn_scales_t* scales, int B,
                     int H, int Lq, int Lk, int d, int causal, float clip_c, int8_t* out,
                     intattn_stream_t stream) {
+  return intattn_forward_variant(q, k, v, scales, B, H, Lq, Lk, d, causal, clip_c, out, INTATTN_VARIANT_AUTO,
+                                 stream);
+}
+
+int intattn_forward_variant(const int8_t* q, const int8_t* k, const int8_t* v, const intattn_scales_t* scales,
+                            int B, int H, int Lq, int Lk, int d, int causal, float clip_c, int8_t* out,
+                            int variant, intattn_stream_t stream) {
+  if (variant != INTATTN_VARIANT_AUTO && variant != INTATTN_VARIANT_THREE_PASS &&
+      variant != INTATTN_VARIANT_SHORT_ROWS)
+    return INTATTN_ERR_INVALID_ARG;
+  if (variant == INTATTN_VARIANT_SHORT_ROWS && Lk > intattn::shortrow::kMaxKeys) return INTATTN_ERR_UNSUPPORTED;
   if (B < 0 || H <= 0 || Lq < 0 || Lk < 1 || Lk > 65535) return INTATTN_ERR_INVALID_ARG;
   if (causal && Lq > Lk) return INTATTN_ERR_INVALID_ARG;
   if (d != 64 && d != 128) return INTATTN_ERR_UNSUPPORTED;
@@ -380,6 +409,11 @@ int intattn_forward(const int8_t* q, const int8_t* k, const int8_t* v, const int
   // persistent kernel: one CTA per SM (each holds all 512 TMEM columns)
   const int grid = args.n_tiles < sms ? args.n_tiles : sms;
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  // rows of at most 512 keys: index codes kept in registers (no third Q.K^T)
+  const bool short_rows = variant == INTATTN_VARIANT_SHORT_ROWS ||
+                          (variant == INTATTN_VARIANT_AUTO && Lk <= intattn::shortrow::kMaxKeys);
+  if (short_rows)
+    return d == 64 ? prefill_short_launch<64>(args, grid, st) : prefill_short_launch<128>(args, grid, st);
   return d == 64 ? prefill_launch<64>(args, grid, st) : prefill_launch<128>(args, grid, st);
 }
 

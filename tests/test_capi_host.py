@@ -102,6 +102,23 @@ def test_forward_argument_errors_need_no_device(ia):
     assert L.intattn_forward(16, 16, 16, None, 1, 1, 4, 4, 64, 0, 8.0, 16, None) == ia.ERR_INVALID_ARG
 
 
+def test_forward_variant_argument_errors_need_no_device(ia):
+    sc = ia.Scales(0.1, 0.1, 0.1, 0.1)
+    s, keep = sc._c()
+    L = ia.lib()
+
+    def fv(variant, Lk=4, d=64, B=1):
+        return L.intattn_forward_variant(16, 16, 16, ctypes.byref(s), B, 2, 4, Lk, d, 0, 8.0, 16, variant, None)
+
+    assert fv(3) == ia.ERR_INVALID_ARG
+    assert fv(-1) == ia.ERR_INVALID_ARG
+    assert fv(ia.VARIANT_SHORT_ROWS, Lk=ia.SHORT_ROWS_MAX_KEYS + 1) == ia.ERR_UNSUPPORTED
+    assert fv(ia.VARIANT_THREE_PASS, d=96) == ia.ERR_UNSUPPORTED
+    assert fv(ia.VARIANT_SHORT_ROWS, Lk=0) == ia.ERR_INVALID_ARG
+    for variant in (ia.VARIANT_AUTO, ia.VARIANT_THREE_PASS, ia.VARIANT_SHORT_ROWS):
+        assert fv(variant, B=0) == ia.OK  # nothing to do, no launch
+
+
 def test_misaligned_pointer_is_rejected(ia):
     sc = ia.Scales(0.1, 0.1, 0.1, 0.1)
     s, keep = sc._c()

@@ -206,3 +206,78 @@ def test_decode_matches_prefill_last_row(ia):
     for i in (0, 350, 699):
         out = ia.decode(_dev(x.q[:, :, i:i + 1]), _dev(x.k), _dev(x.v), sc, i + 1, w.clip_c)
         _assert_equal(out.cpu().numpy()[:, :, 0], pre[:, :, i], f"row {i}")
+
+
+# ---------------------------------------------- kernel variants, short rows
+
+def _variant_forward(ia, x, w, variant, guard=1024):
+    import torch
+    sc = ia.Scales(x.s_q, x.s_k, x.s_v, x.s_o, per_head=w.per_head)
+    q, k, v = _dev(x.q), _dev(x.k), _dev(x.v)
+    n = x.q.size
+    buf = torch.full((n + 2 * guard,), 0x5A, dtype=torch.int8, device="cuda")
+    out = buf[guard:guard + n].view(x.q.shape)
+    ia.forward(q, k, v, sc, w.causal, w.clip_c, out=out, variant=variant)
+    assert ia.device_error() == ia.OK
+    b = buf.cpu().numpy()
+    assert np.all(b[:guard] == 0x5A) and np.all(b[guard + n:] == 0x5A), "write outside out"
+    return out.cpu().numpy()
+
+
+SHORT_SWEEP = [
+    # (B, H, Lq, Lk, d, causal, per_head, dist): every Lk <= 512
+    (1, 1, 1, 1, 64, False, False, "normal"),
+    (2, 3, 32, 32, 128, False, True, "normal"),
+    (1, 2, 33, 33, 64, True, False, "normal"),
+    (2, 2, 127, 127, 64, False, True, "student_t4"),
+    (1, 2, 129, 129, 128, True, True, "normal"),
+    (3, 4, 197, 197, 64, False, True, "student_t4"),
+    (1, 3, 256, 256, 128, False, False, "normal"),
+    (1, 3, 257, 257, 64, True, False, "normal"),
+    (2, 2, 300, 300, 128, False, True, "normal"),
+    (1, 2, 384, 384, 64, True, True, "normal"),
+    (1, 2, 511, 511, 128, True, False, "normal"),
+    (2, 3, 512, 512, 64, False, False, "normal"),
+    (1, 2, 100, 512, 64, True, False, "normal"),     # Lq < Lk, bottom-right causal
+    (1, 2, 600, 200, 128, False, True, "normal"),    # cross attention, more queries than keys
+    (8, 40, 512, 512, 64, True, True, "normal"),     # 1280 tiles: CTAs mix 1..4 key tiles
+    (24, 12, 197, 197, 64, False, True, "student_t4"),  # 576 tiles: several rounds of resident tiles
+]
+
+
+@pytest.mark.parametrize("case", SHORT_SWEEP, ids=lambda c: "B{}H{}Lq{}Lk{}d{}{}{}".format(
+    c[0], c[1], c[2], c[3], c[4], "c" if c[5] else "", "h" if c[6] else ""))
+def test_short_row_variants_match_oracle(ia, oracle_mod, case):
+    """Both kernels on rows of at most 512 keys: the short-row kernel (codes
+    kept in registers, resident scores up to 256 keys) and the three-pass
+    kernel must each give the oracle's bytes."""
+    B, H, Lq, Lk, d, causal, per_head, dist = case
+    w = wl.custom_workload("short", B, H, Lq, Lk, d, causal, per_head=per_head, dist=dist,
+                           clip_c=8.0 if d == 64 else 10.0, index=2000 + Lq + 3 * Lk + d + B)
+    x = wl.make_inputs(w)
+    want = _oracle_forward(oracle_mod, x, w)
+    for variant in (ia.VARIANT_SHORT_ROWS, ia.VARIANT_THREE_PASS):
+        _assert_equal(_variant_forward(ia, x, w, variant), want, f"{case} variant {variant}")
+
+
+@pytest.mark.parametrize("name", ["bert_base_l128", "bert_base_b8_l512", "vit_b16_l197"])
+def test_workload_both_variants(ia, oracle_mod, name):
+    """The short-row workloads through each kernel explicitly."""
+    w = wl.WORKLOADS[name]
+    x = wl.make_inputs(w)
+    want = _oracle_forward(oracle_mod, x, w)
+    for variant in (ia.VARIANT_SHORT_ROWS, ia.VARIANT_THREE_PASS):
+        _assert_equal(_variant_forward(ia, x, w, variant, guard=4096), want, f"{name} variant {variant}")
+
+
+@pytest.mark.parametrize("d", [64, 128])
+def test_short_rows_extreme_codes(ia, oracle_mod, d):
+    """Largest |S| and all-equal rows through the short-row kernel."""
+    import dataclasses
+    w = wl.custom_workload("short_extreme", 2, 3, 300, 300, d, True, index=2700 + d)
+    x = wl.make_inputs(w)
+    cases = [dataclasses.replace(x, q=np.full_like(x.q, -128), k=np.full_like(x.k, -128)),
+             dataclasses.replace(x, q=np.zeros_like(x.q))]
+    for xx in cases:
+        _assert_equal(_variant_forward(ia, xx, w, ia.VARIANT_SHORT_ROWS), _oracle_forward(oracle_mod, xx, w),
+                      "extreme")
