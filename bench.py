@@ -213,7 +213,7 @@ def workload_config(w, world: int) -> dict:
             "parallelism": f"dp{world} (independent problems)"}
 
 
-def time_prefill(ia, w, x, dev, stream, steps: int, warmup: int, clocks=None, world: int = 1):
+def time_prefill(ia, w, x, dev, stream, steps: int, warmup: int, clocks=None, world: int = 1, variant: int = 0):
     """ms per forward of workload w: `steps` calls over rotating copies of the
     inputs, captured as one CUDA graph and replayed between CUDA events on
     `stream`; max over ranks."""
@@ -226,7 +226,7 @@ def time_prefill(ia, w, x, dev, stream, steps: int, warmup: int, clocks=None, wo
 
     def step(i):
         q, k, v, o = sets[i % nsets]
-        ia.forward(q, k, v, sc, w.causal, w.clip_c, out=o, stream=stream)
+        ia.forward(q, k, v, sc, w.causal, w.clip_c, out=o, stream=stream, variant=variant)
 
     # everything on `stream`: the calls, the capture, the replay and the events
     with torch.cuda.stream(stream):
@@ -398,6 +398,20 @@ def run_prefill_configs(args, ia, dev, stream, world, peak_int8, skip):
                                   "unit": "TOPS", "frac": round(tops / peak_int8, 4),
                                   "traffic": kernel_traffic("prefill_kernel", name)},
                      "l2": f"inputs rotate over {nsets} copies ({nsets * set_bytes / 2**20:.0f} MiB > 126 MiB L2)"}
+        if w.Lk <= 2 * ia.SHORT_ROWS_MAX_KEYS:
+            # both ways of handling a short row's scores on the same workload:
+            # resident in tensor memory (what intattn_forward runs up to 256
+            # keys) and recomputed per sweep (the three-pass kernel)
+            variants = {}
+            pairs = [("three_pass", ia.VARIANT_THREE_PASS)]
+            if w.Lk <= ia.SHORT_ROWS_MAX_KEYS:
+                pairs.insert(0, ("short_rows", ia.VARIANT_SHORT_ROWS))
+            for vname, vid in pairs:
+                vms, _ = time_prefill(ia, w, x, dev, stream, steps, max(3, args.warmup), None, world, vid)
+                vt = w.effective_ops / (vms * 1e-3) / 1e12
+                variants[vname] = {"ms_per_call": round(vms, 5), "value": round(vt, 3),
+                                   "frac": round(vt / peak_int8, 4)}
+            res[name]["variants"] = variants
     return res
 
 

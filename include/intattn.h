@@ -113,16 +113,15 @@ int intattn_forward(const int8_t *q, const int8_t *k, const int8_t *v,
 
 /* Kernel choice of intattn_forward_variant. */
 enum {
-    INTATTN_VARIANT_AUTO = 0,        /* what intattn_forward does: SHORT_ROWS when Lk <= 512, else THREE_PASS */
+    INTATTN_VARIANT_AUTO = 0,        /* what intattn_forward does: SHORT_ROWS when Lk <= 256, else THREE_PASS */
     INTATTN_VARIANT_THREE_PASS = 1,  /* scores recomputed by the tensor core in each of the three sweeps */
-    INTATTN_VARIANT_SHORT_ROWS = 2   /* Lk <= 512: index codes kept in registers after the second sweep, so
-                                        the third needs no scores; with Lk <= 256 the scores also stay in
-                                        tensor memory between the first two sweeps (one Q.K^T per key tile) */
+    INTATTN_VARIANT_SHORT_ROWS = 2   /* Lk <= 256: the scores of a 128-row tile stay in tensor memory through
+                                        all three sweeps (one Q.K^T per key tile) */
 };
 
 /* intattn_forward with an explicit kernel choice (for measuring the
  * variants against each other; every variant computes the same bytes).
- * SHORT_ROWS with Lk > 512 returns INTATTN_ERR_UNSUPPORTED; an unknown
+ * SHORT_ROWS with Lk > 256 returns INTATTN_ERR_UNSUPPORTED; an unknown
  * variant INTATTN_ERR_INVALID_ARG.  Otherwise as intattn_forward. */
 int intattn_forward_variant(const int8_t *q, const int8_t *k, const int8_t *v,
                             const intattn_scales_t *scales, int B, int H, int Lq, int Lk, int d,

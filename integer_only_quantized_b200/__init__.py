@@ -30,7 +30,7 @@ EXPORTED = ("intattn_derive_params", "intattn_forward", "intattn_forward_variant
             "intattn_strerror")
 DTYPE_FP16, DTYPE_BF16 = 0, 1
 VARIANT_AUTO, VARIANT_THREE_PASS, VARIANT_SHORT_ROWS = 0, 1, 2
-SHORT_ROWS_MAX_KEYS = 512
+SHORT_ROWS_MAX_KEYS = 256
 
 
 class _GeluParams(ctypes.Structure):

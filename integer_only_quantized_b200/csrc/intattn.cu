@@ -110,6 +110,17 @@ int derive(const intattn_scales_t* sc, int H, int d, float clip_c, uint32_t lut[
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
+// Multiplier and shift with floor(n / d) == (n m) >> sh for every 0 <= n < 2^31
+// and d >= 1: m = ceil(2^(31 + l) / d), sh = 31 + l, l = ceil(log2 d) (the
+// round-up reciprocal of Granlund and Montgomery for 31-bit dividends; m < 2^32).
+void div_magic(uint32_t d, uint32_t* m, int32_t* sh) {
+  int l = 0;
+  while ((1ull << l) < d) ++l;
+  const int k = 31 + l;
+  *m = static_cast<uint32_t>(((1ull << k) + d - 1) / d);
+  *sh = k;
+}
+
 // ------------------------------------------------------------------- TMA
 using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
                                    const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
@@ -404,12 +415,14 @@ int intattn_forward_variant(const int8_t* q, const int8_t* k, const int8_t* v, c
   args.n_qtiles = n_qtiles;
   args.per_head = scales->per_head ? 1 : 0;
   args.n_tiles = static_cast<int32_t>(BH * n_qtiles);
+  div_magic(static_cast<uint32_t>(BH), &args.div_bh_m, &args.div_bh_sh);
+  div_magic(static_cast<uint32_t>(H), &args.div_h_m, &args.div_h_sh);
   int sms = 0;
   if (sm_count(&sms) != INTATTN_OK) return INTATTN_ERR_CUDA;
   // persistent kernel: one CTA per SM (each holds all 512 TMEM columns)
   const int grid = args.n_tiles < sms ? args.n_tiles : sms;
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
-  // rows of at most 512 keys: index codes kept in registers (no third Q.K^T)
+  // rows of at most 256 keys: the scores stay in tensor memory through the three sweeps
   const bool short_rows = variant == INTATTN_VARIANT_SHORT_ROWS ||
                           (variant == INTATTN_VARIANT_AUTO && Lk <= intattn::shortrow::kMaxKeys);
   if (short_rows)

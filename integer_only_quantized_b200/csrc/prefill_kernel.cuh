@@ -27,7 +27,6 @@
 //   warps 20-23 epilogue: O of a finished tile (TMEM lane quadrant
 //               warp % 4, one query row per thread) -> requantised int8 rows,
 //               while the softmax warps already work on the next tile.
-//   warps 18-19 none (they complete the fifth warpgroup).
 //
 // The LUT index of a score depends on the final row max and P depends on
 // the final row sum Z, so a bit-exact result needs three sweeps over the
@@ -61,6 +60,9 @@ struct PrefillArgs {
   CUtensorMap tm_v;  // [B*H, Lk, d]
   int8_t* out;       // [B, H, Lq, d]
   int32_t BH, H, Lq, Lk, causal, n_qtiles, per_head, n_tiles, n_luts;
+  // n / BH and n / H for 0 <= n < 2^31 as (n * m) >> sh (host-computed)
+  uint32_t div_bh_m, div_h_m;
+  int32_t div_bh_sh, div_h_sh;
   uint32_t lut[INTATTN_MAX_CLIPS][32];  // one exp table per distinct clip threshold
   HeadParamsDev hp[INTATTN_MAX_HEADS];
 };
@@ -126,10 +128,14 @@ struct Cfg {
   static constexpr int kNumBars = kBarKvFull + 2 * kStages;
   static constexpr uint32_t kOffQ = 0;                                  // [2] Q tiles
   static constexpr uint32_t kOffKV = kOffQ + 2 * kQBytes;
-  static constexpr uint32_t kOffPtab = kOffKV + kStages * kTileBytes;    // [33][kBM] u32
-  static constexpr uint32_t kOffRed = kOffPtab + 33 * kBM * 4;          // [2][kGroups][kBM] int32
+  // probability table, four copies [b][33][kBM] u32 with P << 8b, so four
+  // looked-up bytes pack into a word by integer adds
+  static constexpr uint32_t kPtabBytes = 33 * kBM * 4;
+  static constexpr uint32_t kOffPtab = kOffKV + kStages * kTileBytes;
+  static constexpr uint32_t kOffRed = kOffPtab + 4 * kPtabBytes;        // [2][kGroups][kBM] int32
   static constexpr uint32_t kOffLut = kOffRed + 2 * kGroups * kBM * 4;
-  static constexpr uint32_t kOffBars = kOffLut + INTATTN_MAX_CLIPS * 32 * 4;
+  static constexpr uint32_t kOffHp = kOffLut + INTATTN_MAX_CLIPS * 32 * 4;  // head parameters
+  static constexpr uint32_t kOffBars = kOffHp + INTATTN_MAX_HEADS * sizeof(HeadParamsDev);
   static constexpr uint32_t kOffTmem = kOffBars + kNumBars * 8;
   static constexpr uint32_t kUsed = kOffTmem + 16;
   // One CTA per SM: every CTA allocates all 512 TMEM columns, so the
@@ -144,6 +150,34 @@ __device__ __forceinline__ float fma_rz_sat(float a, float b, float c) {
   float d;
   asm("fma.rz.sat.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
   return d;
+}
+
+// (a0, a1) * b + c in both lanes, rounded toward zero: one packed FP32 FMA.
+// b2 and c2 hold the multiplier and addend twice (pack2 below).
+__device__ __forceinline__ void fma2_rz(float a0, float a1, unsigned long long b2, unsigned long long c2,
+                                        float& d0, float& d1) {
+  asm("{\n\t.reg .b64 a, d;\n\t"
+      "mov.b64 a, {%2, %3};\n\t"
+      "fma.rz.f32x2 d, a, %4, %5;\n\t"
+      "mov.b64 {%0, %1}, d;\n\t}"
+      : "=f"(d0), "=f"(d1)
+      : "f"(a0), "f"(a1), "l"(b2), "l"(c2));
+}
+
+__device__ __forceinline__ unsigned long long pack2(float x) {
+  const unsigned long long u = __float_as_uint(x);
+  return u | (u << 32);
+}
+
+// R = floor((255 2^32 + floor(Z/2)) / Z), Z >= 1: N < 2^40, so the double
+// quotient is within one unit of R, and one integer step makes it exact.
+__device__ __forceinline__ unsigned long long exact_R(int32_t Z) {
+  const unsigned long long N = (255ull << 32) + static_cast<unsigned long long>(Z >> 1);
+  const unsigned long long Zu = static_cast<unsigned long long>(Z);
+  unsigned long long R = static_cast<unsigned long long>(__ddiv_rn(static_cast<double>(N), static_cast<double>(Z)));
+  if (R * Zu > N) --R;
+  else if ((R + 1) * Zu <= N) ++R;
+  return R;
 }
 
 // Requantise one int32 accumulator: clamp(floor((acc Mo + 2^(so-1)) / 2^so)).
@@ -170,13 +204,18 @@ __device__ __forceinline__ int tile_index(int round, int cta, int ctas) {
   return round * ctas + ((round & 1) ? (ctas - 1 - cta) : cta);
 }
 
+// floor(n / d) for 0 <= n < 2^31 with the multiplier and shift of d.
+__device__ __forceinline__ int fast_div(int n, uint32_t m, int sh) {
+  return static_cast<int>((static_cast<unsigned long long>(static_cast<uint32_t>(n)) * m) >> sh);
+}
+
 __device__ __forceinline__ Tile tile_of(const PrefillArgs& a, int L) {
   Tile t;
-  const int rank = L / a.BH;
+  const int rank = fast_div(L, a.div_bh_m, a.div_bh_sh);
   t.bh = L - rank * a.BH;
   const int qt = a.causal ? (a.n_qtiles - 1 - rank) : rank;
   t.q0 = qt * kBM;
-  t.h = t.bh % a.H;
+  t.h = t.bh - fast_div(t.bh, a.div_h_m, a.div_h_sh) * a.H;
   const int off = a.Lk - a.Lq;
   const int q_last = min(t.q0 + kBM, a.Lq) - 1;
   const int kend = a.causal ? min(a.Lk, q_last + off + 1) : a.Lk;
@@ -196,6 +235,7 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_kernel(const __grid_const
   uint32_t* ptab = reinterpret_cast<uint32_t*>(smem + C::kOffPtab);
   int32_t* red = reinterpret_cast<int32_t*>(smem + C::kOffRed);
   uint32_t* lut_s = reinterpret_cast<uint32_t*>(smem + C::kOffLut);
+  HeadParamsDev* hp_s = reinterpret_cast<HeadParamsDev*>(smem + C::kOffHp);
   const uint32_t bars = s_base + C::kOffBars;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::kOffTmem);
   auto bar = [&](int i) { return bars + 8u * static_cast<uint32_t>(i); };
@@ -231,6 +271,9 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_kernel(const __grid_const
     mbar_fence_init();
   }
   for (int i = tid; i < args.n_luts * 32; i += blockDim.x) lut_s[i] = args.lut[i >> 5][i & 31];
+  // head parameters in shared memory: a dynamically indexed kernel argument
+  // is a constant-bank load that can miss
+  for (int i = tid; i < (args.per_head ? args.H : 1); i += blockDim.x) hp_s[i] = args.hp[i];
   if (warp == kMmaWarp) {
     tmem_alloc(smem_u32(tmem_slot), kTmemCols);
     tmem_relinquish();
@@ -258,7 +301,8 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_kernel(const __grid_const
     // 0); a shuffle whose source lane is the low 5 bits of the code looks it
     // up.  Per tile a thread sums 32 values below 2^15: the float sums are exact.
     int32_t lut_lane = 0;  // set per tile: the table of the tile's head
-    if (sw < 4) ptab[r] = 0u;  // table row 0 (masked keys) stays 0
+    if (sw < 4)
+      for (int b = 0; b < 4; ++b) ptab[b * (C::kPtabBytes / 4) + r] = 0u;  // table row 0 (masked keys) stays 0
     bool ok = true;
     uint32_t sc = 0;  // S tiles of the CTA so far (both teams, all passes and tiles)
     uint32_t pc = 0;  // P tiles of the CTA so far
@@ -301,7 +345,7 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_kernel(const __grid_const
       const int L = tile_index(it, blockIdx.x, gridDim.x);
       if (L >= args.n_tiles) break;
       const Tile T = tile_of(args, L);
-      const HeadParamsDev hp = args.hp[args.per_head ? T.h : 0];
+      const HeadParamsDev hp = hp_s[args.per_head ? T.h : 0];
       const uint32_t* lut_h = lut_s + 32 * hp.lut;
       lut_lane = __float_as_int(lane == 0 ? 0.f : __int2float_rn(static_cast<int32_t>(lut_h[lane - 1])));
       const int off = args.Lk - args.Lq;
@@ -368,6 +412,15 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_kernel(const __grid_const
         const float y = fma_rz_sat(__uint_as_float(Cx - sv), Ms32, c1);
         return __float_as_uint(__fmaf_rz(y, 32.0f, 8388608.0f));
       };
+      // the same for two scores, the second multiply-add as one packed instruction
+      auto idx_bits2 = [&](uint32_t s0, uint32_t s1, uint32_t& b0, uint32_t& b1) {
+        const float y0 = fma_rz_sat(__uint_as_float(Cx - s0), Ms32, c1);
+        const float y1 = fma_rz_sat(__uint_as_float(Cx - s1), Ms32, c1);
+        float k0, k1;
+        fma2_rz(y0, y1, pack2(32.0f), pack2(8388608.0f), k0, k1);
+        b0 = __float_as_uint(k0);
+        b1 = __float_as_uint(k1);
+      };
       constexpr uint32_t kMaskedBits = 0x4B000000u;
 
       // ---- pass B: Z = sum of pseudo-exponentials ----
@@ -379,8 +432,12 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_kernel(const __grid_const
         const bool got = walk_s(sc + j, [&](const uint32_t (&v)[32], int c) {
           if (full) {
 #pragma unroll
-            for (int k = 0; k < 32; ++k)
-              z4[k & 3] += __int_as_float(__shfl_sync(0xffffffffu, lut_lane, static_cast<int>(idx_bits(v[k]))));
+            for (int k = 0; k < 32; k += 2) {
+              uint32_t b0, b1;
+              idx_bits2(v[k], v[k + 1], b0, b1);
+              z4[k & 3] += __int_as_float(__shfl_sync(0xffffffffu, lut_lane, static_cast<int>(b0)));
+              z4[(k + 1) & 3] += __int_as_float(__shfl_sync(0xffffffffu, lut_lane, static_cast<int>(b1)));
+            }
           } else {
             const int nc = nv - 32 * c;
 #pragma unroll
@@ -402,18 +459,13 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_kernel(const __grid_const
       // reciprocal and this row's probability table: row k = Ptab[k - 1]
       // (each of the four threads of a row writes 8 of the rows 1..32)
       {
-        // R = floor(N / Z), N = 255 2^32 + floor(Z/2) < 2^40: the double
-        // quotient is within one unit of R, and one integer step makes it exact.
-        const unsigned long long N = (255ull << 32) + static_cast<unsigned long long>(Z >> 1);
-        const unsigned long long Zu = static_cast<unsigned long long>(Z);
-        unsigned long long R =
-            static_cast<unsigned long long>(__ddiv_rn(static_cast<double>(N), static_cast<double>(Z)));
-        if (R * Zu > N) --R;
-        else if ((R + 1) * Zu <= N) ++R;
+        const unsigned long long R = exact_R(Z);
 #pragma unroll
-        for (int i = grp * 8; i < grp * 8 + 8; ++i)
-          ptab[(i + 1) * kBM + r] =
-              static_cast<uint32_t>((static_cast<unsigned long long>(lut_h[i]) * R + (1ull << 31)) >> 32);
+        for (int i = grp * 8; i < grp * 8 + 8; ++i) {
+          const uint32_t P = static_cast<uint32_t>((static_cast<unsigned long long>(lut_h[i]) * R + (1ull << 31)) >> 32);
+#pragma unroll
+          for (int b = 0; b < 4; ++b) ptab[b * (C::kPtabBytes / 4) + (i + 1) * kBM + r] = P << (8 * b);
+        }
       }
       all_sync(true);  // the table is complete
 
@@ -429,10 +481,12 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_kernel(const __grid_const
           if (full) {
 #pragma unroll
             for (int q = 0; q < 8; ++q) {
-              uint32_t p[4];
+              uint32_t kb[4], p[4];
+              idx_bits2(v[q * 4], v[q * 4 + 1], kb[0], kb[1]);
+              idx_bits2(v[q * 4 + 2], v[q * 4 + 3], kb[2], kb[3]);
 #pragma unroll
-              for (int b = 0; b < 4; ++b) p[b] = lds_u32(idx_bits(v[q * 4 + b]) * 512u + prow);
-              pw[q] = pack4(p[0], p[1], p[2], p[3]);
+              for (int b = 0; b < 4; ++b) p[b] = lds_u32(kb[b] * 512u + prow + b * C::kPtabBytes);
+              pw[q] = (p[0] + p[1]) + (p[2] + p[3]);
             }
           } else {
             const int nc = nv - 32 * c;
@@ -443,9 +497,9 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_kernel(const __grid_const
               for (int b = 0; b < 4; ++b) {
                 const int k = q * 4 + b;
                 const uint32_t ib = k < nc ? idx_bits(v[k]) : kMaskedBits;
-                p[b] = lds_u32(ib * 512u + prow);
+                p[b] = lds_u32(ib * 512u + prow + b * C::kPtabBytes);
               }
-              pw[q] = pack4(p[0], p[1], p[2], p[3]);
+              pw[q] = (p[0] + p[1]) + (p[2] + p[3]);
             }
           }
           tmem_st8(tlane + kColP + pb * 32 + half * (kCols / 4) + c * 8, pw);
@@ -470,7 +524,7 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_kernel(const __grid_const
       const int L = tile_index(it, blockIdx.x, gridDim.x);
       if (L >= args.n_tiles) break;
       const Tile T = tile_of(args, L);
-      const HeadParamsDev hp = args.hp[args.per_head ? T.h : 0];
+      const HeadParamsDev hp = hp_s[args.per_head ? T.h : 0];
       const int ob = it % C::kOBufs;
       if (!mbar_wait_warp(bar(kBarOFull + ob), (it / C::kOBufs) & 1, kRoleEpilogue)) break;
       tc_fence_after();

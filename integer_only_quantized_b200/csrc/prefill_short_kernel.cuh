@@ -1,21 +1,20 @@
-// Short-row prefill kernel (rows of at most 512 keys) of the fully-integer
+// Short-row prefill kernel (rows of at most 256 keys) of the fully-integer
 // attention forward for sm_100a: the same definition as prefill_kernel.cuh
-// (IntAttention, arXiv 2511.21513, "Methodology" items 2-3), with the LUT
-// index codes of a row materialised in registers instead of recomputing the
-// scores for the last sweep.
+// (IntAttention, arXiv 2511.21513, "Methodology" items 2-3), with the scores
+// of a whole row tile materialised in tensor memory instead of recomputed.
 //
 // The final row max fixes every LUT index and the final Z fixes every
 // probability, so three sweeps over a row's keys remain (A: max, B: Z,
-// C: P and P.V).  What changes for short rows:
-//   * pass B keeps the index code of every score it visits (one byte per
-//     key, 32 keys of each of at most 4 key tiles per thread: at most 32
-//     registers), so pass C reads codes from registers and needs neither a
-//     third Q.K^T nor the S tiles;
-//   * with at most 2 key tiles (<= 256 keys) both S tiles stay resident in
-//     TMEM from pass A to pass B: Q.K^T runs once per key tile in total;
-//   * the next tile's first Q.K^T goes to the tensor core ahead of this
-//     tile's P.V, as soon as pass B has released the S buffers, so S is ready
-//     when the softmax warps finish pass C.
+// C: P and P.V).  With at most two key tiles, both S tiles of a 128-row
+// tile (256 TMEM columns) stay resident from pass A to pass C: Q.K^T runs
+// once per key tile, and the softmax warps never wait for the tensor core
+// between passes.  Pass C releases each S buffer right after reading it, and
+// the tensor core computes the next tile's scores for that key tile before
+// this tile's P.V of the same key tile, so the next tile's scores are ready
+// when pass C ends.
+// (Kept in shared memory instead, one byte of index code per key costs more
+// to pack and unpack, at 2 cycles per byte permute, than recomputing the
+// index from the resident scores, at 3 full-rate instructions per key.)
 // Work unit and schedule: one (batch, head, 128-query tile), persistent CTAs
 // in snake order over the tiles sorted longest first (causal).
 // Warp roles (22 warps):
@@ -41,19 +40,21 @@
 namespace intattn {
 namespace shortrow {
 
+using prefill::exact_R;
+using prefill::fma2_rz;
 using prefill::fma_rz_sat;
 using prefill::imax;
 using prefill::kBM;
 using prefill::kBN;
+using prefill::pack2;
 using prefill::pack4;
 using prefill::requant_byte;
 using prefill::Tile;
 using prefill::tile_index;
 using prefill::tile_of;
 
-constexpr int kMaxKeyTiles = 4;              // rows of at most 512 keys
+constexpr int kMaxKeyTiles = 2;              // rows of at most 256 keys: both S tiles resident
 constexpr int kMaxKeys = kMaxKeyTiles * kBN;
-constexpr int kResidentTiles = 2;            // key tiles whose S stays in TMEM from pass A to B
 constexpr int kSoftWarps = 16;
 constexpr int kColGroups = 4;                // column groups of an S tile
 constexpr int kCols = kBN / kColGroups;      // 32 S columns per thread and tile
@@ -63,7 +64,7 @@ constexpr int kEpiWarp0 = 18;
 constexpr int kEpiWarps = 4;
 constexpr int kThreads = 32 * (kEpiWarp0 + kEpiWarps);  // 704
 constexpr uint32_t kTmemCols = 512;
-constexpr uint32_t kColS = 0;    // two S buffers: [0,128) and [128,256)
+constexpr uint32_t kColS = 0;    // S of key tile j in [128 j, 128 j + 128)
 constexpr uint32_t kColO = 256;  // O accumulators: d columns each (two for d = 64)
 constexpr uint32_t kColP = 384;  // four P buffers of 32 columns (128 u8 keys each)
 constexpr int kPBufs = 4;
@@ -74,8 +75,8 @@ enum Role : unsigned { kRoleSoftmax = 1, kRoleProducer = 2, kRoleMma = 3, kRoleE
 enum Bar : int {
   kBarQFull = 0,    // [2]
   kBarQEmpty = 2,   // [2]  every Q.K^T that read that Q buffer is done
-  kBarSFull = 4,    // [2]
-  kBarSEmpty = 6,   // [2]  all 16 softmax warps are done with the S tile
+  kBarSFull = 4,    // [2]  per key tile j: S_j written
+  kBarSEmpty = 6,   // [2]  all 16 softmax warps have read S_j for the last time
   kBarPFull = 8,    // [4]
   kBarPEmpty = 12,  // [4]
   kBarOFull = 16,   // [2]
@@ -96,10 +97,13 @@ struct Cfg {
   static constexpr int kNumBars = kBarKvFull + 2 * kStages;
   static constexpr uint32_t kOffQ = 0;
   static constexpr uint32_t kOffKV = kOffQ + 2 * kQBytes;
-  static constexpr uint32_t kOffPtab = kOffKV + kStages * kTileBytes;      // [33][kBM] u32
-  static constexpr uint32_t kOffRed = kOffPtab + 33 * kBM * 4;            // [2][kColGroups][kBM] int32
+  // probability table, four copies [b][33][kBM] u32 holding P << 8b
+  static constexpr uint32_t kPtabBytes = 33 * kBM * 4;
+  static constexpr uint32_t kOffPtab = kOffKV + kStages * kTileBytes;
+  static constexpr uint32_t kOffRed = kOffPtab + 4 * kPtabBytes;             // [2][kColGroups][kBM] int32
   static constexpr uint32_t kOffLut = kOffRed + 2 * kColGroups * kBM * 4;
-  static constexpr uint32_t kOffBars = kOffLut + INTATTN_MAX_CLIPS * 32 * 4;
+  static constexpr uint32_t kOffHp = kOffLut + INTATTN_MAX_CLIPS * 32 * 4;   // head parameters
+  static constexpr uint32_t kOffBars = kOffHp + INTATTN_MAX_HEADS * sizeof(HeadParamsDev);
   static constexpr uint32_t kOffTmem = kOffBars + kNumBars * 8;
   static constexpr uint32_t kUsed = kOffTmem + 16;
   // one CTA per SM (each CTA allocates all 512 TMEM columns)
@@ -107,37 +111,36 @@ struct Cfg {
 };
 
 // The order in which the tensor core consumes K/V tiles (and the producer
-// loads them) for one CTA: for tile t with n key tiles,
-//   Q.K^T of its first min(n, 2) key tiles (pass A), then P.V of tile t-1,
-//   then Q.K^T of its other key tiles (pass A), then, when n > 2, Q.K^T of
-//   all n key tiles again (pass B); after the last tile, its P.V.
-// `qk(tile, j)` and `pv(tile, j)` are called in that order; they return false
-// to stop the walk.
-template <typename QK, typename PV, typename BEGIN>
+// loads them) for one CTA with tiles t = 0, 1, ...:
+//   Q.K^T of tile 0, key tiles 0 .. n0-1;
+//   then for each t: for j = 0, 1: Q.K^T of tile t+1, key tile j (if it
+//   has one), then P.V of tile t, key tile j (if it has one).
+// `begin(t)` is called before the first Q.K^T of tile t; `qk(t, tile, j)`
+// and `pv(t, tile, j)` in the order above; any of them returns false to
+// stop the walk.
+template <typename BEGIN, typename QK, typename PV>
 __device__ __forceinline__ void walk_schedule(const PrefillArgs& a, BEGIN&& begin, QK&& qk, PV&& pv) {
-  Tile prev{};
-  int it = 0;
-  for (;; ++it) {
-    const int L = tile_index(it, blockIdx.x, gridDim.x);
-    if (L >= a.n_tiles) break;
-    const Tile T = tile_of(a, L);
-    if (!begin(it, T)) return;
-    const int lead = T.nkt < kResidentTiles ? T.nkt : kResidentTiles;
-    for (int j = 0; j < lead; ++j)
-      if (!qk(it, T, j)) return;
-    if (it > 0)
-      for (int j = 0; j < prev.nkt; ++j)
-        if (!pv(it - 1, prev, j)) return;
-    for (int j = lead; j < T.nkt; ++j)
-      if (!qk(it, T, j)) return;
-    if (T.nkt > kResidentTiles)
-      for (int j = 0; j < T.nkt; ++j)
-        if (!qk(it, T, j)) return;
-    prev = T;
+  int L = tile_index(0, blockIdx.x, gridDim.x);
+  if (L >= a.n_tiles) return;
+  Tile T = tile_of(a, L);
+  if (!begin(0, T)) return;
+  for (int j = 0; j < T.nkt; ++j)
+    if (!qk(0, T, j)) return;
+  for (int t = 0;; ++t) {
+    const int Ln = tile_index(t + 1, blockIdx.x, gridDim.x);
+    const bool more = Ln < a.n_tiles;
+    Tile Tn{};
+    if (more) {
+      Tn = tile_of(a, Ln);
+      if (!begin(t + 1, Tn)) return;
+    }
+    for (int j = 0; j < kMaxKeyTiles; ++j) {
+      if (more && j < Tn.nkt && !qk(t + 1, Tn, j)) return;
+      if (j < T.nkt && !pv(t, T, j)) return;
+    }
+    if (!more) return;
+    T = Tn;
   }
-  if (it > 0)
-    for (int j = 0; j < prev.nkt; ++j)
-      if (!pv(it - 1, prev, j)) return;
 }
 
 template <int D>
@@ -150,6 +153,7 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_short_kernel(const __grid
   uint32_t* ptab = reinterpret_cast<uint32_t*>(smem + C::kOffPtab);
   int32_t* red = reinterpret_cast<int32_t*>(smem + C::kOffRed);
   uint32_t* lut_s = reinterpret_cast<uint32_t*>(smem + C::kOffLut);
+  HeadParamsDev* hp_s = reinterpret_cast<HeadParamsDev*>(smem + C::kOffHp);
   const uint32_t bars = s_base + C::kOffBars;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::kOffTmem);
   auto bar = [&](int i) { return bars + 8u * static_cast<uint32_t>(i); };
@@ -184,6 +188,9 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_short_kernel(const __grid
     mbar_fence_init();
   }
   for (int i = tid; i < args.n_luts * 32; i += blockDim.x) lut_s[i] = args.lut[i >> 5][i & 31];
+  // head parameters in shared memory: a dynamically indexed kernel argument
+  // is a constant-bank load that can miss
+  for (int i = tid; i < (args.per_head ? args.H : 1); i += blockDim.x) hp_s[i] = args.hp[i];
   if (warp == kMmaWarp) {
     tmem_alloc(smem_u32(tmem_slot), kTmemCols);
     tmem_relinquish();
@@ -199,32 +206,27 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_short_kernel(const __grid
     const int g = warp >> 2;                 // column group: columns 32g .. 32g+31 of each S tile
     const int r = quad * 32 + lane;          // query row within the tile == TMEM lane
     const uint32_t tlane = tmem + (static_cast<uint32_t>(quad * 32) << 16);
-    const uint32_t trow = tlane + g * kCols;
-    const uint32_t prow = smem_u32(ptab) + 4u * r;  // row k of the table at prow + 512 k
-    if (g == 0) ptab[r] = 0u;                        // table row 0 (masked keys) stays 0
+    const uint32_t trow = tlane + kColS + g * kCols;
+    const uint32_t prow = smem_u32(ptab) + 4u * r;  // row k of copy b at prow + 512 k + b kPtabBytes
+    if (g == 0)
+      for (int b = 0; b < 4; ++b) ptab[b * (C::kPtabBytes / 4) + r] = 0u;  // row 0 (masked keys) stays 0
     bool ok = true;
-    uint32_t sc = 0;  // S fills consumed so far (the MMA warp counts the same way)
-    uint32_t pc = 0;  // P tiles written so far
+    uint32_t sfill[kMaxKeyTiles] = {0, 0};  // fills of each S buffer consumed so far
+    uint32_t pc = 0;                        // P tiles written so far
     auto quad_sync = [&](bool mine) { return bar_red_and(kNbQuad0 + quad, 128, mine); };
     auto arrive_warp = [&](uint32_t b) {
       __syncwarp();
       if (lane == 0) mbar_arrive(b);
     };
-    auto s_buf = [&](uint32_t fill) { return kColS + (fill & 1u) * kBN; };
-    auto wait_s = [&](uint32_t fill) {
-      return mbar_wait_warp(bar(kBarSFull + (fill & 1u)), (fill >> 1) & 1u, kRoleSoftmax);
-    };
-    auto release_s = [&](uint32_t fill) {
-      tc_fence_before();
-      arrive_warp(bar(kBarSEmpty + (fill & 1u)));
-    };
     constexpr uint32_t kMaskedBits = 0x4B000000u;
+    const unsigned long long k32x2 = pack2(32.0f), k2p23x2 = pack2(8388608.0f);
 
-    for (int it = 0;; ++it) {
-      const int L = tile_index(it, blockIdx.x, gridDim.x);
-      if (L >= args.n_tiles) break;
-      const Tile T = tile_of(args, L);
-      const HeadParamsDev hp = args.hp[args.per_head ? T.h : 0];
+    int L = tile_index(0, blockIdx.x, gridDim.x);
+    Tile T = L < args.n_tiles ? tile_of(args, L) : Tile{};
+    for (int it = 0; L < args.n_tiles; ++it) {
+      const int Ln = tile_index(it + 1, blockIdx.x, gridDim.x);
+      const Tile Tn = Ln < args.n_tiles ? tile_of(args, Ln) : Tile{};
+      const HeadParamsDev hp = hp_s[args.per_head ? T.h : 0];
       const uint32_t* lut_h = lut_s + 32 * hp.lut;
       const int32_t lut_lane =
           __float_as_int(lane == 0 ? 0.f : __int2float_rn(static_cast<int32_t>(lut_h[lane - 1])));
@@ -232,21 +234,25 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_short_kernel(const __grid
       const int key_lim = args.causal ? min(args.Lk, T.q0 + r + off + 1) : args.Lk;
       // valid keys of this thread's 32 columns of key tile j: a prefix
       auto nvalid = [&](int j) { return min(max(key_lim - (j * kBN + g * kCols), 0), kCols); };
-      const bool resident = T.nkt <= kResidentTiles;
+      // a warp whose 32 rows are all past the last query row skips the
+      // arithmetic (its four quadrant warps skip together); it still takes
+      // part in every barrier and hand-off
+      const bool rows_live = T.q0 + quad * 32 < args.Lq;
+      // work of this warp on key tile j: live rows and at least one valid key
+      auto live = [&](int j) { return rows_live && __any_sync(0xffffffffu, nvalid(j) > 0); };
 
       // ---- pass A: row max over valid keys ----
       int32_t m = INT_MIN;
 #pragma unroll
       for (int j = 0; j < kMaxKeyTiles; ++j) {
         if (j >= T.nkt || !ok) break;
-        const uint32_t fill = sc + j;
-        if (!wait_s(fill)) { ok = false; break; }
+        if (!mbar_wait_warp(bar(kBarSFull + j), sfill[j] & 1u, kRoleSoftmax)) { ok = false; break; }
         tc_fence_after();
+        if (!live(j)) continue;
         const int nv = nvalid(j);
         uint32_t v[32];
-        tmem_ld32(trow + s_buf(fill), v);
+        tmem_ld32(trow + j * kBN, v);
         tmem_wait_ld();
-        if (!resident) release_s(fill);
         if (nv == kCols) {
           int32_t m4[4] = {INT_MIN, INT_MIN, INT_MIN, INT_MIN};
 #pragma unroll
@@ -262,7 +268,6 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_short_kernel(const __grid
           for (int k = 0; k < 32; ++k) m = imax(m, k < nv ? static_cast<int32_t>(v[k]) : INT_MIN);
         }
       }
-      if (!resident) sc += T.nkt;
       red[g * kBM + r] = m;
       // also carries a failure of the previous tile's pass C to the whole quadrant
       if (!quad_sync(ok)) { ok = false; break; }
@@ -270,73 +275,73 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_short_kernel(const __grid
 
       // LUT index code of a score on the FP32 pipe (see prefill_kernel.cuh):
       // the bits 0x4B000000 + k, k = idx + 1 for idx <= 30 and k = 32 for a
-      // clipped gap; the low byte is k, the low 5 bits the shuffle lane.
+      // clipped gap; the low 5 bits are the shuffle lane, k the table row.
+      // The second multiply-add of two scores is one packed instruction.
       const uint32_t Cx = 0x4B000000u + static_cast<uint32_t>(m);
       const float Mf = __int2float_rn(hp.M);
       const float Ms32 = Mf * __uint_as_float(static_cast<uint32_t>(127 - 5 - hp.s) << 23);
       const float c1 = (1.5f - Mf * __uint_as_float(static_cast<uint32_t>(127 + 23 - hp.s) << 23)) * 0.03125f;
-      auto idx_bits = [&](uint32_t sv) {
-        const float y = fma_rz_sat(__uint_as_float(Cx - sv), Ms32, c1);
-        return __float_as_uint(__fmaf_rz(y, 32.0f, 8388608.0f));
+      auto idx_bits2 = [&](uint32_t s0, uint32_t s1, uint32_t& b0, uint32_t& b1) {
+        const float y0 = fma_rz_sat(__uint_as_float(Cx - s0), Ms32, c1);
+        const float y1 = fma_rz_sat(__uint_as_float(Cx - s1), Ms32, c1);
+        float k0, k1;
+        fma2_rz(y0, y1, k32x2, k2p23x2, k0, k1);
+        b0 = __float_as_uint(k0);
+        b1 = __float_as_uint(k1);
+      };
+      // codes of 4 scores v[o .. o+3] of this thread's columns, masked past nv
+      auto codes4 = [&](const uint32_t* v, int o, int nv, bool full, uint32_t (&kb)[4]) {
+        idx_bits2(v[0], v[1], kb[0], kb[1]);
+        idx_bits2(v[2], v[3], kb[2], kb[3]);
+        if (!full) {
+#pragma unroll
+          for (int b = 0; b < 4; ++b)
+            if (o + b >= nv) kb[b] = kMaskedBits;
+        }
       };
 
-      // ---- pass B: Z, and the code of every key kept in registers ----
-      uint32_t codes[kMaxKeyTiles][8];
-      float zf = 0.f;
+      // ---- pass B: Z = sum of pseudo-exponentials ----
+      float z4[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
       for (int j = 0; j < kMaxKeyTiles; ++j) {
         if (j >= T.nkt || !ok) break;
-        const uint32_t fill = sc + j;
-        if (!resident) {
-          if (!wait_s(fill)) { ok = false; break; }
-          tc_fence_after();
-        }
+        if (!live(j)) continue;
         const int nv = nvalid(j);
-        float z4[4] = {0.f, 0.f, 0.f, 0.f};
-        // two halves of 16 columns: fewer scores live next to the codes
+        const bool full = nv == kCols;
 #pragma unroll
         for (int h = 0; h < 2; ++h) {
           uint32_t v[16];
-          tmem_ld16(trow + s_buf(fill) + 16 * h, v);
+          tmem_ld16(trow + j * kBN + 16 * h, v);
           tmem_wait_ld();
-          if (h == 1) release_s(fill);
-          const bool full = nv == kCols;
 #pragma unroll
           for (int q = 0; q < 4; ++q) {
             uint32_t kb[4];
+            codes4(v + 4 * q, 16 * h + 4 * q, nv, full, kb);
 #pragma unroll
-            for (int b = 0; b < 4; ++b) {
-              const int k = 4 * q + b;
-              kb[b] = (full || 16 * h + k < nv) ? idx_bits(v[k]) : kMaskedBits;
+            for (int b = 0; b < 4; ++b)
               z4[b] += __int_as_float(__shfl_sync(0xffffffffu, lut_lane, static_cast<int>(kb[b])));
-            }
-            codes[j][4 * h + q] = pack4(kb[0], kb[1], kb[2], kb[3]);
           }
         }
-        zf += (z4[0] + z4[1]) + (z4[2] + z4[3]);  // exact: below 2^24
       }
-      sc += T.nkt;
-      red[(kColGroups + g) * kBM + r] = __float2int_rn(zf);
+      // exact: each partial is below 2^24
+      red[(kColGroups + g) * kBM + r] = __float2int_rn((z4[0] + z4[1]) + (z4[2] + z4[3]));
       if (!quad_sync(ok)) { ok = false; break; }
-      const int32_t Z = (red[kColGroups * kBM + r] + red[(kColGroups + 1) * kBM + r]) +
-                        (red[(kColGroups + 2) * kBM + r] + red[(kColGroups + 3) * kBM + r]);
-      {
-        // R = floor(N / Z), N = 255 2^32 + floor(Z/2): the double quotient is
-        // within one unit of R; one integer step makes it exact
-        const unsigned long long N = (255ull << 32) + static_cast<unsigned long long>(Z >> 1);
-        const unsigned long long Zu = static_cast<unsigned long long>(Z);
-        unsigned long long R =
-            static_cast<unsigned long long>(__ddiv_rn(static_cast<double>(N), static_cast<double>(Z)));
-        if (R * Zu > N) --R;
-        else if ((R + 1) * Zu <= N) ++R;
+      if (rows_live) {
+        // rows past the last query row of a live warp read zero-filled Q:
+        // all their scores are 0, so Z >= 2^15 there too
+        const int32_t Z = (red[kColGroups * kBM + r] + red[(kColGroups + 1) * kBM + r]) +
+                          (red[(kColGroups + 2) * kBM + r] + red[(kColGroups + 3) * kBM + r]);
+        const unsigned long long R = exact_R(Z);
 #pragma unroll
-        for (int i = g * 8; i < g * 8 + 8; ++i)
-          ptab[(i + 1) * kBM + r] =
-              static_cast<uint32_t>((static_cast<unsigned long long>(lut_h[i]) * R + (1ull << 31)) >> 32);
+        for (int i = g * 8; i < g * 8 + 8; ++i) {
+          const uint32_t P = static_cast<uint32_t>((static_cast<unsigned long long>(lut_h[i]) * R + (1ull << 31)) >> 32);
+#pragma unroll
+          for (int b = 0; b < 4; ++b) ptab[b * (C::kPtabBytes / 4) + (i + 1) * kBM + r] = P << (8 * b);
+        }
       }
       if (!quad_sync(ok)) { ok = false; break; }  // this quadrant's table rows are complete
 
-      // ---- pass C: P from the codes into TMEM for the P.V MMAs ----
+      // ---- pass C: P into TMEM for the P.V MMAs; each S buffer released after its last read ----
 #pragma unroll
       for (int j = 0; j < kMaxKeyTiles; ++j) {
         if (j >= T.nkt || !ok) break;
@@ -344,20 +349,44 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_short_kernel(const __grid
         const uint32_t pb = pi & (kPBufs - 1);
         if (!mbar_wait_warp(bar(kBarPEmpty + pb), ((pi / kPBufs) & 1) ^ 1, kRoleSoftmax)) { ok = false; break; }
         uint32_t pw[8];
+        if (live(j)) {
+          const int nv = nvalid(j);
+          const bool full = nv == kCols;
 #pragma unroll
-        for (int q = 0; q < 8; ++q) {
-          const uint32_t w = codes[j][q];
-          uint32_t p[4];
+          for (int h = 0; h < 2; ++h) {
+            uint32_t v[16];
+            tmem_ld16(trow + j * kBN + 16 * h, v);
+            tmem_wait_ld();
+            if (h == 1) {  // the last read of S_j
+              tc_fence_before();
+              arrive_warp(bar(kBarSEmpty + j));
+            }
 #pragma unroll
-          for (int b = 0; b < 4; ++b) p[b] = lds_u32(__byte_perm(w, 0u, 0x4440u + b) * 512u + prow);
-          pw[q] = pack4(p[0], p[1], p[2], p[3]);
+            for (int q = 0; q < 4; ++q) {
+              uint32_t kb[4], p[4];
+              codes4(v + 4 * q, 16 * h + 4 * q, nv, full, kb);
+#pragma unroll
+              for (int b = 0; b < 4; ++b) p[b] = lds_u32(kb[b] * 512u + prow + b * C::kPtabBytes);
+              pw[4 * h + q] = (p[0] + p[1]) + (p[2] + p[3]);
+            }
+          }
+        } else {
+          tc_fence_before();
+          arrive_warp(bar(kBarSEmpty + j));
+#pragma unroll
+          for (int q = 0; q < 8; ++q) pw[q] = 0u;  // masked columns: the P.V reads zeros there
         }
-        tmem_st8(tlane + kColP + pb * 32 + g * (kCols / 4), pw);
-        tmem_wait_st();
+        if (rows_live) {  // rows past the last query row: their P is never used
+          tmem_st8(tlane + kColP + pb * 32 + g * (kCols / 4), pw);
+          tmem_wait_st();
+        }
         tc_fence_before();
         arrive_warp(bar(kBarPFull + pb));
+        ++sfill[j];
       }
       pc += T.nkt;
+      L = Ln;
+      T = Tn;
     }
   } else if (warp >= kEpiWarp0) {
     // ============================ epilogue ============================
@@ -368,7 +397,7 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_short_kernel(const __grid
       const int L = tile_index(it, blockIdx.x, gridDim.x);
       if (L >= args.n_tiles) break;
       const Tile T = tile_of(args, L);
-      const HeadParamsDev hp = args.hp[args.per_head ? T.h : 0];
+      const HeadParamsDev hp = hp_s[args.per_head ? T.h : 0];
       const int ob = it % C::kOBufs;
       if (!mbar_wait_warp(bar(kBarOFull + ob), (it / C::kOBufs) & 1, kRoleEpilogue)) break;
       tc_fence_after();
@@ -455,40 +484,38 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_short_kernel(const __grid
     const uint64_t kv_desc0 = smem_desc(sKV, 16, C::kSBO, C::kSwizzle);
     constexpr uint32_t kSlotDesc = C::kTileBytes >> 4;
     uint32_t slot = 0, kv_par = 0;
-    uint32_t sc = 0;   // S fills issued
-    uint32_t pc = 0;   // P tiles consumed
-    int qk_left = 0;   // Q.K^T of the current tile still to issue
-    uint32_t qb = 0;
+    uint32_t sfill0 = 0, sfill1 = 0;  // fills of each S buffer issued (two scalars: j is not a constant here)
+    uint32_t pc = 0;                  // P tiles consumed
     auto next_slot = [&]() {
       if (++slot == static_cast<uint32_t>(C::kStages)) {
         slot = 0;
         kv_par ^= 1;
       }
     };
-    auto begin = [&](int it, const Tile& T) {
-      qb = static_cast<uint32_t>(it & 1);
-      qk_left = T.nkt > kResidentTiles ? 2 * T.nkt : T.nkt;
-      return mbar_wait_warp(bar(kBarQFull + qb), (it >> 1) & 1, kRoleMma);
+    auto begin = [&](int t, const Tile&) {
+      return mbar_wait_warp(bar(kBarQFull + (t & 1)), (t >> 1) & 1, kRoleMma);
     };
-    auto qk = [&](int, const Tile&, int) {
-      const uint32_t buf = sc & 1;
-      if (!mbar_wait2_warp(bar(kBarSEmpty + buf), ((sc >> 1) & 1) ^ 1, bar_kv_full(slot), kv_par, kRoleMma))
+    auto qk = [&](int t, const Tile& T, int j) {
+      // S_j free: all softmax warps have read the previous fill of this buffer
+      const uint32_t fills = j ? sfill1 : sfill0;
+      if (!mbar_wait2_warp(bar(kBarSEmpty + j), (fills & 1) ^ 1, bar_kv_full(slot), kv_par, kRoleMma))
         return false;
       tc_fence_after();
+      const uint32_t qb = static_cast<uint32_t>(t & 1);
       const uint64_t q_desc = smem_desc(sQ(qb), 16, C::kSBO, C::kSwizzle);
       const uint64_t k_desc = kv_desc0 + slot * kSlotDesc;
       if (elect_one()) {
 #pragma unroll
         for (int kk = 0; kk < D / 32; ++kk)
-          mma_i8_ss(tmem + kColS + buf * kBN, q_desc + 2 * kk, k_desc + 2 * kk, idesc_qk, kk > 0);
+          mma_i8_ss(tmem + kColS + j * kBN, q_desc + 2 * kk, k_desc + 2 * kk, idesc_qk, kk > 0);
         mma_commit(bar_kv_empty(slot));
-        mma_commit(bar(kBarSFull + buf));
-        if (qk_left == 1) mma_commit(bar(kBarQEmpty + qb));  // the tile's last read of its Q buffer
+        mma_commit(bar(kBarSFull + j));
+        if (j == T.nkt - 1) mma_commit(bar(kBarQEmpty + qb));  // the tile's last read of its Q buffer
       }
       __syncwarp();
       next_slot();
-      ++sc;
-      --qk_left;
+      if (j) ++sfill1;
+      else ++sfill0;
       return true;
     };
     auto pv = [&](int t, const Tile& T, int j) {

@@ -241,6 +241,8 @@ SHORT_SWEEP = [
     (1, 2, 100, 512, 64, True, False, "normal"),     # Lq < Lk, bottom-right causal
     (1, 2, 600, 200, 128, False, True, "normal"),    # cross attention, more queries than keys
     (8, 40, 512, 512, 64, True, True, "normal"),     # 1280 tiles: CTAs mix 1..4 key tiles
+    (8, 40, 256, 256, 128, True, True, "normal"),    # 640 tiles: CTAs mix 1 and 2 key tiles
+    (4, 30, 250, 250, 64, True, False, "normal"),    # causal, ragged: the second q tile has 122 rows
     (24, 12, 197, 197, 64, False, True, "student_t4"),  # 576 tiles: several rounds of resident tiles
 ]
 
@@ -248,25 +250,29 @@ SHORT_SWEEP = [
 @pytest.mark.parametrize("case", SHORT_SWEEP, ids=lambda c: "B{}H{}Lq{}Lk{}d{}{}{}".format(
     c[0], c[1], c[2], c[3], c[4], "c" if c[5] else "", "h" if c[6] else ""))
 def test_short_row_variants_match_oracle(ia, oracle_mod, case):
-    """Both kernels on rows of at most 512 keys: the short-row kernel (codes
-    kept in registers, resident scores up to 256 keys) and the three-pass
-    kernel must each give the oracle's bytes."""
+    """Rows of at most 512 keys: the short-row kernel (scores resident in
+    tensor memory, up to 256 keys), the three-pass kernel and the automatic
+    choice must each give the oracle's bytes."""
     B, H, Lq, Lk, d, causal, per_head, dist = case
     w = wl.custom_workload("short", B, H, Lq, Lk, d, causal, per_head=per_head, dist=dist,
                            clip_c=8.0 if d == 64 else 10.0, index=2000 + Lq + 3 * Lk + d + B)
     x = wl.make_inputs(w)
     want = _oracle_forward(oracle_mod, x, w)
-    for variant in (ia.VARIANT_SHORT_ROWS, ia.VARIANT_THREE_PASS):
+    variants = [ia.VARIANT_AUTO, ia.VARIANT_THREE_PASS]
+    if Lk <= ia.SHORT_ROWS_MAX_KEYS:
+        variants.append(ia.VARIANT_SHORT_ROWS)
+    for variant in variants:
         _assert_equal(_variant_forward(ia, x, w, variant), want, f"{case} variant {variant}")
 
 
 @pytest.mark.parametrize("name", ["bert_base_l128", "bert_base_b8_l512", "vit_b16_l197"])
 def test_workload_both_variants(ia, oracle_mod, name):
-    """The short-row workloads through each kernel explicitly."""
+    """The short-row workloads through each kernel that takes them."""
     w = wl.WORKLOADS[name]
     x = wl.make_inputs(w)
     want = _oracle_forward(oracle_mod, x, w)
-    for variant in (ia.VARIANT_SHORT_ROWS, ia.VARIANT_THREE_PASS):
+    variants = [ia.VARIANT_THREE_PASS] + ([ia.VARIANT_SHORT_ROWS] if w.Lk <= ia.SHORT_ROWS_MAX_KEYS else [])
+    for variant in variants:
         _assert_equal(_variant_forward(ia, x, w, variant, guard=4096), want, f"{name} variant {variant}")
 
 
@@ -274,7 +280,7 @@ def test_workload_both_variants(ia, oracle_mod, name):
 def test_short_rows_extreme_codes(ia, oracle_mod, d):
     """Largest |S| and all-equal rows through the short-row kernel."""
     import dataclasses
-    w = wl.custom_workload("short_extreme", 2, 3, 300, 300, d, True, index=2700 + d)
+    w = wl.custom_workload("short_extreme", 2, 3, 250, 250, d, True, index=2700 + d)
     x = wl.make_inputs(w)
     cases = [dataclasses.replace(x, q=np.full_like(x.q, -128), k=np.full_like(x.k, -128)),
              dataclasses.replace(x, q=np.zeros_like(x.q))]
