@@ -49,7 +49,7 @@ def parse_args(argv=None):
     p.add_argument("--no-decode", action="store_true")
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--cpu-seconds", type=float, default=12.0)
-    p.add_argument("--leg", choices=["decode", "decode_int4", "quantize", "gelu"], default=None,
+    p.add_argument("--leg", choices=["decode", "decode_int4", "quantize", "gelu", "forward_fp"], default=None,
                    help="run only this secondary leg and print its object (for profiler captures)")
     return p.parse_args(argv)
 
@@ -280,6 +280,8 @@ def run_leg(args):
         out = run_decode(args, dev, stream, world, peaks, peak_src, "llama7b_decode_int4_b64_lk4096")
     elif args.leg == "quantize":
         out = run_quantize(args, dev, stream, world, peaks, peak_src)
+    elif args.leg == "forward_fp":
+        out = run_forward_fp(args, dev, stream, world, peaks, peak_src)
     else:
         out = run_gelu(args, dev, stream, world, peaks, peak_src)
     if rank == 0:
@@ -365,6 +367,7 @@ def run_ours(args):
         line["decode_int4"] = run_decode(args, dev, stream, world, peaks, peak_src,
                                          "llama7b_decode_int4_b64_lk4096")
         line["quantize"] = run_quantize(args, dev, stream, world, peaks, peak_src)
+        line["forward_fp"] = run_forward_fp(args, dev, stream, world, peaks, peak_src)
         line["gelu"] = run_gelu(args, dev, stream, world, peaks, peak_src)
     if not args.no_cpu_baseline and rank == 0 and world == 1:
         line["cpu_baseline"] = cpu_baseline(w, x, args.cpu_seconds)
@@ -451,6 +454,51 @@ def run_quantize(args, dev, stream, world, peaks, peak_src):
                          "frac": round(gbs / peaks["hbm_gbs"], 4), "peak_source": f"{peak_src} hbm_gbs",
                          "traffic": kernel_traffic("quant_fused_kernel", "llama7b_layer_bf16_b1h32l8192d128")},
             "l2": "inputs rotate over 3 copies (201 MB > 126 MB L2)"}
+
+
+def run_forward_fp(args, dev, stream, world, peaks, peak_src):
+    """The forward from bf16 activations (intattn_forward_fp) on the
+    LLaMA-7B causal prefill shape: quantise q, k, v on the device, derive the
+    head parameters on the device, integer forward; every launch of a call
+    is inside the timed region."""
+    import numpy as np
+    import torch
+
+    import integer_only_quantized_b200 as ia
+    from integer_only_quantized_b200 import workloads as wl
+    w = wl.WORKLOADS["llama7b_causal_l8192"]
+    g = torch.Generator(device=dev)
+    g.manual_seed(20251126)
+    shape = (w.B, w.H, w.Lq, w.d)
+    sets = [tuple(torch.randn(shape, generator=g, device=dev, dtype=torch.float32).to(torch.bfloat16)
+                  for _ in range(3)) for _ in range(2)]  # two sets: 2 x 100.7 MB > L2
+    out = torch.empty(shape, dtype=torch.int8, device=dev)
+    ws = torch.empty(ia.forward_fp_workspace_size(w.B, w.H, w.Lq, w.Lk, w.d), dtype=torch.uint8, device=dev)
+    s_o = np.full(w.H, 0.02, np.float32)
+    call = lambda i: ia.forward_fp(*sets[i % 2], True, s_o, w.causal, w.clip_c, out=out, workspace=ws, stream=stream)
+    steps = max(10, min(args.steps, 40))
+    for i in range(max(3, args.warmup)):
+        call(i)
+    torch.cuda.synchronize(dev)
+    barrier(world, dev)
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    t0.record(stream)
+    for i in range(steps):
+        call(i)
+    t1.record(stream)
+    torch.cuda.synchronize(dev)
+    barrier(world, dev)
+    ms = max_over_ranks(t0.elapsed_time(t1) / steps, world, dev)
+    if ia.device_error(stream) != ia.OK:
+        raise RuntimeError("a kernel wait timed out, or a parameter was out of range, in forward_fp")
+    peak_int8, _ = _int8_peak(peaks, sustained=False)
+    tops = w.effective_ops / (ms * 1e-3) / 1e12
+    return {"workload": w.name + "_bf16_inputs", "value": round(aggregate_value(w.effective_ops, world, ms * 1e-3) / 1e12, 3),
+            "unit": "TOPS", "ms_per_call": round(ms, 5), "launches_per_call": 8,
+            "note": "bf16 q, k, v -> int8 out: three quantisations (2 launches each), device-side parameters, forward",
+            "roofline": {"bound": "tensor", "achieved": round(tops, 3), "peak": round(peak_int8, 1), "unit": "TOPS",
+                         "frac": round(tops / peak_int8, 4)},
+            "l2": "inputs alternate between 2 sets (201 MB > 126 MB L2)"}
 
 
 def run_gelu(args, dev, stream, world, peaks, peak_src):

@@ -222,6 +222,42 @@ enum { INTATTN_DTYPE_FP16 = 0, INTATTN_DTYPE_BF16 = 1 };
 int intattn_quantize(const void *x, int dtype, int B, int H, int L, int d, int per_head, int8_t *out,
                      float *scales, intattn_stream_t stream);
 
+/* Bytes of device workspace intattn_forward_fp needs for these sizes (0 for
+ * invalid sizes): int8 copies of q, k and v, three scale arrays, the head
+ * parameters and a status word. */
+size_t intattn_forward_fp_workspace_size(int B, int H, int Lq, int Lk, int d);
+
+/* The forward from fp16 / bf16 activations, with no host round trip: the
+ * quantisation prologue above (the forum page's 动态量化策略: each tensor's, or
+ * each head's, scale taken from the live activations) runs on q, k and v into
+ * the workspace; a one-CTA kernel derives every head's integer parameters on
+ * the device from those scales, in the same IEEE double steps as
+ * intattn_derive_params (so they are identical); the integer forward then
+ * reads them from device memory.  The result equals quantising each tensor
+ * with intattn_quantize and calling intattn_forward with the resulting scales.
+ *   q [B, H, Lq, d], k, v [B, H, Lk, d]: device, dtype INTATTN_DTYPE_FP16 or
+ *   INTATTN_DTYPE_BF16, 16-byte aligned, finite values.
+ *   per_head: scales per head (1) or per tensor (0), for q, k and v alike.
+ *   s_o: HOST, the output scale (H entries per head, or 1).
+ *   clip: HOST per-entry clip thresholds in the layout of s_o, or NULL for
+ *   clip_c everywhere (at most INTATTN_MAX_CLIPS distinct values).
+ *   out [B, H, Lq, d] int8, device.
+ *   scales_out: NULL, or DEVICE floats receiving s_q, s_k, s_v (each H or 1
+ *   entries, in that order) for the caller's own use.
+ *   workspace: device, 256-byte aligned, at least
+ *   intattn_forward_fp_workspace_size bytes; calls that share it must be
+ *   ordered on one stream.
+ * A derived parameter out of range (see intattn_derive_params) cannot be
+ * reported by the return code, since the scales are only known on the
+ * device: the forward then writes nothing, and intattn_device_error returns
+ * INTATTN_ERR_PARAM_RANGE.  Launches: 2 per tensor (quantisation), 1
+ * (parameters), 1 (forward).  Return codes as intattn_forward, plus
+ * INTATTN_ERR_WORKSPACE. */
+int intattn_forward_fp(const void *q, const void *k, const void *v, int dtype, int per_head,
+                       const float *s_o, const float *clip, float clip_c, int B, int H, int Lq, int Lk,
+                       int d, int causal, int8_t *out, float *scales_out, void *workspace,
+                       size_t workspace_bytes, intattn_stream_t stream);
+
 /* Integer GELU (the summary page "[Paper] IntAttention：全整数注意力流水线用于
  * 高效边缘推理", section 局限性与未来工作, names GELU as the next operator for the
  * method; this definition is the library's reading of "the same machinery":
@@ -286,8 +322,10 @@ int intattn_decode_static_scratch(const int8_t *q, const int8_t *k_cache, const 
 int intattn_selftest_timeout(intattn_stream_t stream);
 
 /* Synchronises `stream`, then returns and clears the device error word that a
- * kernel sets when one of its bounded waits runs out (INTATTN_ERR_TIMEOUT), or
- * INTATTN_OK.  INTATTN_ERR_CUDA if the synchronisation itself fails. */
+ * kernel sets when one of its bounded waits runs out (INTATTN_ERR_TIMEOUT) or
+ * when parameters derived on the device are out of range
+ * (INTATTN_ERR_PARAM_RANGE, see intattn_forward_fp), or INTATTN_OK.
+ * INTATTN_ERR_CUDA if the synchronisation itself fails. */
 int intattn_device_error(intattn_stream_t stream);
 
 /* Static description of a return code. */

@@ -23,7 +23,7 @@ MAX_CLIPS = 8
 
 # every function declared in include/intattn.h
 EXPORTED = ("intattn_derive_params", "intattn_forward", "intattn_forward_variant",
-            "intattn_forward_host_workspace_size",
+            "intattn_forward_host_workspace_size", "intattn_forward_fp_workspace_size", "intattn_forward_fp",
             "intattn_forward_host", "intattn_decode_workspace_size",
             "intattn_decode", "intattn_decode_int4", "intattn_decode_static_scratch", "intattn_quantize",
             "intattn_gelu_derive_params", "intattn_gelu", "intattn_selftest_timeout", "intattn_device_error",
@@ -104,6 +104,11 @@ def lib() -> ctypes.CDLL:
                                       i32, f32, vp, vp]
         L.intattn_forward_variant.argtypes = [vp, vp, vp, ctypes.POINTER(_Scales), i32, i32, i32, i32, i32,
                                               i32, f32, vp, i32, vp]
+        L.intattn_forward_fp_workspace_size.argtypes = [i32, i32, i32, i32, i32]
+        L.intattn_forward_fp_workspace_size.restype = ctypes.c_size_t
+        f32p = ctypes.POINTER(ctypes.c_float)
+        L.intattn_forward_fp.argtypes = [vp, vp, vp, i32, i32, f32p, f32p, f32, i32, i32, i32, i32, i32, i32,
+                                         vp, vp, vp, ctypes.c_size_t, vp]
         L.intattn_forward_host_workspace_size.argtypes = [i32, i32, i32, i32, i32]
         L.intattn_forward_host_workspace_size.restype = ctypes.c_size_t
         L.intattn_forward_host.argtypes = [vp, vp, vp, ctypes.POINTER(_Scales), i32, i32, i32, i32, i32,
@@ -225,6 +230,44 @@ def forward_host(q, k, v, scales: Scales, causal: bool, clip_c: float, out=None,
                                     workspace.numel(), _stream_handle(stream, dev))
     del keep
     _check(rc, "intattn_forward_host")
+    return out
+
+
+def forward_fp_workspace_size(B: int, H: int, Lq: int, Lk: int, d: int) -> int:
+    return int(lib().intattn_forward_fp_workspace_size(B, H, Lq, Lk, d))
+
+
+def forward_fp(q, k, v, per_head: bool, s_o, causal: bool, clip_c: float, clip=None, out=None, scales_out=None,
+               workspace=None, stream=None):
+    """intattn_forward_fp: fp16 / bf16 q [B,H,Lq,d], k, v [B,H,Lk,d] (CUDA)
+    -> int8 out, quantising on the device.  s_o (and clip, optional): host
+    floats, H entries per head or 1."""
+    import torch
+    dt = {torch.float16: DTYPE_FP16, torch.bfloat16: DTYPE_BF16}
+    for t, n in ((q, "q"), (k, "k"), (v, "v")):
+        if not isinstance(t, torch.Tensor) or not t.is_cuda or t.dtype not in dt or not t.is_contiguous():
+            raise TypeError(f"{n} must be a contiguous CUDA fp16 / bf16 tensor")
+    if not (q.dtype == k.dtype == v.dtype):
+        raise TypeError("q, k and v must have one dtype")
+    B, H, Lq, d = q.shape
+    Lk = k.shape[2]
+    if k.shape != (B, H, Lk, d) or v.shape != k.shape:
+        raise ValueError("k and v must be [B, H, Lk, d] matching q")
+    if out is None:
+        out = torch.empty((B, H, Lq, d), dtype=torch.int8, device=q.device)
+    _check_tensor(out, "out")
+    so = np.ascontiguousarray(np.atleast_1d(np.asarray(s_o, dtype=np.float32)))
+    cl = None if clip is None else np.ascontiguousarray(np.atleast_1d(np.asarray(clip, dtype=np.float32)))
+    need = forward_fp_workspace_size(B, H, Lq, Lk, d)
+    if workspace is None:
+        workspace = torch.empty(max(need, 1), dtype=torch.uint8, device=q.device)
+    f32p = ctypes.POINTER(ctypes.c_float)
+    rc = lib().intattn_forward_fp(q.data_ptr(), k.data_ptr(), v.data_ptr(), dt[q.dtype], int(bool(per_head)),
+                                  so.ctypes.data_as(f32p), None if cl is None else cl.ctypes.data_as(f32p),
+                                  float(clip_c), B, H, Lq, Lk, d, int(bool(causal)), out.data_ptr(),
+                                  None if scales_out is None else scales_out.data_ptr(), workspace.data_ptr(),
+                                  workspace.numel(), _stream_handle(stream, q.device))
+    _check(rc, "intattn_forward_fp")
     return out
 
 

@@ -19,6 +19,7 @@
 
 #include "decode_kernel.cuh"
 #include "gelu_kernel.cuh"
+#include "params_kernel.cuh"
 #include "quantize_kernel.cuh"
 #include "prefill_kernel.cuh"
 #include "prefill_short_kernel.cuh"
@@ -380,22 +381,14 @@ int intattn_forward(const int8_t* q, const int8_t* k, const int8_t* v, const int
                                  stream);
 }
 
-int intattn_forward_variant(const int8_t* q, const int8_t* k, const int8_t* v, const intattn_scales_t* scales,
-                            int B, int H, int Lq, int Lk, int d, int causal, float clip_c, int8_t* out,
-                            int variant, intattn_stream_t stream) {
-  if (variant != INTATTN_VARIANT_AUTO && variant != INTATTN_VARIANT_THREE_PASS &&
-      variant != INTATTN_VARIANT_SHORT_ROWS)
-    return INTATTN_ERR_INVALID_ARG;
-  if (variant == INTATTN_VARIANT_SHORT_ROWS && Lk > intattn::shortrow::kMaxKeys) return INTATTN_ERR_UNSUPPORTED;
-  if (B < 0 || H <= 0 || Lq < 0 || Lk < 1 || Lk > 65535) return INTATTN_ERR_INVALID_ARG;
-  if (causal && Lq > Lk) return INTATTN_ERR_INVALID_ARG;
-  if (d != 64 && d != 128) return INTATTN_ERR_UNSUPPORTED;
-  if (!scales) return INTATTN_ERR_INVALID_ARG;
-  static_assert(sizeof(PrefillArgs) <= 8192, "kernel argument block too large");
-  PrefillArgs args;
-  std::memset(&args, 0, sizeof(args));
-  int rc = derive(scales, H, d, clip_c, args.lut, args.hp, INTATTN_MAX_HEADS, &args.n_luts);
-  if (rc) return rc;
+}  // extern "C"
+
+namespace {
+
+// The forward launch once the tables and head parameters are in `args`
+// (args.lut, args.n_luts, args.per_head, and args.hp or args.hp_dev).
+int forward_launch(const int8_t* q, const int8_t* k, const int8_t* v, PrefillArgs& args, int B, int H, int Lq,
+                   int Lk, int d, int causal, int8_t* out, int variant, cudaStream_t st) {
   const long long BH = static_cast<long long>(B) * H;
   if (BH == 0 || Lq == 0) return INTATTN_OK;
   if (!q || !k || !v || !out) return INTATTN_ERR_INVALID_ARG;
@@ -413,7 +406,6 @@ int intattn_forward_variant(const int8_t* q, const int8_t* k, const int8_t* v, c
   args.Lk = Lk;
   args.causal = causal ? 1 : 0;
   args.n_qtiles = n_qtiles;
-  args.per_head = scales->per_head ? 1 : 0;
   args.n_tiles = static_cast<int32_t>(BH * n_qtiles);
   div_magic(static_cast<uint32_t>(BH), &args.div_bh_m, &args.div_bh_sh);
   div_magic(static_cast<uint32_t>(H), &args.div_h_m, &args.div_h_sh);
@@ -421,13 +413,154 @@ int intattn_forward_variant(const int8_t* q, const int8_t* k, const int8_t* v, c
   if (sm_count(&sms) != INTATTN_OK) return INTATTN_ERR_CUDA;
   // persistent kernel: one CTA per SM (each holds all 512 TMEM columns)
   const int grid = args.n_tiles < sms ? args.n_tiles : sms;
-  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   // rows of at most 256 keys: the scores stay in tensor memory through the three sweeps
   const bool short_rows = variant == INTATTN_VARIANT_SHORT_ROWS ||
                           (variant == INTATTN_VARIANT_AUTO && Lk <= intattn::shortrow::kMaxKeys);
   if (short_rows)
     return d == 64 ? prefill_short_launch<64>(args, grid, st) : prefill_short_launch<128>(args, grid, st);
   return d == 64 ? prefill_launch<64>(args, grid, st) : prefill_launch<128>(args, grid, st);
+}
+
+// Exp tables of the distinct clip thresholds of n entries (clips[i], or
+// clip_c for all when clips is null) and each entry's table index.
+int clip_tables(const float* clips, float clip_c, int n, uint32_t lut[INTATTN_MAX_CLIPS][32], int32_t* idx,
+                int* n_luts) {
+  float seen[INTATTN_MAX_CLIPS];
+  int m = 0;
+  for (int i = 0; i < n; ++i) {
+    const float c = clips ? clips[i] : clip_c;
+    int id = 0;
+    while (id < m && !(seen[id] == c)) ++id;
+    if (id == m) {
+      if (m == INTATTN_MAX_CLIPS) return INTATTN_ERR_UNSUPPORTED;
+      const int rc = make_lut(static_cast<double>(c), lut[m]);
+      if (rc) return rc;
+      seen[m++] = c;
+    }
+    idx[i] = id;
+  }
+  *n_luts = m;
+  return INTATTN_OK;
+}
+
+size_t align256_fp(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
+
+// Workspace of intattn_forward_fp: int8 q, k, v; the three scale arrays; the
+// head parameters; the derivation status.
+struct FpLayout {
+  size_t q8, k8, v8, sc, hp, status, total;
+};
+
+FpLayout fp_layout(int B, int H, int Lq, int Lk, int d) {
+  const size_t bh = static_cast<size_t>(B) * H;
+  FpLayout L{};
+  L.q8 = 0;
+  L.k8 = L.q8 + align256_fp(bh * Lq * d);
+  L.v8 = L.k8 + align256_fp(bh * Lk * d);
+  L.sc = L.v8 + align256_fp(bh * Lk * d);
+  L.hp = L.sc + 3 * align256_fp(INTATTN_MAX_HEADS * sizeof(float));
+  L.status = L.hp + align256_fp(INTATTN_MAX_HEADS * sizeof(HeadParamsDev));
+  L.total = L.status + 256;
+  return L;
+}
+
+}  // namespace
+
+extern "C" {
+
+int intattn_forward_variant(const int8_t* q, const int8_t* k, const int8_t* v, const intattn_scales_t* scales,
+                            int B, int H, int Lq, int Lk, int d, int causal, float clip_c, int8_t* out,
+                            int variant, intattn_stream_t stream) {
+  if (variant != INTATTN_VARIANT_AUTO && variant != INTATTN_VARIANT_THREE_PASS &&
+      variant != INTATTN_VARIANT_SHORT_ROWS)
+    return INTATTN_ERR_INVALID_ARG;
+  if (variant == INTATTN_VARIANT_SHORT_ROWS && Lk > intattn::shortrow::kMaxKeys) return INTATTN_ERR_UNSUPPORTED;
+  if (B < 0 || H <= 0 || Lq < 0 || Lk < 1 || Lk > 65535) return INTATTN_ERR_INVALID_ARG;
+  if (causal && Lq > Lk) return INTATTN_ERR_INVALID_ARG;
+  if (d != 64 && d != 128) return INTATTN_ERR_UNSUPPORTED;
+  if (!scales) return INTATTN_ERR_INVALID_ARG;
+  static_assert(sizeof(PrefillArgs) <= 8192, "kernel argument block too large");
+  PrefillArgs args;
+  std::memset(&args, 0, sizeof(args));
+  int rc = derive(scales, H, d, clip_c, args.lut, args.hp, INTATTN_MAX_HEADS, &args.n_luts);
+  if (rc) return rc;
+  args.per_head = scales->per_head ? 1 : 0;
+  return forward_launch(q, k, v, args, B, H, Lq, Lk, d, causal, out, variant, reinterpret_cast<cudaStream_t>(stream));
+}
+
+size_t intattn_forward_fp_workspace_size(int B, int H, int Lq, int Lk, int d) {
+  if (B < 0 || H <= 0 || Lq < 0 || Lk < 1 || (d != 64 && d != 128)) return 0;
+  return fp_layout(B, H, Lq, Lk, d).total;
+}
+
+int intattn_forward_fp(const void* q, const void* k, const void* v, int dtype, int per_head, const float* s_o,
+                       const float* clip, float clip_c, int B, int H, int Lq, int Lk, int d, int causal,
+                       int8_t* out, float* scales_out, void* workspace, size_t workspace_bytes,
+                       intattn_stream_t stream) {
+  if (B < 0 || H <= 0 || Lq < 0 || Lk < 1 || Lk > 65535) return INTATTN_ERR_INVALID_ARG;
+  if (causal && Lq > Lk) return INTATTN_ERR_INVALID_ARG;
+  if (d != 64 && d != 128) return INTATTN_ERR_UNSUPPORTED;
+  if (dtype != INTATTN_DTYPE_FP16 && dtype != INTATTN_DTYPE_BF16) return INTATTN_ERR_UNSUPPORTED;
+  if (!s_o) return INTATTN_ERR_INVALID_ARG;
+  const int n = per_head ? H : 1;
+  if (n > INTATTN_MAX_HEADS) return INTATTN_ERR_UNSUPPORTED;
+  static_assert(sizeof(intattn::DeriveArgs) <= 8192, "kernel argument block too large");
+  intattn::DeriveArgs da;
+  std::memset(&da, 0, sizeof(da));
+  PrefillArgs args;
+  std::memset(&args, 0, sizeof(args));
+  int rc = clip_tables(clip, clip_c, n, args.lut, da.lut, &args.n_luts);
+  if (rc) return rc;
+  for (int i = 0; i < n; ++i) {
+    const double so = s_o[i];
+    if (!std::isfinite(so) || !(so > 0.0)) return INTATTN_ERR_PARAM_RANGE;
+    da.s_o[i] = s_o[i];
+    da.clip[i] = clip ? clip[i] : clip_c;
+  }
+  const long long BH = static_cast<long long>(B) * H;
+  if (BH == 0 || Lq == 0) return INTATTN_OK;
+  if (!q || !k || !v || !out) return INTATTN_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out)) return INTATTN_ERR_UNSUPPORTED;
+  if (scales_out && (reinterpret_cast<uintptr_t>(scales_out) & 3u)) return INTATTN_ERR_UNSUPPORTED;
+  const FpLayout L = fp_layout(B, H, Lq, Lk, d);
+  if (!workspace || workspace_bytes < L.total || (reinterpret_cast<uintptr_t>(workspace) & 255u))
+    return INTATTN_ERR_WORKSPACE;
+  char* ws = static_cast<char*>(workspace);
+  int8_t* q8 = reinterpret_cast<int8_t*>(ws + L.q8);
+  int8_t* k8 = reinterpret_cast<int8_t*>(ws + L.k8);
+  int8_t* v8 = reinterpret_cast<int8_t*>(ws + L.v8);
+  float* sc = reinterpret_cast<float*>(ws + L.sc);
+  const size_t sc_step = align256_fp(INTATTN_MAX_HEADS * sizeof(float)) / sizeof(float);
+  float* s_q = sc;
+  float* s_k = sc + sc_step;
+  float* s_v = sc + 2 * sc_step;
+  HeadParamsDev* hp = reinterpret_cast<HeadParamsDev*>(ws + L.hp);
+  uint32_t* status = reinterpret_cast<uint32_t*>(ws + L.status);
+  // quantise on the stream (scales stay on the device)
+  if ((rc = intattn_quantize(q, dtype, B, H, Lq, d, per_head, q8, s_q, stream)) ||
+      (rc = intattn_quantize(k, dtype, B, H, Lk, d, per_head, k8, s_k, stream)) ||
+      (rc = intattn_quantize(v, dtype, B, H, Lk, d, per_head, v8, s_v, stream)))
+    return rc;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  da.s_q = s_q;
+  da.s_k = s_k;
+  da.s_v = s_v;
+  da.hp = hp;
+  da.status = status;
+  da.n = n;
+  da.d = d;
+  intattn::params::derive_params_kernel<<<1, 128, 0, st>>>(da);
+  if ((rc = note_launch(cudaGetLastError()))) return rc;
+  if (scales_out) {
+    for (int t = 0; t < 3; ++t)
+      if ((rc = note_launch(cudaMemcpyAsync(scales_out + t * n, sc + t * sc_step, n * sizeof(float),
+                                            cudaMemcpyDeviceToDevice, st))))
+        return rc;
+  }
+  args.per_head = per_head ? 1 : 0;
+  args.hp_dev = hp;
+  args.status = status;
+  return forward_launch(q8, k8, v8, args, B, H, Lq, Lk, d, causal, out, INTATTN_VARIANT_AUTO, st);
 }
 
 // ------------------------------------------------ forward from host buffers
@@ -840,7 +973,7 @@ int intattn_device_error(intattn_stream_t stream) {
   if (v == 0) return INTATTN_OK;
   const unsigned int zero = 0;
   if (cudaMemcpyToSymbol(intattn::g_device_error, &zero, sizeof(zero)) != cudaSuccess) return INTATTN_ERR_CUDA;
-  return INTATTN_ERR_TIMEOUT;
+  return (v & intattn::kErrTimeout) ? INTATTN_ERR_TIMEOUT : INTATTN_ERR_PARAM_RANGE;
 }
 
 const char* intattn_strerror(int code) {

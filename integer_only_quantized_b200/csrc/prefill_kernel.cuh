@@ -65,6 +65,10 @@ struct PrefillArgs {
   int32_t div_bh_sh, div_h_sh;
   uint32_t lut[INTATTN_MAX_CLIPS][32];  // one exp table per distinct clip threshold
   HeadParamsDev hp[INTATTN_MAX_HEADS];
+  // parameters derived on the device instead (then hp is unused), and the
+  // status of that derivation: the kernel writes nothing unless it is 0
+  const HeadParamsDev* hp_dev;
+  const uint32_t* status;
 };
 
 namespace prefill {
@@ -246,6 +250,7 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_kernel(const __grid_const
   const int tid = threadIdx.x;
   const int warp = tid >> 5;
   const int lane = tid & 31;
+  if (args.status != nullptr && *args.status != 0u) return;  // parameters out of range: no output
 
   // ---- set-up: barriers, LUT, TMEM (once per CTA) ----
   if (tid == 0) {
@@ -273,7 +278,7 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_kernel(const __grid_const
   for (int i = tid; i < args.n_luts * 32; i += blockDim.x) lut_s[i] = args.lut[i >> 5][i & 31];
   // head parameters in shared memory: a dynamically indexed kernel argument
   // is a constant-bank load that can miss
-  for (int i = tid; i < (args.per_head ? args.H : 1); i += blockDim.x) hp_s[i] = args.hp[i];
+  for (int i = tid; i < (args.per_head ? args.H : 1); i += blockDim.x) hp_s[i] = args.hp_dev ? args.hp_dev[i] : args.hp[i];
   if (warp == kMmaWarp) {
     tmem_alloc(smem_u32(tmem_slot), kTmemCols);
     tmem_relinquish();

@@ -164,6 +164,7 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_short_kernel(const __grid
   const int tid = threadIdx.x;
   const int warp = tid >> 5;
   const int lane = tid & 31;
+  if (args.status != nullptr && *args.status != 0u) return;  // parameters out of range: no output
 
   if (tid == 0) {
     for (int i = 0; i < 2; ++i) {
@@ -190,7 +191,7 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_short_kernel(const __grid
   for (int i = tid; i < args.n_luts * 32; i += blockDim.x) lut_s[i] = args.lut[i >> 5][i & 31];
   // head parameters in shared memory: a dynamically indexed kernel argument
   // is a constant-bank load that can miss
-  for (int i = tid; i < (args.per_head ? args.H : 1); i += blockDim.x) hp_s[i] = args.hp[i];
+  for (int i = tid; i < (args.per_head ? args.H : 1); i += blockDim.x) hp_s[i] = args.hp_dev ? args.hp_dev[i] : args.hp[i];
   if (warp == kMmaWarp) {
     tmem_alloc(smem_u32(tmem_slot), kTmemCols);
     tmem_relinquish();

@@ -119,6 +119,30 @@ def test_forward_variant_argument_errors_need_no_device(ia):
         assert fv(variant, B=0) == ia.OK  # nothing to do, no launch
 
 
+def test_forward_fp_argument_errors_need_no_device(ia):
+    import numpy as np
+    L = ia.lib()
+    f32p = ctypes.POINTER(ctypes.c_float)
+    so = np.array([0.03, 0.03], np.float32)
+    bad = np.array([0.03, 0.0], np.float32)
+    need = ia.forward_fp_workspace_size(1, 2, 64, 64, 64)
+    assert need > 3 * 2 * 64 * 64 and ia.forward_fp_workspace_size(1, 2, 64, 64, 96) == 0
+
+    def call(dtype=1, per_head=1, s_o=so, d=64, ws=256, wsb=None, B=1):
+        return L.intattn_forward_fp(16, 16, 16, dtype, per_head, s_o.ctypes.data_as(f32p) if s_o is not None else None,
+                                    None, 8.0, B, 2, 64, 64, d, 0, 16, None, ws,
+                                    need if wsb is None else wsb, None)
+
+    assert call(dtype=7) == ia.ERR_UNSUPPORTED
+    assert call(d=96) == ia.ERR_UNSUPPORTED
+    assert call(s_o=None) == ia.ERR_INVALID_ARG
+    assert call(s_o=bad) == ia.ERR_PARAM_RANGE
+    assert call(wsb=need - 1) == ia.ERR_WORKSPACE
+    assert call(ws=None) == ia.ERR_WORKSPACE
+    assert call(ws=256 + 16) == ia.ERR_WORKSPACE   # misaligned workspace
+    assert call(B=0) == ia.OK                        # nothing to do, no launch
+
+
 def test_misaligned_pointer_is_rejected(ia):
     sc = ia.Scales(0.1, 0.1, 0.1, 0.1)
     s, keep = sc._c()
