@@ -31,7 +31,8 @@
  *   - Tensor pointers are DEVICE pointers, 16-byte aligned, row-major and
  *     contiguous with the innermost dimension d.  The caller owns them.
  *   - The library allocates and frees nothing, never synchronises the stream
- *     (except intattn_device_error), and launches only on the given stream.
+ *     (except intattn_device_error and intattn_calibrate_clip, which return
+ *     results to the host), and launches only on the given stream.
  *     Calls are asynchronous: a 0 return means the work was enqueued.
  *     One exception: intattn_forward_host (host buffers) creates two copy
  *     streams per device and events per workspace on first use, runs its
@@ -257,6 +258,36 @@ int intattn_forward_fp(const void *q, const void *k, const void *v, int dtype, i
                        const float *s_o, const float *clip, float clip_c, int B, int H, int Lq, int Lk,
                        int d, int causal, int8_t *out, float *scales_out, void *workspace,
                        size_t workspace_bytes, intattn_stream_t stream);
+
+/* Bytes of device workspace intattn_calibrate_clip needs (0 for invalid sizes). */
+size_t intattn_calibrate_workspace_size(int B, int H);
+
+/* Adaptive clip thresholds from the scores themselves.  The summary pages
+ * (sections 概览 / Overview and 局限性与未来工作 / Limitations & Future Work)
+ * describe the clip as sparsity-aware, limiting extreme activations
+ * dynamically, and name an adaptive threshold as future work without a rule;
+ * this is the library's reading:
+ *   sampled rows i = stride - 1, 2 stride - 1, ... < Lq of every (b, h);
+ *   G_i = m_i - S_i,(K): the gap from the row max to the K-th largest score
+ *   (K = keep) over the row's valid keys (causal as intattn_forward), or to
+ *   the smallest score when fewer than K keys are valid;
+ *   G = max of G_i over the sampled rows and the batch (per head), or over
+ *   everything (per-tensor scales);
+ *   c = clamp(alpha G 31 / 30, c_min, c_max), alpha = s_q s_k / sqrt(d), in
+ *   IEEE double in that order, then rounded to float.
+ * Every sampled row then keeps at least K keys at a table index <= 30
+ * (unclipped), with the threshold, and so the table spacing c / 31, as small
+ * as that allows.  The result goes to the clip_c member of intattn_scales_t.
+ *   q [B, H, Lq, d], k [B, H, Lk, d]: device int8.  scales: HOST, s_q and s_k
+ *   used (per_head as given).  clip_out: HOST, H entries per head or 1.
+ *   gaps_out: NULL or HOST, the same count: the integer G of each entry.
+ *   workspace: device, 256-byte aligned, intattn_calibrate_workspace_size.
+ * Unlike the other entry points this one returns its result to the host, so
+ * it synchronises `stream` before returning (one kernel launch, one copy). */
+int intattn_calibrate_clip(const int8_t *q, const int8_t *k, const intattn_scales_t *scales, int B, int H,
+                           int Lq, int Lk, int d, int causal, int keep, int stride, float c_min, float c_max,
+                           float *clip_out, int32_t *gaps_out, void *workspace, size_t workspace_bytes,
+                           intattn_stream_t stream);
 
 /* Integer GELU (the summary page "[Paper] IntAttention：全整数注意力流水线用于
  * 高效边缘推理", section 局限性与未来工作, names GELU as the next operator for the

@@ -24,6 +24,7 @@ MAX_CLIPS = 8
 # every function declared in include/intattn.h
 EXPORTED = ("intattn_derive_params", "intattn_forward", "intattn_forward_variant",
             "intattn_forward_host_workspace_size", "intattn_forward_fp_workspace_size", "intattn_forward_fp",
+            "intattn_calibrate_workspace_size", "intattn_calibrate_clip",
             "intattn_forward_host", "intattn_decode_workspace_size",
             "intattn_decode", "intattn_decode_int4", "intattn_decode_static_scratch", "intattn_quantize",
             "intattn_gelu_derive_params", "intattn_gelu", "intattn_selftest_timeout", "intattn_device_error",
@@ -109,6 +110,11 @@ def lib() -> ctypes.CDLL:
         f32p = ctypes.POINTER(ctypes.c_float)
         L.intattn_forward_fp.argtypes = [vp, vp, vp, i32, i32, f32p, f32p, f32, i32, i32, i32, i32, i32, i32,
                                          vp, vp, vp, ctypes.c_size_t, vp]
+        L.intattn_calibrate_workspace_size.argtypes = [i32, i32]
+        L.intattn_calibrate_workspace_size.restype = ctypes.c_size_t
+        L.intattn_calibrate_clip.argtypes = [vp, vp, ctypes.POINTER(_Scales), i32, i32, i32, i32, i32, i32, i32,
+                                             i32, f32, f32, f32p, ctypes.POINTER(ctypes.c_int32), vp,
+                                             ctypes.c_size_t, vp]
         L.intattn_forward_host_workspace_size.argtypes = [i32, i32, i32, i32, i32]
         L.intattn_forward_host_workspace_size.restype = ctypes.c_size_t
         L.intattn_forward_host.argtypes = [vp, vp, vp, ctypes.POINTER(_Scales), i32, i32, i32, i32, i32,
@@ -269,6 +275,34 @@ def forward_fp(q, k, v, per_head: bool, s_o, causal: bool, clip_c: float, clip=N
                                   workspace.numel(), _stream_handle(stream, q.device))
     _check(rc, "intattn_forward_fp")
     return out
+
+
+def calibrate_clip(q, k, scales: Scales, causal: bool, keep: int, stride: int, c_min: float = 0.25,
+                   c_max: float = 64.0, workspace=None, stream=None):
+    """intattn_calibrate_clip: (thresholds float32 [H or 1], gaps int32 [H or 1])
+    for int8 CUDA q [B,H,Lq,d], k [B,H,Lk,d].  Synchronises the stream."""
+    import torch
+    _check_tensor(q, "q")
+    _check_tensor(k, "k")
+    B, H, Lq, d = q.shape
+    Lk = k.shape[2]
+    if k.shape != (B, H, Lk, d):
+        raise ValueError("k must be [B, H, Lk, d] matching q")
+    n = H if scales.per_head else 1
+    clip = np.zeros(n, dtype=np.float32)
+    gaps = np.zeros(n, dtype=np.int32)
+    if workspace is None:
+        workspace = torch.empty(max(int(lib().intattn_calibrate_workspace_size(B, H)), 1), dtype=torch.uint8,
+                                device=q.device)
+    sc, keep_alive = scales._c()
+    rc = lib().intattn_calibrate_clip(q.data_ptr(), k.data_ptr(), ctypes.byref(sc), B, H, Lq, Lk, d,
+                                      int(bool(causal)), int(keep), int(stride), float(c_min), float(c_max),
+                                      clip.ctypes.data_as(ctypes.POINTER(ctypes.c_float)),
+                                      gaps.ctypes.data_as(ctypes.POINTER(ctypes.c_int32)), workspace.data_ptr(),
+                                      workspace.numel(), _stream_handle(stream, q.device))
+    del keep_alive
+    _check(rc, "intattn_calibrate_clip")
+    return clip, gaps
 
 
 def decode_workspace_size(B: int, H: int, Lk: int, d: int) -> int:

@@ -14,9 +14,11 @@
 #include <cstring>
 #include <mutex>
 #include <unordered_map>
+#include <vector>
 
 #include "intattn.h"
 
+#include "calibrate_kernel.cuh"
 #include "decode_kernel.cuh"
 #include "gelu_kernel.cuh"
 #include "params_kernel.cuh"
@@ -959,6 +961,60 @@ int intattn_gelu(const int8_t* x, int8_t* y, long long n, float s_x, float s_y, 
   const unsigned grid = static_cast<unsigned>(std::min<long long>(want, static_cast<long long>(sms) * occ));
   intattn::gelu::gelu_kernel<<<grid, intattn::gelu::kThreads, 0, reinterpret_cast<cudaStream_t>(stream)>>>(a);
   return note_launch(cudaGetLastError());
+}
+
+size_t intattn_calibrate_workspace_size(int B, int H) {
+  if (B < 0 || H <= 0) return 0;
+  return (static_cast<size_t>(B) * H * sizeof(int32_t) + 255) & ~static_cast<size_t>(255);
+}
+
+int intattn_calibrate_clip(const int8_t* q, const int8_t* k, const intattn_scales_t* scales, int B, int H, int Lq,
+                           int Lk, int d, int causal, int keep, int stride, float c_min, float c_max, float* clip_out,
+                           int32_t* gaps_out, void* workspace, size_t workspace_bytes, intattn_stream_t stream) {
+  if (B < 0 || H <= 0 || Lq < 0 || Lk < 1 || Lk > 65535 || keep < 1 || stride < 1) return INTATTN_ERR_INVALID_ARG;
+  if (causal && Lq > Lk) return INTATTN_ERR_INVALID_ARG;
+  if (d != 64 && d != 128) return INTATTN_ERR_UNSUPPORTED;
+  if (!scales || !scales->s_q || !scales->s_k || !clip_out) return INTATTN_ERR_INVALID_ARG;
+  if (!std::isfinite(c_min) || !std::isfinite(c_max) || !(c_min > 0.0f) || !(c_max >= c_min))
+    return INTATTN_ERR_PARAM_RANGE;
+  const int n = scales->per_head ? H : 1;
+  for (int i = 0; i < n; ++i)
+    if (!std::isfinite(scales->s_q[i]) || !std::isfinite(scales->s_k[i]) || !(scales->s_q[i] > 0.0f) ||
+        !(scales->s_k[i] > 0.0f))
+      return INTATTN_ERR_PARAM_RANGE;
+  const long long BH = static_cast<long long>(B) * H;
+  if (BH > 65535) return INTATTN_ERR_UNSUPPORTED;  // grid y
+  std::vector<int32_t> G(static_cast<size_t>(BH), 0);
+  const int rows = Lq / stride;  // sampled rows stride - 1, 2 stride - 1, ...
+  if (BH > 0 && rows > 0) {
+    if (!q || !k) return INTATTN_ERR_INVALID_ARG;
+    if (!aligned16(q) || !aligned16(k)) return INTATTN_ERR_UNSUPPORTED;
+    if (!workspace || workspace_bytes < intattn_calibrate_workspace_size(B, H) ||
+        (reinterpret_cast<uintptr_t>(workspace) & 255u))
+      return INTATTN_ERR_WORKSPACE;
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    int32_t* dG = static_cast<int32_t*>(workspace);
+    intattn::CalibArgs a{q, k, dG, Lq, Lk, d, causal ? 1 : 0, keep, stride};
+    int rc = note_launch(cudaMemsetAsync(dG, 0, static_cast<size_t>(BH) * sizeof(int32_t), st));
+    if (rc) return rc;
+    intattn::calib::gap_kernel<<<dim3(rows, static_cast<unsigned>(BH)), intattn::calib::kThreads, 0, st>>>(a);
+    if ((rc = note_launch(cudaGetLastError()))) return rc;
+    if ((rc = note_launch(cudaMemcpyAsync(G.data(), dG, G.size() * sizeof(int32_t), cudaMemcpyDeviceToHost, st))))
+      return rc;
+    if ((rc = note_launch(cudaStreamSynchronize(st)))) return rc;
+  }
+  // the threshold of each entry from its largest gap, IEEE double in this order
+  for (int e = 0; e < n; ++e) {
+    int32_t g = 0;
+    for (long long bh = 0; bh < BH; ++bh)
+      if (!scales->per_head || bh % H == e) g = std::max(g, G[static_cast<size_t>(bh)]);
+    const double alpha = (static_cast<double>(scales->s_q[e]) * static_cast<double>(scales->s_k[e])) /
+                         std::sqrt(static_cast<double>(d));
+    const double c = ((alpha * static_cast<double>(g)) * 31.0) / 30.0;
+    clip_out[e] = static_cast<float>(std::min(std::max(c, static_cast<double>(c_min)), static_cast<double>(c_max)));
+    if (gaps_out) gaps_out[e] = g;
+  }
+  return INTATTN_OK;
 }
 
 int intattn_selftest_timeout(intattn_stream_t stream) {

@@ -143,6 +143,32 @@ def test_forward_fp_argument_errors_need_no_device(ia):
     assert call(B=0) == ia.OK                        # nothing to do, no launch
 
 
+def test_calibrate_argument_errors_need_no_device(ia):
+    import numpy as np
+    L = ia.lib()
+    sc = ia.Scales([0.02, 0.03], [0.02, 0.03], [0.1, 0.1], [0.1, 0.1], per_head=True)
+    s, keep_alive = sc._c()
+    clip = np.zeros(2, np.float32)
+    fp = ctypes.POINTER(ctypes.c_float)
+    ws = ia.lib().intattn_calibrate_workspace_size(1, 2)
+    assert ws >= 8 and ia.lib().intattn_calibrate_workspace_size(1, 0) == 0
+
+    def call(keep=4, stride=2, c_min=0.5, c_max=20.0, out=True, d=64, wsb=None, B=1):
+        return L.intattn_calibrate_clip(16, 16, ctypes.byref(s), B, 2, 64, 64, d, 0, keep, stride, c_min, c_max,
+                                        clip.ctypes.data_as(fp) if out else None, None, 256,
+                                        ws if wsb is None else wsb, None)
+
+    assert call(keep=0) == ia.ERR_INVALID_ARG
+    assert call(stride=0) == ia.ERR_INVALID_ARG
+    assert call(c_min=0.0) == ia.ERR_PARAM_RANGE
+    assert call(c_max=0.1) == ia.ERR_PARAM_RANGE
+    assert call(out=False) == ia.ERR_INVALID_ARG
+    assert call(d=96) == ia.ERR_UNSUPPORTED
+    assert call(wsb=ws - 4) == ia.ERR_WORKSPACE
+    # nothing sampled (B = 0): no launch, every threshold is c_min
+    assert call(B=0, c_min=0.75) == ia.OK and clip.tolist() == [0.75, 0.75]
+
+
 def test_misaligned_pointer_is_rejected(ia):
     sc = ia.Scales(0.1, 0.1, 0.1, 0.1)
     s, keep = sc._c()
