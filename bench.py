@@ -392,6 +392,8 @@ def run_prefill_configs(args, ia, dev, stream, world, peak_int8, skip):
         steps = max(args.steps, 100, nsets)  # every copy is used at least once
         ms, _ = time_prefill(ia, w, x, dev, stream, steps, max(3, args.warmup), None, world)
         tops = w.effective_ops / (ms * 1e-3) / 1e12
+        # the kernel intattn_forward picks for this row length
+        kname = "prefill_short_kernel" if w.Lk <= ia.SHORT_ROWS_MAX_KEYS else "prefill_kernel"
         if tops > 1.5 * peak_int8:
             raise RuntimeError(f"{name}: {tops:.0f} TOPS is far above the int8 peak: the timed region missed the work")
         res[name] = {"value": round(aggregate_value(w.effective_ops, world, ms * 1e-3) / 1e12, 3), "unit": "TOPS",
@@ -399,7 +401,7 @@ def run_prefill_configs(args, ia, dev, stream, world, peak_int8, skip):
                      "effective_ops": w.effective_ops,
                      "roofline": {"bound": "tensor", "achieved": round(tops, 3), "peak": round(peak_int8, 1),
                                   "unit": "TOPS", "frac": round(tops / peak_int8, 4),
-                                  "traffic": kernel_traffic("prefill_kernel", name)},
+                                  "kernel": kname, "traffic": kernel_traffic(kname, name)},
                      "l2": f"inputs rotate over {nsets} copies ({nsets * set_bytes / 2**20:.0f} MiB > 126 MiB L2)"}
         if w.Lk <= 2 * ia.SHORT_ROWS_MAX_KEYS:
             # both ways of handling a short row's scores on the same workload:
