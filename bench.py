@@ -49,7 +49,7 @@ def parse_args(argv=None):
     p.add_argument("--no-decode", action="store_true")
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--cpu-seconds", type=float, default=12.0)
-    p.add_argument("--leg", choices=["decode", "decode_int4", "quantize", "gelu", "forward_fp"], default=None,
+    p.add_argument("--leg", choices=["decode", "decode_int4", "quantize", "gelu", "forward_fp", "calibrate"], default=None,
                    help="run only this secondary leg and print its object (for profiler captures)")
     return p.parse_args(argv)
 
@@ -282,6 +282,8 @@ def run_leg(args):
         out = run_quantize(args, dev, stream, world, peaks, peak_src)
     elif args.leg == "forward_fp":
         out = run_forward_fp(args, dev, stream, world, peaks, peak_src)
+    elif args.leg == "calibrate":
+        out = run_calibrate(args, dev, stream, world)
     else:
         out = run_gelu(args, dev, stream, world, peaks, peak_src)
     if rank == 0:
@@ -368,6 +370,7 @@ def run_ours(args):
                                          "llama7b_decode_int4_b64_lk4096")
         line["quantize"] = run_quantize(args, dev, stream, world, peaks, peak_src)
         line["forward_fp"] = run_forward_fp(args, dev, stream, world, peaks, peak_src)
+        line["calibrate"] = run_calibrate(args, dev, stream, world)
         line["gelu"] = run_gelu(args, dev, stream, world, peaks, peak_src)
     if not args.no_cpu_baseline and rank == 0 and world == 1:
         line["cpu_baseline"] = cpu_baseline(w, x, args.cpu_seconds)
@@ -501,6 +504,56 @@ def run_forward_fp(args, dev, stream, world, peaks, peak_src):
             "roofline": {"bound": "tensor", "achieved": round(tops, 3), "peak": round(peak_int8, 1), "unit": "TOPS",
                          "frac": round(tops / peak_int8, 4)},
             "l2": "inputs alternate between 2 sets (201 MB > 126 MB L2)"}
+
+
+def run_calibrate(args, dev, stream, world):
+    """Adaptive clip thresholds (intattn_calibrate_clip) on the LLaMA-7B
+    causal prefill codes: every 64th query row of each head sampled, the gap
+    to its 32nd largest score.  Each sampled row's scores are recomputed
+    (dp4a) in each of the three radix-select sweeps, so the kernel's work is
+    3 x (sampled rows x valid keys x d) multiply-adds, its K reads served by
+    L2.  Timed with CUDA events around whole calls (the call copies the gaps
+    to the host and synchronises)."""
+    import torch
+
+    import integer_only_quantized_b200 as ia
+    from integer_only_quantized_b200 import workloads as wl
+    w = wl.WORKLOADS["llama7b_causal_l8192"]
+    x = wl.make_inputs(w)
+    q = torch.from_numpy(x.q).to(dev)
+    k = torch.from_numpy(x.k).to(dev)
+    sc = ia.Scales(x.s_q, x.s_k, x.s_v, x.s_o, per_head=w.per_head)
+    keep, stride = 32, 64
+    ws = torch.empty(max(ia.calibrate_workspace_size(w.B, w.H), 1), dtype=torch.uint8, device=dev)
+    call = lambda: ia.calibrate_clip(q, k, sc, w.causal, keep, stride, workspace=ws, stream=stream)
+    for _ in range(max(3, args.warmup)):
+        call()
+    steps = max(5, min(args.steps, 20))
+    barrier(world, dev)
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    t0.record(stream)
+    for _ in range(steps):
+        call()
+    t1.record(stream)
+    torch.cuda.synchronize(dev)
+    barrier(world, dev)
+    ms = max_over_ranks(t0.elapsed_time(t1) / steps, world, dev)
+    if ia.device_error(stream) != ia.OK:
+        raise RuntimeError("a kernel wait timed out in calibrate_clip")
+    rows = list(range(stride - 1, w.Lq, stride))
+    off = w.Lk - w.Lq
+    keys = sum(min(w.Lk, i + off + 1) if w.causal else w.Lk for i in rows) * w.B * w.H
+    ops = 3 * keys * w.d * 2  # three sweeps of int8 multiply-adds
+    tops = ops / (ms * 1e-3) / 1e12
+    # dp4a issues at half the FP32 rate: 64 per clock per SM, 8 int8 ops each
+    peak = 148 * 64 * 8 * 1.965e9 / 1e12
+    return {"workload": w.name + f"_keep{keep}_stride{stride}", "ms_per_call": round(ms, 5), "launches_per_call": 2,
+            "sampled_rows": len(rows) * w.B * w.H, "scores_per_sweep": keys,
+            "note": "memset of the gap buffer + gap kernel; thresholds from the gaps on the host",
+            "value": round(aggregate_value(ops, world, ms * 1e-3) / 1e12, 3), "unit": "TOPS (dp4a int8)",
+            "roofline": {"bound": "alu", "achieved": round(tops, 3), "peak": round(peak, 1), "unit": "TOPS",
+                         "frac": round(tops / peak, 4), "peak_source": "148 SMs x 64 dp4a/clk x 8 ops x 1965 MHz",
+                         "traffic": None}}
 
 
 def run_gelu(args, dev, stream, world, peaks, peak_src):
