@@ -61,6 +61,11 @@ def lib():
                                              i32p, ctypes.c_longlong, i8p, c_int]
         _lib.oracle_decode.argtypes = [i8p, i8p, i8p, c_int, f32p, f32p, f32p, f32p, c_int,
                                        c_int, c_int, c_int, c_int, c_float, i8p, c_int]
+        vp = ctypes.c_void_p
+        _lib.oracle_forward_zp.argtypes = [i8p, vp, vp, i32p, i32p, c_int, f32p, f32p, f32p, f32p,
+                                           c_int, c_int, c_int, c_int, c_int, c_int, c_float, i8p, c_int]
+        _lib.oracle_decode_zp.argtypes = [i8p, vp, vp, i32p, i32p, c_int, f32p, f32p, f32p, f32p,
+                                          c_int, c_int, c_int, c_int, c_int, c_float, i8p, c_int]
     return _lib
 
 
@@ -145,7 +150,24 @@ def requant(acc: int, Mo: int, so: int) -> int:
     return int(lib().oracle_requant(int(acc), Mo, so))
 
 
-def forward(q, k, v, per_head, s_q, s_k, s_v, s_o, causal, clip_c, nthreads=None):
+def _codes_and_zero_points(x, z):
+    """K or V codes with their zero-points: u8 codes and an int32 array when
+    z is given, else int8 codes and None (zero-point 0)."""
+    if z is None:
+        return np.ascontiguousarray(x, dtype=np.int8), None
+    return (np.ascontiguousarray(x, dtype=np.uint8),
+            np.ascontiguousarray(np.atleast_1d(np.asarray(z)), dtype=np.int32))
+
+
+def _zp_ptr(z):
+    return None if z is None else _p(z, ctypes.c_int32)
+
+
+def forward(q, k, v, per_head, s_q, s_k, s_v, s_o, causal, clip_c, nthreads=None, z_k=None, z_v=None):
+    """Prefill.  With z_k (z_v) given, k (v) holds u8 codes whose zero-points
+    are z_k (z_v), one per head or one in all; else int8 codes."""
+    if z_k is not None or z_v is not None:
+        return _forward_zp(q, k, v, per_head, s_q, s_k, s_v, s_o, causal, clip_c, nthreads, z_k, z_v)
     q = np.ascontiguousarray(q, dtype=np.int8)
     k = np.ascontiguousarray(k, dtype=np.int8)
     v = np.ascontiguousarray(v, dtype=np.int8)
@@ -159,6 +181,23 @@ def forward(q, k, v, per_head, s_q, s_k, s_v, s_o, causal, clip_c, nthreads=None
                               int(causal), float(np.float32(clip_c)), _p(out, ctypes.c_int8),
                               int(nthreads or os.cpu_count() or 1))
     _check(rc, "oracle_forward")
+    return out
+
+
+def _forward_zp(q, k, v, per_head, s_q, s_k, s_v, s_o, causal, clip_c, nthreads, z_k, z_v):
+    q = np.ascontiguousarray(q, dtype=np.int8)
+    k, zk = _codes_and_zero_points(k, z_k)
+    v, zv = _codes_and_zero_points(v, z_v)
+    B, H, Lq, d = q.shape
+    Lk = k.shape[2]
+    out = np.zeros((B, H, Lq, d), dtype=np.int8)
+    sq, sk, sv, so = _f32(s_q), _f32(s_k), _f32(s_v), _f32(s_o)
+    rc = lib().oracle_forward_zp(_p(q, ctypes.c_int8), k.ctypes.data, v.ctypes.data, _zp_ptr(zk), _zp_ptr(zv),
+                                 int(per_head), _p(sq, ctypes.c_float), _p(sk, ctypes.c_float),
+                                 _p(sv, ctypes.c_float), _p(so, ctypes.c_float), B, H, Lq, Lk, d,
+                                 int(causal), float(np.float32(clip_c)), _p(out, ctypes.c_int8),
+                                 int(nthreads or os.cpu_count() or 1))
+    _check(rc, "oracle_forward_zp")
     return out
 
 
@@ -183,7 +222,23 @@ def forward_rows(q, k, v, per_head, s_q, s_k, s_v, s_o, causal, clip_c, rows, nt
     return out
 
 
-def decode(q, k_cache, v_cache, per_head, s_q, s_k, s_v, s_o, Lk, clip_c, nthreads=None):
+def decode(q, k_cache, v_cache, per_head, s_q, s_k, s_v, s_o, Lk, clip_c, nthreads=None, z_k=None, z_v=None):
+    """Decode over the first Lk rows of the caches; zero-points as in forward."""
+    if z_k is not None or z_v is not None:
+        q = np.ascontiguousarray(q, dtype=np.int8)
+        kc, zk = _codes_and_zero_points(k_cache, z_k)
+        vc, zv = _codes_and_zero_points(v_cache, z_v)
+        B, H, one, d = q.shape
+        assert one == 1
+        out = np.zeros((B, H, 1, d), dtype=np.int8)
+        sq, sk, sv, so = _f32(s_q), _f32(s_k), _f32(s_v), _f32(s_o)
+        rc = lib().oracle_decode_zp(_p(q, ctypes.c_int8), kc.ctypes.data, vc.ctypes.data, _zp_ptr(zk),
+                                    _zp_ptr(zv), int(per_head), _p(sq, ctypes.c_float), _p(sk, ctypes.c_float),
+                                    _p(sv, ctypes.c_float), _p(so, ctypes.c_float), B, H, int(Lk), kc.shape[2],
+                                    d, float(np.float32(clip_c)), _p(out, ctypes.c_int8),
+                                    int(nthreads or os.cpu_count() or 1))
+        _check(rc, "oracle_decode_zp")
+        return out
     q = np.ascontiguousarray(q, dtype=np.int8)
     kc = np.ascontiguousarray(k_cache, dtype=np.int8)
     vc = np.ascontiguousarray(v_cache, dtype=np.int8)

@@ -37,6 +37,14 @@
  *     P_j   = floor((E_j * R + 2^31) / 2^32)              in [0, 255]
  *     acc_t = sum_j P_j * V[j,t]                          (int32)
  *     out_t = clamp(floor((acc_t * Mo + 2^(so-1)) / 2^so), -127, 127)
+ *
+ *   Zero-points (the forum page "IntAttention：面向边缘设备的纯整数注意力推理加速方案",
+ *   section 动态量化策略: a dynamic scale and zero-point per layer).  K and V
+ *   may be stored as u8 codes with a zero-point z per tensor or per head:
+ *   code c stands for the integer c - z (real value s * (c - z)).  The
+ *   definition above then reads K[j,t] = k_code - z_k and V[j,t] = v_code -
+ *   z_v; Q stays symmetric int8.  oracle_forward_zp / oracle_decode_zp
+ *   compute exactly that, literally.
  */
 #include <math.h>
 #include <pthread.h>
@@ -196,6 +204,33 @@ static void attention_row(const int8_t *q, const int8_t *k, const int8_t *v, int
     for (int t = 0; t < d; t++) out[t] = oracle_requant(acc[t], p->Mo, p->so);
 }
 
+/* One attention row whose K and / or V codes carry a zero-point: kz / vz
+ * are u8 codes with zero-points zk / zv when k_u8 / v_u8, else int8 codes
+ * (zero-point 0).  Written out on its own, element by element. */
+static int32_t code_at(const void *base, int is_u8, size_t i)
+{
+    return is_u8 ? (int32_t)((const uint8_t *)base)[i] : (int32_t)((const int8_t *)base)[i];
+}
+
+static void attention_row_zp(const int8_t *q, const void *kz, int k_u8, int32_t zk,
+                             const void *vz, int v_u8, int32_t zv, int n, int d,
+                             const oracle_head_params *p, const int32_t lut[32], int32_t *S,
+                             uint8_t *P, int32_t *acc, int8_t *out)
+{
+    for (int j = 0; j < n; j++) {
+        int64_t dot = 0;
+        for (int t = 0; t < d; t++)
+            dot += (int64_t)q[t] * (int64_t)(code_at(kz, k_u8, (size_t)j * d + t) - zk);
+        S[j] = (int32_t)dot;
+    }
+    oracle_index_softmax(S, n, p->M, p->s, p->D, lut, P, NULL, NULL, NULL);
+    for (int t = 0; t < d; t++) acc[t] = 0;
+    for (int j = 0; j < n; j++)
+        for (int t = 0; t < d; t++)
+            acc[t] += (int32_t)P[j] * (code_at(vz, v_u8, (size_t)j * d + t) - zv);
+    for (int t = 0; t < d; t++) out[t] = oracle_requant(acc[t], p->Mo, p->so);
+}
+
 typedef struct {
     const int8_t *q, *k, *v;
     int8_t *out;
@@ -205,6 +240,8 @@ typedef struct {
     const int32_t *rows; /* NULL: all rows; else nrows triples (b, h, i) */
     long long nrows;
     int tid, nthreads;
+    /* zero-points per head (H entries), NULL: int8 codes, zero-point 0 */
+    const int32_t *zk, *zv;
 } job_t;
 
 static void *run_rows(void *arg)
@@ -235,7 +272,13 @@ static void *run_rows(void *arg)
         const int8_t *kb = J->k + bh * (size_t)J->Lkv * J->d;
         const int8_t *vb = J->v + bh * (size_t)J->Lkv * J->d;
         int8_t *o = J->out + (J->rows ? (size_t)r * J->d : (bh * J->Lq + (size_t)i) * J->d);
-        attention_row(qrow, kb, vb, n, J->d, &J->hp[h], J->lut, S, P, acc, o);
+        if (J->zk || J->zv) {
+            /* K / V codes are one byte each either way: the same offsets */
+            attention_row_zp(qrow, kb, J->zk != NULL, J->zk ? J->zk[h] : 0, vb, J->zv != NULL,
+                             J->zv ? J->zv[h] : 0, n, J->d, &J->hp[h], J->lut, S, P, acc, o);
+        } else {
+            attention_row(qrow, kb, vb, n, J->d, &J->hp[h], J->lut, S, P, acc, o);
+        }
     }
     free(S);
     free(P);
@@ -289,7 +332,7 @@ int oracle_forward(const int8_t *q, const int8_t *k, const int8_t *v, int per_he
     oracle_head_params *hp = (oracle_head_params *)malloc(sizeof(oracle_head_params) * (size_t)H);
     rc = oracle_params(per_head, s_q, s_k, s_v, s_o, H, d, clip_c, lut, hp);
     if (rc == ORC_OK && B > 0) {
-        job_t J = {q, k, v, out, B, H, Lq, Lk, Lk, d, causal, hp, lut, NULL, 0, 0, 1};
+        job_t J = {q, k, v, out, B, H, Lq, Lk, Lk, d, causal, hp, lut, NULL, 0, 0, 1, NULL, NULL};
         rc = run_threads(&J, nthreads);
     }
     free(hp);
@@ -315,7 +358,7 @@ int oracle_forward_rows(const int8_t *q, const int8_t *k, const int8_t *v, int p
     oracle_head_params *hp = (oracle_head_params *)malloc(sizeof(oracle_head_params) * (size_t)H);
     rc = oracle_params(per_head, s_q, s_k, s_v, s_o, H, d, clip_c, lut, hp);
     if (rc == ORC_OK) {
-        job_t J = {q, k, v, out, B, H, Lq, Lk, Lk, d, causal, hp, lut, rows, nrows, 0, 1};
+        job_t J = {q, k, v, out, B, H, Lq, Lk, Lk, d, causal, hp, lut, rows, nrows, 0, 1, NULL, NULL};
         rc = run_threads(&J, nthreads);
     }
     free(hp);
@@ -336,9 +379,81 @@ int oracle_decode(const int8_t *q, const int8_t *k_cache, const int8_t *v_cache,
     oracle_head_params *hp = (oracle_head_params *)malloc(sizeof(oracle_head_params) * (size_t)H);
     rc = oracle_params(per_head, s_q, s_k, s_v, s_o, H, d, clip_c, lut, hp);
     if (rc == ORC_OK && B > 0) {
-        job_t J = {q, k_cache, v_cache, out, B, H, 1, Lk, Lmax, d, 0, hp, lut, NULL, 0, 0, 1};
+        job_t J = {q, k_cache, v_cache, out, B, H, 1, Lk, Lmax, d, 0, hp, lut, NULL, 0, 0, 1, NULL, NULL};
         rc = run_threads(&J, nthreads);
     }
     free(hp);
+    return rc;
+}
+
+/* Zero-points of every head from a per-tensor (one entry) or per-head (H
+ * entries) array; NULL stays NULL.  Each must be a u8 code, 0..255. */
+static int expand_zero_points(const int32_t *z, int per_head, int H, int32_t **out)
+{
+    *out = NULL;
+    if (!z) return ORC_OK;
+    int32_t *e = (int32_t *)malloc(sizeof(int32_t) * (size_t)H);
+    for (int h = 0; h < H; h++) {
+        int32_t v = z[per_head ? h : 0];
+        if (v < 0 || v > 255) {
+            free(e);
+            return ORC_INVALID_ARG;
+        }
+        e[h] = v;
+    }
+    *out = e;
+    return ORC_OK;
+}
+
+/* Prefill with zero-points: k / v are u8 codes [B,H,Lk,d] when z_k / z_v is
+ * given (per_head: H entries, else one), int8 codes otherwise. */
+int oracle_forward_zp(const int8_t *q, const void *k, const void *v, const int32_t *z_k,
+                      const int32_t *z_v, int per_head, const float *s_q, const float *s_k,
+                      const float *s_v, const float *s_o, int B, int H, int Lq, int Lk, int d,
+                      int causal, float clip_c, int8_t *out, int nthreads)
+{
+    int rc = check_common(q, (const int8_t *)k, (const int8_t *)v, out, B, H, Lq, Lk, d, causal);
+    if (rc) return rc;
+    int32_t *zk = NULL, *zv = NULL;
+    rc = expand_zero_points(z_k, per_head, H, &zk);
+    if (rc == ORC_OK) rc = expand_zero_points(z_v, per_head, H, &zv);
+    int32_t lut[32];
+    oracle_head_params *hp = (oracle_head_params *)malloc(sizeof(oracle_head_params) * (size_t)H);
+    if (rc == ORC_OK) rc = oracle_params(per_head, s_q, s_k, s_v, s_o, H, d, clip_c, lut, hp);
+    if (rc == ORC_OK && B > 0) {
+        job_t J = {q, (const int8_t *)k, (const int8_t *)v, out, B, H, Lq, Lk, Lk, d, causal, hp, lut,
+                   NULL, 0, 0, 1, zk, zv};
+        rc = run_threads(&J, nthreads);
+    }
+    free(hp);
+    free(zk);
+    free(zv);
+    return rc;
+}
+
+/* Decode with zero-points: caches [B,H,Lmax,d] of u8 codes where z_k / z_v is
+ * given, int8 codes otherwise; the first Lk rows are attended. */
+int oracle_decode_zp(const int8_t *q, const void *k_cache, const void *v_cache,
+                     const int32_t *z_k, const int32_t *z_v, int per_head, const float *s_q,
+                     const float *s_k, const float *s_v, const float *s_o, int B, int H, int Lk,
+                     int Lmax, int d, float clip_c, int8_t *out, int nthreads)
+{
+    int rc = check_common(q, (const int8_t *)k_cache, (const int8_t *)v_cache, out, B, H, 1, Lk, d, 0);
+    if (rc) return rc;
+    if (Lmax < Lk) return ORC_INVALID_ARG;
+    int32_t *zk = NULL, *zv = NULL;
+    rc = expand_zero_points(z_k, per_head, H, &zk);
+    if (rc == ORC_OK) rc = expand_zero_points(z_v, per_head, H, &zv);
+    int32_t lut[32];
+    oracle_head_params *hp = (oracle_head_params *)malloc(sizeof(oracle_head_params) * (size_t)H);
+    if (rc == ORC_OK) rc = oracle_params(per_head, s_q, s_k, s_v, s_o, H, d, clip_c, lut, hp);
+    if (rc == ORC_OK && B > 0) {
+        job_t J = {q, (const int8_t *)k_cache, (const int8_t *)v_cache, out, B, H, 1, Lk, Lmax, d, 0,
+                   hp, lut, NULL, 0, 0, 1, zk, zv};
+        rc = run_threads(&J, nthreads);
+    }
+    free(hp);
+    free(zk);
+    free(zv);
     return rc;
 }

@@ -11,6 +11,16 @@ range = max |x|, 127 levels each side, round half to even.  Definition:
     s    = amax / 127 and inv = min(127 / amax, FLT_MAX) in IEEE fp32 (both 1
            when amax = 0)
     code = clamp(rint(x * inv), -127, 127), the fp32 product rounded to nearest
+
+The same page names a zero-point beside the scale; ``quantize_asym`` is that
+form (u8 codes), with the readings: the range always holds 0 (so that 0 is a
+code), 255 levels, the width in IEEE double, round half to even:
+    hi   = max(max x, 0),  lo = min(min x, 0)  over the tensor or one head
+    w    = hi - lo                      (double)
+    s    = RN32(w / 255),  inv = RN32(min(255 / w, FLT_MAX))  (both 1 when w = 0)
+    z    = clamp(rint(RN32(-lo * inv)), 0, 255)
+    code = clamp(rint(RN32(x * inv)) + z, 0, 255)
+A code c stands for s (c - z).
 """
 import numpy as np
 
@@ -34,3 +44,30 @@ def quantize(x, per_head: bool):
     per = inv if per_head else np.repeat(inv, H)
     q = np.rint(x * per[None, :, None, None].astype(np.float32))  # float32 product, half-even
     return np.clip(q, -127, 127).astype(np.int8), s
+
+
+def quantize_asym(x, per_head: bool):
+    """x: float32 [B, H, L, d] holding fp16 / bf16 values.  Returns (codes
+    uint8 [B, H, L, d], scales float32 [H] or [1], zero-points int32 [H] or [1])."""
+    x = np.asarray(x, dtype=np.float32)
+    B, H, L, d = x.shape
+    axes = (0, 2, 3) if per_head else None
+    n = H if per_head else 1
+    if x.size:
+        hi = np.maximum(np.asarray(x.max(axis=axes), np.float32).reshape(n), np.float32(0))
+        lo = np.minimum(np.asarray(x.min(axis=axes), np.float32).reshape(n), np.float32(0))
+    else:
+        hi = np.zeros(n, np.float32)
+        lo = np.zeros(n, np.float32)
+    w = hi.astype(np.float64) - lo.astype(np.float64)
+    s = np.ones(n, np.float32)
+    inv = np.ones(n, np.float32)
+    nz = w != 0
+    s[nz] = (w[nz] / 255.0).astype(np.float32)
+    inv[nz] = np.minimum(255.0 / w[nz], float(np.finfo(np.float32).max)).astype(np.float32)
+    z = np.clip(np.rint((-lo) * inv), 0, 255).astype(np.int32)  # float32 product, half-even
+    per_inv = inv if per_head else np.repeat(inv, H)
+    per_z = z if per_head else np.repeat(z, H)
+    p = np.rint(x * per_inv[None, :, None, None].astype(np.float32))  # float32 product, half-even
+    codes = np.clip(p + per_z[None, :, None, None], 0, 255).astype(np.uint8)
+    return codes, s, z
