@@ -84,6 +84,17 @@ typedef struct intattn_scales {
     const float *s_v;
     const float *s_o;
     const float *clip_c;
+    /* Zero-points (optional, host, the layout of the scales), the forum page's
+     * dynamic scale and zero-point (section 动态量化策略): z_k != NULL means the K
+     * codes are u8 (the k / k_cache pointer is read as uint8_t) and code c
+     * stands for c - z_k; likewise z_v for V.  Each zero-point is 0 .. 255,
+     * else INTATTN_ERR_INVALID_ARG.  The definition then reads
+     * S_j = sum_t Q[i,t] (K[j,t] - z_k) and acc_t = sum_j P_j (V[j,t] - z_v).
+     * Q stays symmetric int8.  Accepted by the forward, intattn_forward_variant,
+     * intattn_forward_host and the int8 decode; intattn_decode_int4 and
+     * intattn_calibrate_clip return INTATTN_ERR_UNSUPPORTED for them. */
+    const int32_t *z_k;
+    const int32_t *z_v;
 } intattn_scales_t;
 
 #define INTATTN_MAX_CLIPS 8
@@ -222,6 +233,22 @@ enum { INTATTN_DTYPE_FP16 = 0, INTATTN_DTYPE_BF16 = 1 };
  * reported by intattn_device_error. */
 int intattn_quantize(const void *x, int dtype, int B, int H, int L, int d, int per_head, int8_t *out,
                      float *scales, intattn_stream_t stream);
+
+/* Asymmetric quantisation prologue: the zero-point the same page names beside
+ * the scale.  u8 codes and a zero-point per tensor or head:
+ *   hi = max(max x, 0), lo = min(min x, 0) over the tensor (or head h) -- the
+ *   range always holds 0, so 0 is the code z;
+ *   w = hi - lo in IEEE double; s = RN32(w / 255) and inv = RN32(min(255 / w,
+ *   FLT_MAX)) (both 1 when w = 0);
+ *   z = clamp(rint(RN32(-lo * inv)), 0, 255);
+ *   code = clamp(rint(RN32(x * inv)) + z, 0, 255), rint half to even.
+ * A code c stands for s * (c - z).
+ *   out [B, H, L, d] u8 codes (first 8 bytes: barrier counters until the end)
+ *   scales: DEVICE float [H] or [1]; zero_points: DEVICE int32 [H] or [1]
+ *   (holds the bits of max(-lo) until the end).  Everything else as
+ *   intattn_quantize; INVALID_ARG for zero_points == NULL. */
+int intattn_quantize_zp(const void *x, int dtype, int B, int H, int L, int d, int per_head, uint8_t *out,
+                        float *scales, int32_t *zero_points, intattn_stream_t stream);
 
 /* Bytes of device workspace intattn_forward_fp needs for these sizes (0 for
  * invalid sizes): int8 copies of q, k and v, three scale arrays, the head

@@ -27,6 +27,7 @@ EXPORTED = ("intattn_derive_params", "intattn_forward", "intattn_forward_variant
             "intattn_calibrate_workspace_size", "intattn_calibrate_clip",
             "intattn_forward_host", "intattn_decode_workspace_size",
             "intattn_decode", "intattn_decode_int4", "intattn_decode_static_scratch", "intattn_quantize",
+            "intattn_quantize_zp",
             "intattn_gelu_derive_params", "intattn_gelu", "intattn_selftest_timeout", "intattn_device_error",
             "intattn_strerror")
 DTYPE_FP16, DTYPE_BF16 = 0, 1
@@ -51,7 +52,9 @@ class _Scales(ctypes.Structure):
                 ("s_k", ctypes.POINTER(ctypes.c_float)),
                 ("s_v", ctypes.POINTER(ctypes.c_float)),
                 ("s_o", ctypes.POINTER(ctypes.c_float)),
-                ("clip_c", ctypes.POINTER(ctypes.c_float))]
+                ("clip_c", ctypes.POINTER(ctypes.c_float)),
+                ("z_k", ctypes.POINTER(ctypes.c_int32)),
+                ("z_v", ctypes.POINTER(ctypes.c_int32))]
 
 
 class _HeadParams(ctypes.Structure):
@@ -66,13 +69,17 @@ FloatArg = Union[float, Sequence[float], np.ndarray]
 class Scales:
     """Quantisation scales (real = scale * code).  per_head: arrays of H.
     clip: optional per-head clip thresholds (same layout as the scales);
-    None: the call's clip_c applies to every head."""
+    None: the call's clip_c applies to every head.
+    z_k / z_v: optional zero-points (same layout, 0..255): the K / V codes
+    are then uint8 tensors and code c stands for c - z."""
     s_q: FloatArg
     s_k: FloatArg
     s_v: FloatArg
     s_o: FloatArg
     per_head: bool = False
     clip: Optional[FloatArg] = None
+    z_k: Optional[FloatArg] = None
+    z_v: Optional[FloatArg] = None
 
     def _c(self):
         arrs = [np.ascontiguousarray(np.atleast_1d(np.asarray(x, dtype=np.float32)))
@@ -82,8 +89,17 @@ class Scales:
         if self.clip is not None:
             clip = np.ascontiguousarray(np.atleast_1d(np.asarray(self.clip, dtype=np.float32)))
             arrs.append(clip)
+        ip = ctypes.POINTER(ctypes.c_int32)
+        zs = []
+        for z in (self.z_k, self.z_v):
+            if z is None:
+                zs.append(ip())
+            else:
+                za = np.ascontiguousarray(np.atleast_1d(np.asarray(z)).astype(np.int32))
+                arrs.append(za)
+                zs.append(za.ctypes.data_as(ip))
         s = _Scales(int(bool(self.per_head)), *[a.ctypes.data_as(fp) for a in arrs[:4]],
-                    clip.ctypes.data_as(fp) if clip is not None else fp())
+                    clip.ctypes.data_as(fp) if clip is not None else fp(), *zs)
         return s, arrs  # keep the arrays alive for the duration of the call
 
 
@@ -128,6 +144,7 @@ def lib() -> ctypes.CDLL:
         L.intattn_decode_static_scratch.argtypes = [vp, vp, vp, ctypes.POINTER(_Scales), i32, i32, i32,
                                                     i32, i32, f32, vp, vp]
         L.intattn_quantize.argtypes = [vp, i32, i32, i32, i32, i32, i32, vp, vp, vp]
+        L.intattn_quantize_zp.argtypes = [vp, i32, i32, i32, i32, i32, i32, vp, vp, vp, vp]
         L.intattn_gelu_derive_params.argtypes = [f32, f32, f32, ctypes.POINTER(_GeluParams)]
         L.intattn_gelu.argtypes = [vp, vp, ctypes.c_longlong, f32, f32, f32, vp]
         L.intattn_selftest_timeout.argtypes = [vp]
@@ -174,13 +191,25 @@ def _check_tensor(t, name: str):
         raise ValueError(f"{name} must be contiguous")
 
 
+def _check_codes(t, name: str, zero_point, cuda: bool = True):
+    """K or V codes: uint8 when the tensor has a zero-point, else int8."""
+    import torch
+    want = torch.uint8 if zero_point is not None else torch.int8
+    if not isinstance(t, torch.Tensor) or t.dtype != want or t.is_cuda != cuda:
+        raise TypeError(f"{name} must be a {'CUDA' if cuda else 'CPU'} {want} tensor"
+                        + (" (it has a zero-point)" if zero_point is not None else ""))
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+
+
 def forward(q, k, v, scales: Scales, causal: bool, clip_c: float, out=None, stream=None, variant: int = 0):
     """out[B,H,Lq,d] int8 = IntAttention forward of int8 q[B,H,Lq,d], k/v[B,H,Lk,d].
     variant: VARIANT_AUTO (intattn_forward), VARIANT_THREE_PASS or
     VARIANT_SHORT_ROWS (intattn_forward_variant); the bytes are the same."""
     import torch
-    for t, n in ((q, "q"), (k, "k"), (v, "v")):
-        _check_tensor(t, n)
+    _check_tensor(q, "q")
+    _check_codes(k, "k", scales.z_k)
+    _check_codes(v, "v", scales.z_v)
     B, H, Lq, d = q.shape
     Lk = k.shape[2]
     if k.shape != (B, H, Lk, d) or v.shape != k.shape:
@@ -215,9 +244,10 @@ def forward_host(q, k, v, scales: Scales, causal: bool, clip_c: float, out=None,
     consecutive calls with one workspace overlap.  Returns out (a CPU tensor,
     valid once `stream` has reached the end of the call)."""
     import torch
-    for t, name in ((q, "q"), (k, "k"), (v, "v")):
-        if not isinstance(t, torch.Tensor) or t.dtype != torch.int8 or t.is_cuda or not t.is_contiguous():
-            raise TypeError(f"{name} must be a contiguous CPU int8 tensor")
+    if not isinstance(q, torch.Tensor) or q.dtype != torch.int8 or q.is_cuda or not q.is_contiguous():
+        raise TypeError("q must be a contiguous CPU int8 tensor")
+    _check_codes(k, "k", scales.z_k, cuda=False)
+    _check_codes(v, "v", scales.z_v, cuda=False)
     B, H, Lq, d = q.shape
     Lk = k.shape[2]
     if k.shape != (B, H, Lk, d) or v.shape != k.shape:
@@ -277,6 +307,10 @@ def forward_fp(q, k, v, per_head: bool, s_o, causal: bool, clip_c: float, clip=N
     return out
 
 
+def calibrate_workspace_size(B: int, H: int) -> int:
+    return int(lib().intattn_calibrate_workspace_size(int(B), int(H)))
+
+
 def calibrate_clip(q, k, scales: Scales, causal: bool, keep: int, stride: int, c_min: float = 0.25,
                    c_max: float = 64.0, workspace=None, stream=None):
     """intattn_calibrate_clip: (thresholds float32 [H or 1], gaps int32 [H or 1])
@@ -313,8 +347,9 @@ def decode(q, k_cache, v_cache, scales: Scales, Lk: int, clip_c: float, out=None
            stream=None):
     """out[B,H,1,d] int8: one query per (b, h) over the first Lk rows of the caches."""
     import torch
-    for t, n in ((q, "q"), (k_cache, "k_cache"), (v_cache, "v_cache")):
-        _check_tensor(t, n)
+    _check_tensor(q, "q")
+    _check_codes(k_cache, "k_cache", scales.z_k)
+    _check_codes(v_cache, "v_cache", scales.z_v)
     B, H, one, d = q.shape
     if one != 1:
         raise ValueError("decode takes one query per (b, h): q is [B, H, 1, d]")
@@ -399,6 +434,37 @@ def quantize(x, per_head: bool, out=None, scales=None, stream=None):
     _check(lib().intattn_quantize(x.data_ptr(), dt, B, H, L, d, int(bool(per_head)), out.data_ptr(),
                                   scales.data_ptr(), _stream_handle(stream, x.device)), "intattn_quantize")
     return out, scales
+
+
+def quantize_zp(x, per_head: bool, out=None, scales=None, zero_points=None, stream=None):
+    """u8 codes, device scales and device zero-points of an fp16 / bf16 CUDA
+    tensor [B, H, L, d] (asymmetric, dynamic, per tensor or per head)."""
+    import torch
+    if not isinstance(x, torch.Tensor) or not x.is_cuda or x.dtype not in (torch.float16, torch.bfloat16):
+        raise TypeError("x must be a CUDA float16 or bfloat16 tensor")
+    if not x.is_contiguous() or x.dim() != 4:
+        raise ValueError("x must be a contiguous [B, H, L, d] tensor")
+    B, H, L, d = x.shape
+    if out is None:
+        out = torch.empty(x.shape, dtype=torch.uint8, device=x.device)
+    if not isinstance(out, torch.Tensor) or out.dtype != torch.uint8 or not out.is_cuda or not out.is_contiguous():
+        raise TypeError("out must be a contiguous CUDA uint8 tensor")
+    if out.shape != x.shape:
+        raise ValueError("out must match x")
+    n = H if per_head else 1
+    if scales is None:
+        scales = torch.empty(n, dtype=torch.float32, device=x.device)
+    if zero_points is None:
+        zero_points = torch.empty(n, dtype=torch.int32, device=x.device)
+    if scales.dtype != torch.float32 or not scales.is_cuda or scales.numel() < n:
+        raise ValueError(f"scales must be a CUDA float32 tensor of at least {n} entries")
+    if zero_points.dtype != torch.int32 or not zero_points.is_cuda or zero_points.numel() < n:
+        raise ValueError(f"zero_points must be a CUDA int32 tensor of at least {n} entries")
+    dt = DTYPE_BF16 if x.dtype == torch.bfloat16 else DTYPE_FP16
+    _check(lib().intattn_quantize_zp(x.data_ptr(), dt, B, H, L, d, int(bool(per_head)), out.data_ptr(),
+                                     scales.data_ptr(), zero_points.data_ptr(), _stream_handle(stream, x.device)),
+           "intattn_quantize_zp")
+    return out, scales, zero_points
 
 
 def gelu_params(s_x: float, s_y: float, c: float):

@@ -21,6 +21,10 @@
 // u = x + 8 of its even and of its odd channels (nibble ^ 8: one logic op
 // per 4 channels); dp4a works on u and the bias is removed exactly:
 // q.x = q.u - 8 sum(q), and sum P x = sum P u - 8 sum(P).
+// Zero-points (int8 cache only): u8 K codes need only the dp4a operand type
+// (the per-row constant q.z_k cancels in every gap); u8 V codes with
+// zero-point z_v give sum P (v - z_v) = sum P v - z_v sum P, with sum P
+// found by decode_z in a second sweep over the scores once R is known.
 #pragma once
 #include <climits>
 #include <cstdint>
@@ -39,8 +43,9 @@ struct DecodeArgs {
   int32_t* ws_max;   // [BH, nsplit]      chunk maxima
   int32_t* ws_part;  // [BH, nsplit, d]   partial P.V sums
   uint32_t* ws_cnt;  // [BH]              arrival tickets
-  int32_t* ws_mr;    // [BH, 2]           row max and reciprocal R
+  int32_t* ws_mr;    // [BH, 4]           row max, reciprocal R, sum of P (V zero-point only)
   int32_t BH, H, Lk, Lmax, nsplit, chunk, per_head, ld_s;
+  int32_t k_u8, v_u8;  // int8 cache: K / V codes are u8 (they carry zero-points)
   uint32_t lut[INTATTN_MAX_CLIPS][32];  // one exp table per distinct clip threshold
   HeadParamsDev hp[INTATTN_MAX_HEADS];
 };
@@ -106,7 +111,7 @@ struct Layout {
   static_assert(kChunk % kRowsPerStep == 0, "chunk must be whole steps");
 };
 
-template <int D>
+template <int D, bool KU8>
 __global__ void __launch_bounds__(kThreads) decode_qk_kernel(const __grid_constant__ DecodeArgs a) {
   using Lt = Layout<D>;
   const int bh = blockIdx.y;
@@ -137,10 +142,17 @@ __global__ void __launch_bounds__(kThreads) decode_qk_kernel(const __grid_consta
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
       int32_t acc = 0;
-      acc = dp4a_ss(kv[i].x, qv.x, acc);
-      acc = dp4a_ss(kv[i].y, qv.y, acc);
-      acc = dp4a_ss(kv[i].z, qv.z, acc);
-      acc = dp4a_ss(kv[i].w, qv.w, acc);
+      if constexpr (KU8) {  // s8 q times u8 K codes
+        acc = dp4a_su(qv.x, kv[i].x, acc);
+        acc = dp4a_su(qv.y, kv[i].y, acc);
+        acc = dp4a_su(qv.z, kv[i].z, acc);
+        acc = dp4a_su(qv.w, kv[i].w, acc);
+      } else {
+        acc = dp4a_ss(kv[i].x, qv.x, acc);
+        acc = dp4a_ss(kv[i].y, qv.y, acc);
+        acc = dp4a_ss(kv[i].z, qv.z, acc);
+        acc = dp4a_ss(kv[i].w, qv.w, acc);
+      }
       s[i] = acc;
     }
     // reduce the CPR partial sums of each of the 4 rows (transpose-reduce)
@@ -237,17 +249,40 @@ __global__ void __launch_bounds__(kThreads) decode_z_kernel(const __grid_constan
   for (int o = 16; o > 0; o >>= 1) z += __shfl_xor_sync(0xffffffffu, z, o);
   if (lane == 0) red[tid >> 5] = z;
   __syncthreads();
+  __shared__ uint32_t R_s;
   if (tid == 0) {
     int32_t Z = 0;
     for (int w = 0; w < kThreads / 32; ++w) Z += red[w];
     const unsigned long long R =
         ((255ull << 32) + static_cast<unsigned long long>(Z >> 1)) / static_cast<unsigned long long>(Z);
-    a.ws_mr[2 * bh] = m;
-    a.ws_mr[2 * bh + 1] = static_cast<int32_t>(R);
+    a.ws_mr[4 * bh] = m;
+    a.ws_mr[4 * bh + 1] = static_cast<int32_t>(R);
+    R_s = static_cast<uint32_t>(R);
+  }
+  if (hp.zv == 0) return;
+  // V zero-point: sum_j P_j over the row, P_j from the same table as decode_pv
+  __shared__ uint32_t ptab_s[32];
+  __syncthreads();
+  if (tid < 32)
+    ptab_s[tid] = static_cast<uint32_t>((static_cast<unsigned long long>(lut_s[tid]) * R_s + (1ull << 31)) >> 32);
+  __syncthreads();
+  int32_t ps = 0;
+  for (int j = tid; j < a.Lk; j += kThreads) {
+    const int32_t t = imax32(__ldcg(a.ws_s + static_cast<size_t>(bh) * a.ld_s + j), lo);
+    ps += static_cast<int32_t>(ptab_s[(Cm - static_cast<uint32_t>(t) * Mu) >> sh]);
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) ps += __shfl_xor_sync(0xffffffffu, ps, o);
+  if (lane == 0) red[tid >> 5] = ps;
+  __syncthreads();
+  if (tid == 0) {
+    int32_t P = 0;
+    for (int w = 0; w < kThreads / 32; ++w) P += red[w];
+    a.ws_mr[4 * bh + 2] = P;
   }
 }
 
-template <int D>
+template <int D, bool VU8>
 __global__ void __launch_bounds__(kThreads) decode_pv_kernel(const __grid_constant__ DecodeArgs a) {
   using Lt = Layout<D>;
   const int bh = blockIdx.y;
@@ -263,8 +298,8 @@ __global__ void __launch_bounds__(kThreads) decode_pv_kernel(const __grid_consta
   __shared__ int32_t part[16 * kPartStride];       // per-thread partial sums, [channel][thread]
   __shared__ int last_flag;
 
-  const int32_t m = __ldcg(a.ws_mr + 2 * bh);
-  const unsigned long long R = static_cast<uint32_t>(__ldcg(a.ws_mr + 2 * bh + 1));
+  const int32_t m = __ldcg(a.ws_mr + 4 * bh);
+  const unsigned long long R = static_cast<uint32_t>(__ldcg(a.ws_mr + 4 * bh + 1));
   if (tid < 32)
     ptab_s[tid] = static_cast<uint32_t>((static_cast<unsigned long long>(a.lut[hp.lut][tid]) * R + (1ull << 31)) >> 32);
   const long long lo64 = static_cast<long long>(m) - hp.D;
@@ -326,10 +361,17 @@ __global__ void __launch_bounds__(kThreads) decode_pv_kernel(const __grid_consta
       const uint32_t ab_hi = __byte_perm(w0[q], w1[q], 0x7362);
       const uint32_t cd_lo = __byte_perm(w2[q], w3[q], 0x5140);
       const uint32_t cd_hi = __byte_perm(w2[q], w3[q], 0x7362);
-      acc[4 * q + 0] = dp4a_su(__byte_perm(ab_lo, cd_lo, 0x5410), p4, acc[4 * q + 0]);
-      acc[4 * q + 1] = dp4a_su(__byte_perm(ab_lo, cd_lo, 0x7632), p4, acc[4 * q + 1]);
-      acc[4 * q + 2] = dp4a_su(__byte_perm(ab_hi, cd_hi, 0x5410), p4, acc[4 * q + 2]);
-      acc[4 * q + 3] = dp4a_su(__byte_perm(ab_hi, cd_hi, 0x7632), p4, acc[4 * q + 3]);
+      if constexpr (VU8) {  // u8 V codes
+        acc[4 * q + 0] = dp4a_uu(__byte_perm(ab_lo, cd_lo, 0x5410), p4, acc[4 * q + 0]);
+        acc[4 * q + 1] = dp4a_uu(__byte_perm(ab_lo, cd_lo, 0x7632), p4, acc[4 * q + 1]);
+        acc[4 * q + 2] = dp4a_uu(__byte_perm(ab_hi, cd_hi, 0x5410), p4, acc[4 * q + 2]);
+        acc[4 * q + 3] = dp4a_uu(__byte_perm(ab_hi, cd_hi, 0x7632), p4, acc[4 * q + 3]);
+      } else {
+        acc[4 * q + 0] = dp4a_su(__byte_perm(ab_lo, cd_lo, 0x5410), p4, acc[4 * q + 0]);
+        acc[4 * q + 1] = dp4a_su(__byte_perm(ab_lo, cd_lo, 0x7632), p4, acc[4 * q + 1]);
+        acc[4 * q + 2] = dp4a_su(__byte_perm(ab_hi, cd_hi, 0x5410), p4, acc[4 * q + 2]);
+        acc[4 * q + 3] = dp4a_su(__byte_perm(ab_hi, cd_hi, 0x7632), p4, acc[4 * q + 3]);
+      }
     }
     if (more) {
 #pragma unroll
@@ -361,6 +403,7 @@ __global__ void __launch_bounds__(kThreads) decode_pv_kernel(const __grid_consta
       int32_t tot = 0;
       const int32_t* p0 = a.ws_part + static_cast<size_t>(bh) * a.nsplit * D + tid;
       for (int i = 0; i < a.nsplit; ++i) tot += __ldcg(p0 + static_cast<size_t>(i) * D);
+      if (hp.zv != 0) tot -= hp.zv * __ldcg(a.ws_mr + 4 * bh + 2);  // sum P (v - z_v)
       const long long t = static_cast<long long>(tot) * hp.Mo + (1ll << (hp.so - 1));
       long long y = t >> hp.so;
       y = y > 127 ? 127 : (y < -127 ? -127 : y);
@@ -529,8 +572,8 @@ __global__ void __launch_bounds__(kThreads, 3) decode4_pv_kernel(const __grid_co
     m = __ldcg(a.ws_max + bh);  // the only chunk's maximum
     if (tid < 32) ptab_s[tid] = a.lut[hp.lut][tid];  // the exp table until R is known
   } else {
-    m = __ldcg(a.ws_mr + 2 * bh);
-    const unsigned long long R = static_cast<uint32_t>(__ldcg(a.ws_mr + 2 * bh + 1));
+    m = __ldcg(a.ws_mr + 4 * bh);
+    const unsigned long long R = static_cast<uint32_t>(__ldcg(a.ws_mr + 4 * bh + 1));
     if (tid < 32)
       ptab_s[tid] = static_cast<uint32_t>((static_cast<unsigned long long>(a.lut[hp.lut][tid]) * R + (1ull << 31)) >> 32);
   }

@@ -106,6 +106,10 @@ int derive(const intattn_scales_t* sc, int H, int d, float clip_c, uint32_t lut[
     rc = requant_params(sc->s_v[i], sc->s_o[i], &hp[i]);
     if (rc) return rc;
     hp[i].lut = id;
+    // zero-points: u8 codes, 0 .. 255 (K's cancels in every gap: checked only)
+    if (sc->z_k && (sc->z_k[i] < 0 || sc->z_k[i] > 255)) return INTATTN_ERR_INVALID_ARG;
+    if (sc->z_v && (sc->z_v[i] < 0 || sc->z_v[i] > 255)) return INTATTN_ERR_INVALID_ARG;
+    hp[i].zv = sc->z_v ? sc->z_v[i] : 0;
   }
   if (n_luts) *n_luts = nclips;
   return INTATTN_OK;
@@ -234,7 +238,7 @@ DecodeLayout decode_layout(long long BH, int Lk, int d, int chunk = intattn::dec
   L.off_part = L.off_max + round256(static_cast<size_t>(BH) * L.nsplit * 4);
   L.off_cnt = L.off_part + round256(static_cast<size_t>(BH) * L.nsplit * d * 4);
   L.off_mr = L.off_cnt + round256(static_cast<size_t>(BH) * 4);
-  L.total = L.off_mr + round256(static_cast<size_t>(BH) * 8);
+  L.total = L.off_mr + round256(static_cast<size_t>(BH) * 16);
   return L;
 }
 
@@ -244,7 +248,10 @@ int decode_launch(const DecodeArgs& a, cudaStream_t stream) {
   if constexpr (kInt4) {
     intattn::decode::decode4_qk_kernel<D><<<grid, intattn::decode::kThreads, 0, stream>>>(a);
   } else {
-    intattn::decode::decode_qk_kernel<D><<<grid, intattn::decode::kThreads, 0, stream>>>(a);
+    if (a.k_u8)
+      intattn::decode::decode_qk_kernel<D, true><<<grid, intattn::decode::kThreads, 0, stream>>>(a);
+    else
+      intattn::decode::decode_qk_kernel<D, false><<<grid, intattn::decode::kThreads, 0, stream>>>(a);
   }
   const int rc = note_launch(cudaGetLastError());
   if (rc != INTATTN_OK) return rc;
@@ -259,7 +266,10 @@ int decode_launch(const DecodeArgs& a, cudaStream_t stream) {
   if constexpr (kInt4) {
     intattn::decode::decode4_pv_kernel<D, false><<<grid, intattn::decode::kThreads, 0, stream>>>(a);
   } else {
-    intattn::decode::decode_pv_kernel<D><<<grid, intattn::decode::kThreads, 0, stream>>>(a);
+    if (a.v_u8)
+      intattn::decode::decode_pv_kernel<D, true><<<grid, intattn::decode::kThreads, 0, stream>>>(a);
+    else
+      intattn::decode::decode_pv_kernel<D, false><<<grid, intattn::decode::kThreads, 0, stream>>>(a);
   }
   return note_launch(cudaGetLastError());
 }
@@ -341,6 +351,8 @@ int decode_setup(const int8_t* q, const int8_t* k_cache, const int8_t* v_cache, 
   a->ld_s = L->ld_s;
   a->chunk = chunk;
   a->per_head = scales->per_head ? 1 : 0;
+  a->k_u8 = scales->z_k ? 1 : 0;
+  a->v_u8 = scales->z_v ? 1 : 0;
   return INTATTN_OK;
 }
 
@@ -487,6 +499,8 @@ int intattn_forward_variant(const int8_t* q, const int8_t* k, const int8_t* v, c
   int rc = derive(scales, H, d, clip_c, args.lut, args.hp, INTATTN_MAX_HEADS, &args.n_luts);
   if (rc) return rc;
   args.per_head = scales->per_head ? 1 : 0;
+  args.k_u8 = scales->z_k ? 1 : 0;
+  args.v_u8 = scales->z_v ? 1 : 0;
   return forward_launch(q, k, v, args, B, H, Lq, Lk, d, causal, out, variant, reinterpret_cast<cudaStream_t>(stream));
 }
 
@@ -789,6 +803,7 @@ int intattn_decode(const int8_t* q, const int8_t* k_cache, const int8_t* v_cache
 int intattn_decode_int4(const int8_t* q, const uint8_t* k_cache, const uint8_t* v_cache,
                         const intattn_scales_t* scales, int B, int H, int Lk, int Lmax, int d, float clip_c,
                         int8_t* out, void* workspace, size_t workspace_bytes, intattn_stream_t stream) {
+  if (scales && (scales->z_k || scales->z_v)) return INTATTN_ERR_UNSUPPORTED;  // int4 codes: no zero-points
   DecodeArgs a;
   DecodeLayout L{};
   bool empty = false;
@@ -825,29 +840,34 @@ int intattn_decode_static_scratch(const int8_t* q, const int8_t* k_cache, const 
   return d == 64 ? decode_launch<64>(a, st) : decode_launch<128>(a, st);
 }
 
-int intattn_quantize(const void* x, int dtype, int B, int H, int L, int d, int per_head, int8_t* out,
-                     float* scales, intattn_stream_t stream) {
+namespace {
+
+// intattn_quantize (zero_points == nullptr) and intattn_quantize_zp.
+int quantize_impl(const void* x, int dtype, int B, int H, int L, int d, int per_head, void* out, float* scales,
+                  int32_t* zero_points, cudaStream_t st) {
   if (B < 0 || H <= 0 || L < 0 || d <= 0) return INTATTN_ERR_INVALID_ARG;
   if (dtype != INTATTN_DTYPE_FP16 && dtype != INTATTN_DTYPE_BF16) return INTATTN_ERR_UNSUPPORTED;
   if (!scales) return INTATTN_ERR_INVALID_ARG;
   const long long slice = static_cast<long long>(L) * d;
   if (slice % intattn::quant::kVec) return INTATTN_ERR_UNSUPPORTED;  // whole 16-byte vectors per (b, h)
   if (reinterpret_cast<uintptr_t>(scales) & 3u) return INTATTN_ERR_UNSUPPORTED;
+  if (zero_points && (reinterpret_cast<uintptr_t>(zero_points) & 3u)) return INTATTN_ERR_UNSUPPORTED;
   const long long BH = static_cast<long long>(B) * H;
   const int n_scales = per_head ? H : 1;
-  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  uint32_t* nmax = reinterpret_cast<uint32_t*>(zero_points);
   if (BH == 0 || slice == 0) {
-    // no elements: amax 0 -> every scale is 1
-    if (note_launch(cudaMemsetAsync(scales, 0, n_scales * sizeof(float), st))) return INTATTN_ERR_CUDA;
-    intattn::quant::quant_scales_kernel<<<1, 128, 0, st>>>(reinterpret_cast<uint32_t*>(scales), n_scales);
+    // no elements: every scale is 1 (and every zero-point 0)
+    intattn::quant::quant_scales_kernel<<<1, 128, 0, st>>>(reinterpret_cast<uint32_t*>(scales), nmax, n_scales);
     return note_launch(cudaGetLastError());
   }
   if (!x || !out) return INTATTN_ERR_INVALID_ARG;
   if (!aligned16(x) || !aligned16(out)) return INTATTN_ERR_UNSUPPORTED;
   intattn::QuantArgs a;
   a.x = x;
-  a.out = out;
+  a.out = static_cast<int8_t*>(out);
   a.amax = reinterpret_cast<uint32_t*>(scales);
+  a.nmax = nmax;
+  a.asym = nmax ? 1 : 0;
   a.nvec = BH * (slice / intattn::quant::kVec);
   a.seg = per_head ? slice / intattn::quant::kVec : a.nvec;
   a.H = H;
@@ -864,7 +884,7 @@ int intattn_quantize(const void* x, int dtype, int B, int H, int L, int d, int p
     return note_launch(cudaGetLastError());
   const long long want = (a.nvec + intattn::quant::kThreads - 1) / intattn::quant::kThreads;
   const unsigned grid = static_cast<unsigned>(std::min<long long>(want, static_cast<long long>(sms) * occ));
-  intattn::quant::quant_zero_kernel<<<1, 128, 0, st>>>(a.amax, n_scales, reinterpret_cast<uint32_t*>(out));
+  intattn::quant::quant_zero_kernel<<<1, 128, 0, st>>>(a.amax, a.nmax, n_scales, reinterpret_cast<uint32_t*>(out));
   const int rc = note_launch(cudaGetLastError());
   if (rc) return rc;
   // cooperative: all CTAs resident (the grid barrier); programmatic
@@ -881,6 +901,20 @@ int intattn_quantize(const void* x, int dtype, int B, int H, int L, int d, int p
   cfg.attrs = attrs;
   cfg.numAttrs = 2;
   return note_launch(cudaLaunchKernelEx(&cfg, intattn::quant::quant_fused_kernel, a));
+}
+
+}  // namespace
+
+int intattn_quantize(const void* x, int dtype, int B, int H, int L, int d, int per_head, int8_t* out,
+                     float* scales, intattn_stream_t stream) {
+  return quantize_impl(x, dtype, B, H, L, d, per_head, out, scales, nullptr, reinterpret_cast<cudaStream_t>(stream));
+}
+
+int intattn_quantize_zp(const void* x, int dtype, int B, int H, int L, int d, int per_head, uint8_t* out,
+                        float* scales, int32_t* zero_points, intattn_stream_t stream) {
+  if (!zero_points) return INTATTN_ERR_INVALID_ARG;
+  return quantize_impl(x, dtype, B, H, L, d, per_head, out, scales, zero_points,
+                       reinterpret_cast<cudaStream_t>(stream));
 }
 
 namespace {
@@ -975,6 +1009,7 @@ int intattn_calibrate_clip(const int8_t* q, const int8_t* k, const intattn_scale
   if (causal && Lq > Lk) return INTATTN_ERR_INVALID_ARG;
   if (d != 64 && d != 128) return INTATTN_ERR_UNSUPPORTED;
   if (!scales || !scales->s_q || !scales->s_k || !clip_out) return INTATTN_ERR_INVALID_ARG;
+  if (scales->z_k || scales->z_v) return INTATTN_ERR_UNSUPPORTED;  // int8 codes only
   if (!std::isfinite(c_min) || !std::isfinite(c_max) || !(c_min > 0.0f) || !(c_max >= c_min))
     return INTATTN_ERR_PARAM_RANGE;
   const int n = scales->per_head ? H : 1;

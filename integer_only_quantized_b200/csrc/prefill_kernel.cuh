@@ -38,6 +38,14 @@
 // S is recomputed by the tensor cores in each pass; K streams three times
 // (from L2 after the first), V once.
 //
+// Zero-points (K and / or V as u8 codes with a zero-point per tensor or
+// head): S = Q.(K - z_k) differs from Q.K_code by a per-row constant, which
+// cancels in every gap m - S, so the kernel runs on the codes (the MMA reads K
+// as u8).  P.(V - z_v) = P.V_code - z_v sum_j P_j: pass C also sums each
+// thread's P bytes, each team then writes one correction P tile (see
+// zv_correction_bytes) and the MMA warp adds it against a constant tile
+// after the tile's last P.V.
+//
 // Every mbarrier wait is bounded (polls with a time limit).  Each softmax
 // warp polls its own barriers (one vote per poll).  A warp whose wait runs
 // out leaves its pass loop; every softmax warp still reaches the same
@@ -69,6 +77,7 @@ struct PrefillArgs {
   // status of that derivation: the kernel writes nothing unless it is 0
   const HeadParamsDev* hp_dev;
   const uint32_t* status;
+  int32_t k_u8, v_u8;  // K / V codes are u8 (they carry zero-points), else int8
 };
 
 namespace prefill {
@@ -132,10 +141,14 @@ struct Cfg {
   static constexpr int kNumBars = kBarKvFull + 2 * kStages;
   static constexpr uint32_t kOffQ = 0;                                  // [2] Q tiles
   static constexpr uint32_t kOffKV = kOffQ + 2 * kQBytes;
+  // constant s8 tile [32 keys][D] of the V zero-point correction (rows 16 g:
+  // -1, rows 16 g + 1 .. 16 g + 4: -128, else 0), laid out like a V tile
+  static constexpr uint32_t kOffCorr = kOffKV + kStages * kTileBytes;
+  static constexpr int kCorrGroup = 16;  // keys of a correction tile per partial owner (two per team)
   // probability table, four copies [b][33][kBM] u32 with P << 8b, so four
   // looked-up bytes pack into a word by integer adds
   static constexpr uint32_t kPtabBytes = 33 * kBM * 4;
-  static constexpr uint32_t kOffPtab = kOffKV + kStages * kTileBytes;
+  static constexpr uint32_t kOffPtab = kOffCorr + 32 * D;
   static constexpr uint32_t kOffRed = kOffPtab + 4 * kPtabBytes;        // [2][kGroups][kBM] int32
   static constexpr uint32_t kOffLut = kOffRed + 2 * kGroups * kBM * 4;
   static constexpr uint32_t kOffHp = kOffLut + INTATTN_MAX_CLIPS * 32 * 4;  // head parameters
@@ -279,6 +292,15 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_kernel(const __grid_const
   // head parameters in shared memory: a dynamically indexed kernel argument
   // is a constant-bank load that can miss
   for (int i = tid; i < (args.per_head ? args.H : 1); i += blockDim.x) hp_s[i] = args.hp_dev ? args.hp_dev[i] : args.hp[i];
+  {
+    // the zero-point correction tile (uniform rows: the swizzle moves bytes within a row only)
+    uint32_t* corr = reinterpret_cast<uint32_t*>(smem + C::kOffCorr);
+    for (int i = tid; i < 8 * D; i += blockDim.x) {
+      const int key = (4 * i) / D % C::kCorrGroup;
+      corr[i] = key == 0 ? 0xFFFFFFFFu : (key <= 4 ? 0x80808080u : 0u);
+    }
+    fence_proxy_async_smem();
+  }
   if (warp == kMmaWarp) {
     tmem_alloc(smem_u32(tmem_slot), kTmemCols);
     tmem_relinquish();
@@ -475,6 +497,8 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_kernel(const __grid_const
       all_sync(true);  // the table is complete
 
       // ---- pass C: P tiles into TMEM for the P.V MMAs ----
+      const bool corr = hp.zv != 0;  // V zero-point: sum this thread's P bytes
+      uint32_t psum = 0;
       for (int j = first_j(sc); j < T.nkt; j += kTeams) {
         const uint32_t pi = pc + j;  // running P index of this tile
         const uint32_t pb = pi & (kPBufs - 1);
@@ -507,6 +531,10 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_kernel(const __grid_const
               pw[q] = (p[0] + p[1]) + (p[2] + p[3]);
             }
           }
+          if (corr) {
+#pragma unroll
+            for (int q = 0; q < 8; ++q) psum = __dp4a(pw[q], 0x01010101u, psum);
+          }
           tmem_st8(tlane + kColP + pb * 32 + half * (kCols / 4) + c * 8, pw);
         });
         if (!got) { ok = false; break; }
@@ -514,8 +542,24 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_kernel(const __grid_const
         tc_fence_before();
         arrive_warp(bar(kBarPFull + pb));
       }
+      if (corr && ok) {
+        // this team's correction tile: P index pc + nkt + team, keys
+        // kCorrGroup * half .. of it hold this thread's share
+        const uint32_t pi = pc + T.nkt + team;
+        const uint32_t pb = pi & (kPBufs - 1);
+        if (!team_wait(bar(kBarPEmpty + pb), ((pi / kPBufs) & 1) ^ 1)) {
+          ok = false;
+        } else {
+          uint32_t w0, w1;
+          zv_correction_bytes(hp.zv * static_cast<int32_t>(psum), w0, w1);
+          tmem_st4(tlane + kColP + pb * 32 + half * (C::kCorrGroup / 4), w0, w1, 0u, 0u);
+          tmem_wait_st();
+          tc_fence_before();
+          arrive_warp(bar(kBarPFull + pb));
+        }
+      }
       sc += T.nkt;
-      pc += T.nkt;
+      pc += T.nkt + (corr ? kTeams : 0);
 
     }
   } else if (warp >= kEpiWarp0) {
@@ -627,9 +671,11 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_kernel(const __grid_const
     // The whole warp runs this loop on uniform values (descriptors stay in
     // uniform registers) and waits for both inputs of an MMA group with one
     // vote per poll; one elected lane issues the group and its commits.
-    constexpr uint32_t idesc_qk = idesc_i8(kBM, kBN, 1, 1, 0);  // s8 x s8, K-major B
-    constexpr uint32_t idesc_pv = idesc_i8(kBM, D, 0, 1, 1);    // u8 x s8, N-major B
+    const uint32_t idesc_qk = idesc_i8(kBM, kBN, 1, args.k_u8 ? 0u : 1u, 0);  // s8 x (s8 | u8), K-major B
+    const uint32_t idesc_pv = idesc_i8(kBM, D, 0, args.v_u8 ? 0u : 1u, 1);    // u8 x (s8 | u8), N-major B
+    constexpr uint32_t idesc_corr = idesc_i8(kBM, D, 0, 1, 1);                // u8 x s8: the correction tile
     const uint64_t kv_desc0 = smem_desc(sKV, 16, C::kSBO, C::kSwizzle);
+    const uint64_t corr_desc = smem_desc(s_base + C::kOffCorr, 16, C::kSBO, C::kSwizzle);
     constexpr uint32_t kSlotDesc = C::kTileBytes >> 4;  // descriptor step between ring slots
     bool ok = true;
     uint32_t slot = 0, kv_par = 0;  // ring slot and phase parity of the next K/V tile
@@ -702,6 +748,23 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_kernel(const __grid_const
         next_slot();
       }
       if (!ok) break;
+      if (hp_s[args.per_head ? T.h : 0].zv != 0) {
+        // O -= z_v sum_j P_j: one correction tile per softmax team
+        for (int t = 0; t < kTeams; ++t, ++pc) {
+          const uint32_t pb = pc & (kPBufs - 1);
+          if (!mbar_wait_warp(bar(kBarPFull + pb), (pc / kPBufs) & 1, kRoleMma)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          if (elect_one()) {
+            mma_i8_ts(tmem + kColO + (it % C::kOBufs) * D, tmem + kColP + pb * 32, corr_desc, idesc_corr, 1u);
+            mma_commit(bar(kBarPEmpty + pb));
+          }
+          __syncwarp();
+        }
+        if (!ok) break;
+      }
       mma_commit_elect(bar(kBarQEmpty + qb));  // every MMA that read this Q buffer
       mma_commit_elect(bar(kBarOFull + it % C::kOBufs));
     }

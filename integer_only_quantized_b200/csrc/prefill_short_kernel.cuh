@@ -15,6 +15,9 @@
 // (Kept in shared memory instead, one byte of index code per key costs more
 // to pack and unpack, at 2 cycles per byte permute, than recomputing the
 // index from the resident scores, at 3 full-rate instructions per key.)
+// Zero-points of K and V as in prefill_kernel.cuh: u8 K needs nothing but
+// the MMA's operand type; a V zero-point adds one correction P tile per
+// query tile (the four column groups' shares of sum_j P_j).
 // Work unit and schedule: one (batch, head, 128-query tile), persistent CTAs
 // in snake order over the tiles sorted longest first (causal).
 // Warp roles (22 warps):
@@ -97,9 +100,13 @@ struct Cfg {
   static constexpr int kNumBars = kBarKvFull + 2 * kStages;
   static constexpr uint32_t kOffQ = 0;
   static constexpr uint32_t kOffKV = kOffQ + 2 * kQBytes;
+  // the V zero-point correction tile [32 keys][D] s8, laid out like a V tile:
+  // rows 8 g: -1, rows 8 g + 1 .. 8 g + 4: -128 (g = column group), else 0
+  static constexpr uint32_t kOffCorr = kOffKV + kStages * kTileBytes;
+  static constexpr int kCorrGroup = 8;
   // probability table, four copies [b][33][kBM] u32 holding P << 8b
   static constexpr uint32_t kPtabBytes = 33 * kBM * 4;
-  static constexpr uint32_t kOffPtab = kOffKV + kStages * kTileBytes;
+  static constexpr uint32_t kOffPtab = kOffCorr + 32 * D;
   static constexpr uint32_t kOffRed = kOffPtab + 4 * kPtabBytes;             // [2][kColGroups][kBM] int32
   static constexpr uint32_t kOffLut = kOffRed + 2 * kColGroups * kBM * 4;
   static constexpr uint32_t kOffHp = kOffLut + INTATTN_MAX_CLIPS * 32 * 4;   // head parameters
@@ -192,6 +199,14 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_short_kernel(const __grid
   // head parameters in shared memory: a dynamically indexed kernel argument
   // is a constant-bank load that can miss
   for (int i = tid; i < (args.per_head ? args.H : 1); i += blockDim.x) hp_s[i] = args.hp_dev ? args.hp_dev[i] : args.hp[i];
+  {
+    uint32_t* corr = reinterpret_cast<uint32_t*>(smem + C::kOffCorr);
+    for (int i = tid; i < 8 * D; i += blockDim.x) {
+      const int key = (4 * i) / D % C::kCorrGroup;
+      corr[i] = key == 0 ? 0xFFFFFFFFu : (key <= 4 ? 0x80808080u : 0u);
+    }
+    fence_proxy_async_smem();
+  }
   if (warp == kMmaWarp) {
     tmem_alloc(smem_u32(tmem_slot), kTmemCols);
     tmem_relinquish();
@@ -343,6 +358,8 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_short_kernel(const __grid
       if (!quad_sync(ok)) { ok = false; break; }  // this quadrant's table rows are complete
 
       // ---- pass C: P into TMEM for the P.V MMAs; each S buffer released after its last read ----
+      const bool corr = hp.zv != 0;  // V zero-point: sum this thread's P bytes
+      uint32_t psum = 0;
 #pragma unroll
       for (int j = 0; j < kMaxKeyTiles; ++j) {
         if (j >= T.nkt || !ok) break;
@@ -378,6 +395,10 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_short_kernel(const __grid
           for (int q = 0; q < 8; ++q) pw[q] = 0u;  // masked columns: the P.V reads zeros there
         }
         if (rows_live) {  // rows past the last query row: their P is never used
+          if (corr) {
+#pragma unroll
+            for (int q = 0; q < 8; ++q) psum = __dp4a(pw[q], 0x01010101u, psum);
+          }
           tmem_st8(tlane + kColP + pb * 32 + g * (kCols / 4), pw);
           tmem_wait_st();
         }
@@ -385,7 +406,24 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_short_kernel(const __grid
         arrive_warp(bar(kBarPFull + pb));
         ++sfill[j];
       }
-      pc += T.nkt;
+      if (corr && ok) {
+        // the correction tile, P index pc + nkt: column group g's share in keys 8 g ..
+        const uint32_t pi = pc + T.nkt;
+        const uint32_t pb = pi & (kPBufs - 1);
+        if (!mbar_wait_warp(bar(kBarPEmpty + pb), ((pi / kPBufs) & 1) ^ 1, kRoleSoftmax)) {
+          ok = false;
+        } else {
+          if (rows_live) {
+            uint32_t w0, w1;
+            zv_correction_bytes(hp.zv * static_cast<int32_t>(psum), w0, w1);
+            tmem_st2(tlane + kColP + pb * 32 + g * (C::kCorrGroup / 4), w0, w1);
+            tmem_wait_st();
+          }
+          tc_fence_before();
+          arrive_warp(bar(kBarPFull + pb));
+        }
+      }
+      pc += T.nkt + (corr ? 1 : 0);
       L = Ln;
       T = Tn;
     }
@@ -480,9 +518,11 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_short_kernel(const __grid
     __syncwarp();
   } else if (warp == kMmaWarp) {
     // ============================= MMA issuer =============================
-    constexpr uint32_t idesc_qk = idesc_i8(kBM, kBN, 1, 1, 0);  // s8 x s8, K-major B
-    constexpr uint32_t idesc_pv = idesc_i8(kBM, D, 0, 1, 1);    // u8 x s8, N-major B
+    const uint32_t idesc_qk = idesc_i8(kBM, kBN, 1, args.k_u8 ? 0u : 1u, 0);  // s8 x (s8 | u8), K-major B
+    const uint32_t idesc_pv = idesc_i8(kBM, D, 0, args.v_u8 ? 0u : 1u, 1);    // u8 x (s8 | u8), N-major B
+    constexpr uint32_t idesc_corr = idesc_i8(kBM, D, 0, 1, 1);                // u8 x s8: the correction tile
     const uint64_t kv_desc0 = smem_desc(sKV, 16, C::kSBO, C::kSwizzle);
+    const uint64_t corr_desc = smem_desc(s_base + C::kOffCorr, 16, C::kSBO, C::kSwizzle);
     constexpr uint32_t kSlotDesc = C::kTileBytes >> 4;
     uint32_t slot = 0, kv_par = 0;
     uint32_t sfill0 = 0, sfill1 = 0;  // fills of each S buffer issued (two scalars: j is not a constant here)
@@ -534,11 +574,25 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_short_kernel(const __grid
                     idesc_pv, (j > 0 || kk > 0) ? 1u : 0u);
         mma_commit(bar_kv_empty(slot));
         mma_commit(bar(kBarPEmpty + pb));
-        if (j == T.nkt - 1) mma_commit(bar(kBarOFull + ob));
       }
       __syncwarp();
       next_slot();
       ++pc;
+      if (j == T.nkt - 1) {
+        if (hp_s[args.per_head ? T.h : 0].zv != 0) {
+          // O -= z_v sum_j P_j through the correction tile
+          const uint32_t cb = pc & (kPBufs - 1);
+          if (!mbar_wait_warp(bar(kBarPFull + cb), (pc / kPBufs) & 1, kRoleMma)) return false;
+          tc_fence_after();
+          if (elect_one()) {
+            mma_i8_ts(tmem + kColO + ob * D, tmem + kColP + cb * 32, corr_desc, idesc_corr, 1u);
+            mma_commit(bar(kBarPEmpty + cb));
+          }
+          __syncwarp();
+          ++pc;
+        }
+        mma_commit_elect(bar(kBarOFull + ob));
+      }
       return true;
     };
     walk_schedule(args, begin, qk, pv);

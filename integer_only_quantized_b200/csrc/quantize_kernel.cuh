@@ -23,6 +23,13 @@
 // pass 2, CTA 0 turns amax into s in place and writes code vector 0 over the
 // counters.  Each wait is bounded in time and records a timeout in
 // g_device_error.
+//
+// Asymmetric mode (the same page names a zero-point beside the scale): u8
+// codes.  hi = max(max x, 0) and -lo = max(max -x, 0) over the tensor or
+// head (pass 1 keeps both, the second in the caller's zero-point buffer);
+// w = hi - lo in IEEE double; s = RN32(w / 255), inv = RN32(min(255 / w,
+// FLT_MAX)) (both 1 when w = 0); z = clamp(rint(RN32(-lo * inv)), 0, 255);
+// code = clamp(rint(RN32(x * inv)) + z, 0, 255).
 #pragma once
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
@@ -36,9 +43,12 @@ struct QuantArgs {
   const void* x;     // [B, H, L, d] fp16 or bf16
   int8_t* out;       // [B, H, L, d]
   uint32_t* amax;    // [H] or [1]: the caller's float scale buffer, used as bits
+                     // (asymmetric: max(max x, 0))
+  uint32_t* nmax;    // asymmetric: the caller's zero-point buffer, holding the
+                     // bits of max(max -x, 0) until the end; else null
   int64_t nvec;      // B * H * L * d / 8: 16-byte input vectors in all
   int64_t seg;       // vectors sharing one scale: L * d / 8 per head, or nvec
-  int32_t H, per_head, bf16, n_scales;
+  int32_t H, per_head, bf16, n_scales, asym;
 };
 
 namespace quant {
@@ -127,6 +137,47 @@ __device__ __forceinline__ float2 mul_rn2(float x0, float x1, float m) {
   return r;
 }
 
+// Asymmetric parameters from hi = max(max x, 0) and nl = max(max -x, 0).
+struct AsymParams {
+  float s, inv;
+  int32_t z;
+};
+__device__ __forceinline__ AsymParams asym_params(uint32_t hi_bits, uint32_t nl_bits) {
+  const double w = static_cast<double>(__uint_as_float(hi_bits)) + static_cast<double>(__uint_as_float(nl_bits));
+  AsymParams p;
+  if (w == 0.0) {
+    p.s = 1.0f;
+    p.inv = 1.0f;
+    p.z = 0;
+    return p;
+  }
+  p.s = __double2float_rn(__ddiv_rn(w, 255.0));
+  p.inv = __double2float_rn(fmin(__ddiv_rn(255.0, w), 3.4028234663852886e38));
+  const int32_t z = __float2int_rn(__fmul_rn(__uint_as_float(nl_bits), p.inv));
+  p.z = min(max(z, 0), 255);
+  return p;
+}
+
+// Asymmetric codes of 8 elements: rint(RN(x * inv)) as in codes8, then
+// + z and the clamp to [0, 255].  zoff = 0x4B400000 - z, so that the bits of
+// RN(p + 1.5 * 2^23) minus zoff are rint(p) + z.
+__device__ __forceinline__ uint2 codes8_asym(uint4 v, bool bf16, float inv, int32_t zoff) {
+  constexpr float kRound = 12582912.0f;  // 1.5 * 2^23
+  float f[8];
+  to_float8(v, bf16, f);
+  uint32_t t[8];
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const float2 p = mul_rn2(f[2 * i], f[2 * i + 1], inv);
+    const int32_t a = static_cast<int32_t>(__float_as_uint(__fadd_rn(p.x, kRound))) - zoff;
+    const int32_t b = static_cast<int32_t>(__float_as_uint(__fadd_rn(p.y, kRound))) - zoff;
+    t[2 * i] = static_cast<uint32_t>(min(max(a, 0), 255));
+    t[2 * i + 1] = static_cast<uint32_t>(min(max(b, 0), 255));
+  }
+  return make_uint2(__byte_perm(__byte_perm(t[0], t[1], 0x0040), __byte_perm(t[2], t[3], 0x0040), 0x5410),
+                    __byte_perm(__byte_perm(t[4], t[5], 0x0040), __byte_perm(t[6], t[7], 0x0040), 0x5410));
+}
+
 __device__ __forceinline__ uint2 codes8(uint4 v, bool bf16, float inv) {
   constexpr float kRound = 12582912.0f;  // 1.5 * 2^23
   float f[8];
@@ -150,7 +201,7 @@ __global__ void __launch_bounds__(kThreads) quant_fused_kernel(const __grid_cons
   uint2* dst = reinterpret_cast<uint2*>(a.out);
   uint32_t* arrive = reinterpret_cast<uint32_t*>(a.out);  // code bytes 0-3 until the end
   uint32_t* depart = arrive + 1;                           // code bytes 4-7
-  __shared__ float red[kThreads / 32];
+  __shared__ float red[kThreads / 32], red2[kThreads / 32];
   __shared__ int ok;
   int64_t lo0, hi;
   cta_range(a.nvec, lo0, hi);
@@ -162,8 +213,10 @@ __global__ void __launch_bounds__(kThreads) quant_fused_kernel(const __grid_cons
     const int64_t seg_id = lo / a.seg;
     const int64_t end = min(hi, (seg_id + 1) * a.seg);
     // max |x| as 16-bit patterns, two per word: with the sign bit cleared,
-    // finite fp16 / bf16 values order like their unsigned bit patterns
-    uint32_t mh = 0;
+    // finite fp16 / bf16 values order like their unsigned bit patterns.
+    // Asymmetric: mh takes the non-negative halves, mn the magnitudes of the
+    // negative ones (a half whose sign is set counts as 0 in mh).
+    uint32_t mh = 0, mn = 0;
     for (int64_t base = lo; base < end; base += kStep) {
       // all of a batch's loads are issued before any is used
       uint4 v[kBatch];
@@ -176,25 +229,52 @@ __global__ void __launch_bounds__(kThreads) quant_fused_kernel(const __grid_cons
         for (int it = 0; it < kBatch; ++it)
           v[it] = base + it * kThreads + threadIdx.x < end ? __ldg(p + it * kThreads) : make_uint4(0, 0, 0, 0);
       }
+      if (a.asym) {
 #pragma unroll
-      for (int it = 0; it < kBatch; ++it) {
-        mh = __vmaxu2(mh, v[it].x & 0x7FFF7FFFu);
-        mh = __vmaxu2(mh, v[it].y & 0x7FFF7FFFu);
-        mh = __vmaxu2(mh, v[it].z & 0x7FFF7FFFu);
-        mh = __vmaxu2(mh, v[it].w & 0x7FFF7FFFu);
+        for (int it = 0; it < kBatch; ++it) {
+          const uint32_t w4[4] = {v[it].x, v[it].y, v[it].z, v[it].w};
+#pragma unroll
+          for (int c = 0; c < 4; ++c) {
+            const uint32_t sm = ((w4[c] >> 15) & 0x00010001u) * 0xFFFFu;  // each half's sign spread over the half
+            mh = __vmaxu2(mh, w4[c] & ~sm);
+            mn = __vmaxu2(mn, w4[c] & sm & 0x7FFF7FFFu);
+          }
+        }
+      } else {
+#pragma unroll
+        for (int it = 0; it < kBatch; ++it) {
+          mh = __vmaxu2(mh, v[it].x & 0x7FFF7FFFu);
+          mh = __vmaxu2(mh, v[it].y & 0x7FFF7FFFu);
+          mh = __vmaxu2(mh, v[it].z & 0x7FFF7FFFu);
+          mh = __vmaxu2(mh, v[it].w & 0x7FFF7FFFu);
+        }
       }
     }
-    const uint32_t m16 = max(mh & 0xFFFFu, mh >> 16);
-    float m = a.bf16 ? __uint_as_float(m16 << 16) : __half2float(__ushort_as_half(static_cast<unsigned short>(m16)));
+    auto to_f = [&](uint32_t pair) {
+      const uint32_t m16 = max(pair & 0xFFFFu, pair >> 16);
+      return a.bf16 ? __uint_as_float(m16 << 16) : __half2float(__ushort_as_half(static_cast<unsigned short>(m16)));
+    };
+    float m = to_f(mh), mneg = to_f(mn);
 #pragma unroll
-    for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
-    if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = m;
+    for (int o = 16; o > 0; o >>= 1) {
+      m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+      mneg = fmaxf(mneg, __shfl_xor_sync(0xffffffffu, mneg, o));
+    }
+    if ((threadIdx.x & 31) == 0) {
+      red[threadIdx.x >> 5] = m;
+      red2[threadIdx.x >> 5] = mneg;
+    }
     __syncthreads();
     if (threadIdx.x == 0) {
-      for (int w = 1; w < kThreads / 32; ++w) m = fmaxf(m, red[w]);
+      for (int w = 1; w < kThreads / 32; ++w) {
+        m = fmaxf(m, red[w]);
+        mneg = fmaxf(mneg, red2[w]);
+      }
       if (!zeroed) griddep_wait();  // quant_zero has completed
       zeroed = true;
-      atomicMax(a.amax + (a.per_head ? static_cast<int>(seg_id % a.H) : 0), __float_as_uint(m));
+      const int e = a.per_head ? static_cast<int>(seg_id % a.H) : 0;
+      atomicMax(a.amax + e, __float_as_uint(m));
+      if (a.asym) atomicMax(a.nmax + e, __float_as_uint(mneg));
     }
     __syncthreads();  // red is reused by the next segment
     lo = end;
@@ -216,7 +296,17 @@ __global__ void __launch_bounds__(kThreads) quant_fused_kernel(const __grid_cons
   for (int64_t top = hi; top > lo0;) {
     const int64_t seg_id = (top - 1) / a.seg;
     const int64_t start = max(lo0, seg_id * a.seg);
-    const float inv = inv_scale_of(__ldcg(a.amax + (a.per_head ? static_cast<int>(seg_id % a.H) : 0)));
+    const int e = a.per_head ? static_cast<int>(seg_id % a.H) : 0;
+    float inv;
+    int32_t zoff = 0;
+    if (a.asym) {
+      const AsymParams ap = asym_params(__ldcg(a.amax + e), __ldcg(a.nmax + e));
+      inv = ap.inv;
+      zoff = 0x4B400000 - ap.z;
+    } else {
+      inv = inv_scale_of(__ldcg(a.amax + e));
+    }
+    auto code = [&](uint4 x) { return a.asym ? codes8_asym(x, a.bf16, inv, zoff) : codes8(x, a.bf16, inv); };
     for (int64_t base = start + (top - 1 - start) / kStep * kStep; base >= start; base -= kStep) {
       uint4 v[kBatch];
       const uint4* p = src + base + threadIdx.x;
@@ -225,7 +315,7 @@ __global__ void __launch_bounds__(kThreads) quant_fused_kernel(const __grid_cons
 #pragma unroll
         for (int it = 0; it < kBatch; ++it) v[it] = __ldg(p + it * kThreads);
 #pragma unroll
-        for (int it = 0; it < kBatch; ++it) q[it * kThreads] = codes8(v[it], a.bf16, inv);
+        for (int it = 0; it < kBatch; ++it) q[it * kThreads] = code(v[it]);
       } else {
 #pragma unroll
         for (int it = 0; it < kBatch; ++it)
@@ -234,7 +324,7 @@ __global__ void __launch_bounds__(kThreads) quant_fused_kernel(const __grid_cons
         for (int it = 0; it < kBatch; ++it) {
           const int64_t e = base + it * kThreads + threadIdx.x;
           if (e < top) {
-            const uint2 c = codes8(v[it], a.bf16, inv);
+            const uint2 c = code(v[it]);
             if (e == 0) first = c;
             else q[it * kThreads] = c;
           }
@@ -254,20 +344,35 @@ __global__ void __launch_bounds__(kThreads) quant_fused_kernel(const __grid_cons
   if (threadIdx.x == 0) ok = wait_count(depart, gridDim.x);
   __syncthreads();
   if (!ok) return;
-  for (int i = threadIdx.x; i < a.n_scales; i += kThreads) a.amax[i] = __float_as_uint(scale_of(__ldcg(a.amax + i)));
+  for (int i = threadIdx.x; i < a.n_scales; i += kThreads) {
+    if (a.asym) {
+      const AsymParams ap = asym_params(__ldcg(a.amax + i), __ldcg(a.nmax + i));
+      a.amax[i] = __float_as_uint(ap.s);
+      a.nmax[i] = static_cast<uint32_t>(ap.z);
+    } else {
+      a.amax[i] = __float_as_uint(scale_of(__ldcg(a.amax + i)));
+    }
+  }
   if (threadIdx.x == 0) dst[0] = first;  // thread 0 of CTA 0 owns vector 0
 }
 
-// one CTA: zero the amax slots and the two barrier counters
-__global__ void quant_zero_kernel(uint32_t* amax, int n, uint32_t* counters) {
+// one CTA: zero the amax slots (and the asymmetric second maxima) and the
+// two barrier counters
+__global__ void quant_zero_kernel(uint32_t* amax, uint32_t* nmax, int n, uint32_t* counters) {
   griddep_trigger();  // quant_fused waits for completion before it uses these
-  for (int i = threadIdx.x; i < n; i += blockDim.x) amax[i] = 0u;
+  for (int i = threadIdx.x; i < n; i += blockDim.x) {
+    amax[i] = 0u;
+    if (nmax) nmax[i] = 0u;
+  }
   if (threadIdx.x < 2) counters[threadIdx.x] = 0u;
 }
 
-// one CTA: amax bits -> the float scale, in place (the empty tensor: s = 1)
-__global__ void quant_scales_kernel(uint32_t* amax, int n) {
-  for (int i = threadIdx.x; i < n; i += blockDim.x) amax[i] = __float_as_uint(scale_of(amax[i]));
+// one CTA, the empty tensor: every scale 1 (and every zero-point 0)
+__global__ void quant_scales_kernel(uint32_t* amax, uint32_t* nmax, int n) {
+  for (int i = threadIdx.x; i < n; i += blockDim.x) {
+    amax[i] = __float_as_uint(1.0f);
+    if (nmax) nmax[i] = 0u;
+  }
 }
 
 }  // namespace quant

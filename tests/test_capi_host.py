@@ -143,6 +143,47 @@ def test_forward_fp_argument_errors_need_no_device(ia):
     assert call(B=0) == ia.OK                        # nothing to do, no launch
 
 
+def test_quantize_zp_argument_errors_need_no_device(ia):
+    L = ia.lib()
+
+    def call(dtype=1, B=1, H=2, Lr=64, d=64, x=16, out=16, scales=256, zps=512):
+        return L.intattn_quantize_zp(x, dtype, B, H, Lr, d, 1, out, scales, zps, None)
+
+    assert call(zps=None) == ia.ERR_INVALID_ARG
+    assert call(scales=None) == ia.ERR_INVALID_ARG
+    assert call(dtype=5) == ia.ERR_UNSUPPORTED
+    assert call(Lr=3, d=6) == ia.ERR_UNSUPPORTED      # L * d not whole 16-byte vectors
+    assert call(zps=514) == ia.ERR_UNSUPPORTED        # misaligned zero-point buffer
+    assert call(H=0) == ia.ERR_INVALID_ARG
+    assert call(x=None) == ia.ERR_INVALID_ARG
+    assert call(out=24) == ia.ERR_UNSUPPORTED         # misaligned codes
+
+
+def test_zero_point_argument_errors_need_no_device(ia):
+    """Zero-points out of 0..255 are rejected before any launch; the int4
+    decode and the calibration take no zero-points."""
+    import numpy as np
+    L = ia.lib()
+    one = np.array([0.02], np.float32)
+
+    def scales(zk=None, zv=None):
+        return ia.Scales(one, one, one, one, z_k=zk, z_v=zv)._c()
+
+    for zk, zv in ((256, None), (None, -1), (0, 300)):
+        sc, keep = scales(zk, zv)
+        rc = L.intattn_forward_variant(16, 16, 16, ctypes.byref(sc), 1, 2, 64, 64, 64, 0, 8.0, 16, 0, None)
+        assert rc == ia.ERR_INVALID_ARG, (zk, zv)
+        rc = L.intattn_decode(16, 16, 16, ctypes.byref(sc), 1, 2, 64, 64, 64, 8.0, 16, 256, 1 << 20, None)
+        assert rc == ia.ERR_INVALID_ARG, (zk, zv)
+    sc, keep = scales(3, 4)
+    assert L.intattn_decode_int4(16, 16, 16, ctypes.byref(sc), 1, 2, 64, 64, 64, 8.0, 16, 256, 1 << 20,
+                                 None) == ia.ERR_UNSUPPORTED
+    clip = np.zeros(1, np.float32)
+    assert L.intattn_calibrate_clip(16, 16, ctypes.byref(sc), 1, 2, 64, 64, 64, 0, 4, 4, 0.5, 8.0,
+                                    clip.ctypes.data_as(ctypes.POINTER(ctypes.c_float)), None, 256, 1 << 20,
+                                    None) == ia.ERR_UNSUPPORTED
+
+
 def test_calibrate_argument_errors_need_no_device(ia):
     import numpy as np
     L = ia.lib()

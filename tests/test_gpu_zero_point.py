@@ -1,0 +1,164 @@
+"""GPU parity of the attention with K / V zero-points (u8 codes; the forum
+page's per-layer scale and zero-point, section 动态量化策略) against the CPU
+oracle, byte for byte: both prefill kernels, the int8 decode and the
+host-buffer forward.  The oracle computes S = q.(k - z_k) and
+acc = P.(v - z_v) literally; the kernels run on the codes and subtract
+z_v sum P through a correction tile (prefill) or after the reduction
+(decode)."""
+import numpy as np
+import pytest
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def ia():
+    import torch
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    from integer_only_quantized_b200 import build
+    build.build()
+    import integer_only_quantized_b200 as mod
+    mod.lib()
+    return mod
+
+
+def _dev(x):
+    import torch
+    return torch.from_numpy(np.ascontiguousarray(x)).cuda()
+
+
+def _inputs(seed, B, H, Lq, Lk, d, per_head, zk, zv):
+    """Q int8 N(0, 30); K / V codes: u8 spread around their zero-point (one-
+    sided when z is near 0 or 255) when it is given, else int8."""
+    rng = np.random.default_rng(seed)
+    q = np.clip(np.rint(rng.standard_normal((B, H, Lq, d)) * 30), -128, 127).astype(np.int8)
+
+    def codes(z):
+        x = rng.standard_normal((B, H, Lk, d)) * 40
+        if z is None:
+            return np.clip(np.rint(x), -128, 127).astype(np.int8)
+        zz = np.asarray(z).reshape((1, -1, 1, 1)) if per_head else np.asarray(z).reshape(1, 1, 1, 1)
+        return np.clip(np.rint(x) + zz, 0, 255).astype(np.uint8)
+
+    k, v = codes(zk), codes(zv)
+    n = H if per_head else 1
+    s_q = np.full(n, 0.02, np.float32)
+    s_k = np.linspace(0.01, 0.03, n).astype(np.float32)
+    s_v = np.full(n, 0.05, np.float32)
+    s_o = np.linspace(0.02, 0.04, n).astype(np.float32)
+    return q, k, v, s_q, s_k, s_v, s_o
+
+
+def _zp(kind, H, per_head):
+    """Zero-points of the test cases: None (int8 codes), or per head / per tensor."""
+    if kind is None:
+        return None
+    vals = {"mid": [128, 100, 150, 90], "edges": [0, 255, 1, 254], "zero": [0, 0, 0, 0]}[kind]
+    return np.array([vals[h % 4] for h in range(H)] if per_head else vals[:1], np.int32)
+
+
+CASES = [  # B, H, Lq, Lk, d, causal, per_head, z_k kind, z_v kind
+    (2, 3, 200, 200, 64, False, True, "mid", "mid"),
+    (1, 4, 197, 197, 64, False, True, None, "edges"),
+    (2, 2, 128, 128, 128, True, False, "edges", None),
+    (1, 3, 300, 700, 128, True, True, "mid", "edges"),
+    (1, 2, 129, 1500, 64, False, False, "edges", "mid"),
+    (2, 4, 256, 256, 128, True, True, "zero", "zero"),
+    (1, 2, 1, 1, 64, False, True, "mid", "mid"),
+    (1, 4, 333, 512, 64, True, True, None, "mid"),
+]
+
+
+def _variants(ia, Lk):
+    vs = [ia.VARIANT_AUTO, ia.VARIANT_THREE_PASS]
+    if Lk <= ia.SHORT_ROWS_MAX_KEYS:
+        vs.append(ia.VARIANT_SHORT_ROWS)
+    return vs
+
+
+@pytest.mark.parametrize("case", CASES, ids=lambda c: "B{}H{}Lq{}Lk{}d{}{}{}-k{}-v{}".format(
+    *c[:5], "c" if c[5] else "", "h" if c[6] else "", c[7], c[8]))
+def test_prefill_with_zero_points_matches_oracle(ia, oracle_mod, case):
+    B, H, Lq, Lk, d, causal, per_head, kk, kv = case
+    zk, zv = _zp(kk, H, per_head), _zp(kv, H, per_head)
+    q, k, v, s_q, s_k, s_v, s_o = _inputs(sum(case[:5]), B, H, Lq, Lk, d, per_head, zk, zv)
+    want = oracle_mod.forward(q, k, v, per_head, s_q, s_k, s_v, s_o, causal, 8.0, z_k=zk, z_v=zv)
+    sc = ia.Scales(s_q, s_k, s_v, s_o, per_head=per_head, z_k=zk, z_v=zv)
+    for variant in _variants(ia, Lk):
+        got = ia.forward(_dev(q), _dev(k), _dev(v), sc, causal, 8.0, variant=variant).cpu().numpy()
+        assert ia.device_error() == ia.OK
+        if not np.array_equal(got, want):
+            bad = np.argwhere(got != want)
+            raise AssertionError(f"variant {variant}: {len(bad)} bytes differ, first {bad[:3].tolist()}")
+
+
+@pytest.mark.parametrize("d", [64, 128])
+def test_prefill_extreme_codes_with_zero_points(ia, oracle_mod, d):
+    """The widest gaps the u8 K range allows (rows of q all -128 or all 127
+    against K rows of codes 0 and 255: |gap| up to 128 * 255 * d) and V at
+    both ends of its range, with zero-points at the ends."""
+    B, H, L = 1, 2, 160
+    q = np.where((np.arange(L) % 2 == 0)[:, None], -128, 127).astype(np.int8)[None, None].repeat(H, 1)
+    q = np.ascontiguousarray(np.broadcast_to(q, (B, H, L, d)))
+    k = np.zeros((B, H, L, d), np.uint8)
+    k[:, :, ::3] = 255
+    v = np.zeros((B, H, L, d), np.uint8)
+    v[:, :, 1::2] = 255
+    zk = np.array([0, 255], np.int32)
+    zv = np.array([255, 0], np.int32)
+    s_q = np.full(H, 0.001, np.float32)
+    s_k = np.full(H, 0.001, np.float32)
+    s_v = np.full(H, 0.01, np.float32)
+    s_o = np.full(H, 0.02, np.float32)
+    want = oracle_mod.forward(q, k, v, True, s_q, s_k, s_v, s_o, False, 10.0, z_k=zk, z_v=zv)
+    sc = ia.Scales(s_q, s_k, s_v, s_o, per_head=True, z_k=zk, z_v=zv)
+    for variant in _variants(ia, L):
+        got = ia.forward(_dev(q), _dev(k), _dev(v), sc, False, 10.0, variant=variant).cpu().numpy()
+        assert np.array_equal(got, want), variant
+
+
+def test_reexpressed_codes_give_the_symmetric_bytes(ia):
+    """int8 K / V shifted to u8 with zero-point 128 run through the kernels
+    give the bytes of the symmetric call."""
+    B, H, L, d = 2, 3, 400, 128
+    q, k, v, s_q, s_k, s_v, s_o = _inputs(5, B, H, L, L, d, True, None, None)
+    sym = ia.forward(_dev(q), _dev(k), _dev(v), ia.Scales(s_q, s_k, s_v, s_o, per_head=True), True, 8.0)
+    ku = (k.astype(np.int16) + 128).astype(np.uint8)
+    vu = (v.astype(np.int16) + 128).astype(np.uint8)
+    z = np.full(H, 128, np.int32)
+    asym = ia.forward(_dev(q), _dev(ku), _dev(vu), ia.Scales(s_q, s_k, s_v, s_o, per_head=True, z_k=z, z_v=z),
+                      True, 8.0)
+    assert np.array_equal(sym.cpu().numpy(), asym.cpu().numpy())
+
+
+DECODE_CASES = [(4, 3, 1000, 1100, 128, True, "mid", "edges"), (2, 2, 4096, 4096, 64, False, "edges", "mid"),
+                (3, 4, 37, 64, 128, True, None, "mid"), (1, 2, 513, 600, 64, True, "mid", None)]
+
+
+@pytest.mark.parametrize("case", DECODE_CASES, ids=lambda c: "B{}H{}Lk{}Lmax{}d{}-k{}-v{}".format(*c[:5], c[6], c[7]))
+def test_decode_with_zero_points_matches_oracle(ia, oracle_mod, case):
+    B, H, Lk, Lmax, d, per_head, kk, kv = case
+    zk, zv = _zp(kk, H, per_head), _zp(kv, H, per_head)
+    q, kc, vc, s_q, s_k, s_v, s_o = _inputs(Lk + d, B, H, 1, Lmax, d, per_head, zk, zv)
+    want = oracle_mod.decode(q, kc, vc, per_head, s_q, s_k, s_v, s_o, Lk, 8.0, z_k=zk, z_v=zv)
+    sc = ia.Scales(s_q, s_k, s_v, s_o, per_head=per_head, z_k=zk, z_v=zv)
+    import torch
+    ws = torch.full((ia.decode_workspace_size(B, H, Lk, d),), 0x5A, dtype=torch.uint8, device="cuda")
+    for _ in range(2):  # the second call reuses the workspace left by the first
+        got = ia.decode(_dev(q), _dev(kc), _dev(vc), sc, Lk, 8.0, workspace=ws).cpu().numpy()
+        assert ia.device_error() == ia.OK
+        assert np.array_equal(got, want)
+
+
+def test_forward_host_with_zero_points(ia, oracle_mod):
+    import torch
+    B, H, L, d = 2, 2, 300, 64
+    zk, zv = _zp("mid", H, True), _zp("edges", H, True)
+    q, k, v, s_q, s_k, s_v, s_o = _inputs(9, B, H, L, L, d, True, zk, zv)
+    want = oracle_mod.forward(q, k, v, True, s_q, s_k, s_v, s_o, True, 8.0, z_k=zk, z_v=zv)
+    sc = ia.Scales(s_q, s_k, s_v, s_o, per_head=True, z_k=zk, z_v=zv)
+    pin = lambda a: torch.from_numpy(a).pin_memory()
+    out = ia.forward_host(pin(q), pin(k), pin(v), sc, True, 8.0)
+    torch.cuda.synchronize()
+    assert np.array_equal(out.numpy(), want)
