@@ -213,12 +213,13 @@ def workload_config(w, world: int) -> dict:
             "parallelism": f"dp{world} (independent problems)"}
 
 
-def time_prefill(ia, w, x, dev, stream, steps: int, warmup: int, clocks=None, world: int = 1, variant: int = 0):
+def time_prefill(ia, w, x, dev, stream, steps: int, warmup: int, clocks=None, world: int = 1, variant: int = 0,
+                 scales=None):
     """ms per forward of workload w: `steps` calls over rotating copies of the
     inputs, captured as one CUDA graph and replayed between CUDA events on
     `stream`; max over ranks."""
     import torch
-    sc = ia.Scales(x.s_q, x.s_k, x.s_v, x.s_o, per_head=w.per_head)
+    sc = scales if scales is not None else ia.Scales(x.s_q, x.s_k, x.s_v, x.s_o, per_head=w.per_head)
     nsets, _ = rotation(w)
     q0, k0, v0 = (torch.from_numpy(a).to(dev) for a in (x.q, x.k, x.v))
     sets = [(q0.clone(), k0.clone(), v0.clone(), torch.empty_like(q0)) for _ in range(nsets)]
@@ -229,6 +230,8 @@ def time_prefill(ia, w, x, dev, stream, steps: int, warmup: int, clocks=None, wo
         ia.forward(q, k, v, sc, w.causal, w.clip_c, out=o, stream=stream, variant=variant)
 
     # everything on `stream`: the calls, the capture, the replay and the events
+    # (the copies above ran on the default stream: complete them first)
+    torch.cuda.synchronize(dev)
     with torch.cuda.stream(stream):
         for i in range(warmup):
             step(i)
@@ -324,6 +327,7 @@ def run_ours(args):
     def e2e_step(i):
         ia.forward_host(hq, hk, hv, sc, w.causal, w.clip_c, out=ho, workspace=hws, stream=stream, device=dev)
 
+    torch.cuda.synchronize(dev)  # inputs made on the default stream are complete before `stream` reads them
     for i in range(args.warmup):
         e2e_step(i)
     torch.cuda.synchronize(dev)
@@ -336,6 +340,9 @@ def run_ours(args):
     torch.cuda.synchronize(dev)
     barrier(world, dev)
     e2e_ms = max_over_ranks(e0.elapsed_time(e1) / args.steps, world, dev)
+    err = ia.device_error(stream)
+    if err != ia.OK:
+        raise RuntimeError(f"device error {err} ({ia.strerror(err)}) in the host-buffer forward")
     e2e_val = aggregate_value(ops, world, e2e_ms * 1e-3) / 1e12
 
     peaks, peak_src = load_peaks()
@@ -364,6 +371,7 @@ def run_ours(args):
 
     if not args.no_configs:
         line["prefill_configs"] = run_prefill_configs(args, ia, dev, stream, world, peak_int8, w.name)
+        line["zero_points"] = run_zero_point(args, ia, dev, stream, world, peak_int8, ms)
     if not args.no_decode:
         line["decode"] = run_decode(args, dev, stream, world, peaks, peak_src, args.decode_workload)
         line["decode_int4"] = run_decode(args, dev, stream, world, peaks, peak_src,
@@ -439,6 +447,7 @@ def run_quantize(args, dev, stream, world, peaks, peak_src):
     out = torch.empty(shape, dtype=torch.int8, device=dev)
     scales = torch.empty(shape[1], dtype=torch.float32, device=dev)
     steps = max(10, min(args.steps, 60))
+    torch.cuda.synchronize(dev)  # inputs made on the default stream are complete before `stream` reads them
     for i in range(max(3, args.warmup)):
         ia.quantize(xs[i % 3], True, out=out, scales=scales, stream=stream)
     torch.cuda.synchronize(dev)
@@ -451,6 +460,9 @@ def run_quantize(args, dev, stream, world, peaks, peak_src):
     torch.cuda.synchronize(dev)
     barrier(world, dev)
     ms = max_over_ranks(t0.elapsed_time(t1) / steps, world, dev)
+    err = ia.device_error(stream)
+    if err != ia.OK:
+        raise RuntimeError(f"device error {err} ({ia.strerror(err)}) in the quantisation leg")
     algo = 3 * n  # 2 bytes read + 1 byte written per element
     gbs = algo / (ms * 1e-3) / 1e9
     return {"workload": "llama7b_layer_bf16_b1h32l8192d128", "value": round(aggregate_value(algo, world, ms * 1e-3) / 1e9, 1),
@@ -482,6 +494,7 @@ def run_forward_fp(args, dev, stream, world, peaks, peak_src):
     s_o = np.full(w.H, 0.02, np.float32)
     call = lambda i: ia.forward_fp(*sets[i % 2], True, s_o, w.causal, w.clip_c, out=out, workspace=ws, stream=stream)
     steps = max(10, min(args.steps, 40))
+    torch.cuda.synchronize(dev)  # inputs made on the default stream are complete before `stream` reads them
     for i in range(max(3, args.warmup)):
         call(i)
     torch.cuda.synchronize(dev)
@@ -494,8 +507,9 @@ def run_forward_fp(args, dev, stream, world, peaks, peak_src):
     torch.cuda.synchronize(dev)
     barrier(world, dev)
     ms = max_over_ranks(t0.elapsed_time(t1) / steps, world, dev)
-    if ia.device_error(stream) != ia.OK:
-        raise RuntimeError("a kernel wait timed out, or a parameter was out of range, in forward_fp")
+    err = ia.device_error(stream)
+    if err != ia.OK:
+        raise RuntimeError(f"device error {err} ({ia.strerror(err)}) in the forward from bf16")
     peak_int8, _ = _int8_peak(peaks, sustained=False)
     tops = w.effective_ops / (ms * 1e-3) / 1e12
     return {"workload": w.name + "_bf16_inputs", "value": round(aggregate_value(w.effective_ops, world, ms * 1e-3) / 1e12, 3),
@@ -504,6 +518,37 @@ def run_forward_fp(args, dev, stream, world, peaks, peak_src):
             "roofline": {"bound": "tensor", "achieved": round(tops, 3), "peak": round(peak_int8, 1), "unit": "TOPS",
                          "frac": round(tops / peak_int8, 4)},
             "l2": "inputs alternate between 2 sets (201 MB > 126 MB L2)"}
+
+
+def run_zero_point(args, ia, dev, stream, world, peak_int8, base_ms):
+    """The headline prefill with K and V as u8 codes carrying zero-points
+    (the int8 codes re-expressed as code + 128 with zero-point 128, so the
+    output bytes are the headline's): the cost of the zero-point path, timed
+    exactly like the headline."""
+    import dataclasses
+
+    import numpy as np
+
+    from integer_only_quantized_b200 import workloads as wl
+    w = wl.WORKLOADS[args.workload]
+    x = wl.make_inputs(w)
+    xu = dataclasses.replace(x, k=(x.k.astype(np.int16) + 128).astype(np.uint8),
+                             v=(x.v.astype(np.int16) + 128).astype(np.uint8))
+    n = w.H if w.per_head else 1
+    z = np.full(n, 128, np.int32)
+    sc = ia.Scales(x.s_q, x.s_k, x.s_v, x.s_o, per_head=w.per_head, z_k=z, z_v=z)
+    nsets, _ = rotation(w)
+    steps = max(10, min(args.steps, 40), nsets)
+    ms, _ = time_prefill(ia, w, xu, dev, stream, steps, max(3, args.warmup), None, world, scales=sc)
+    tops = w.effective_ops / (ms * 1e-3) / 1e12
+    return {"workload": w.name + "_u8_kv_zero_points", "value": round(aggregate_value(w.effective_ops, world,
+                                                                                      ms * 1e-3) / 1e12, 3),
+            "unit": "TOPS", "ms_per_call": round(ms, 5), "launches_per_call": 1,
+            "vs_symmetric": round(ms / base_ms, 4),
+            "note": "u8 K and V with zero-point 128 per head: the MMA reads u8, and z_v sum P is subtracted "
+                    "through one correction MMA per softmax team per query tile",
+            "roofline": {"bound": "tensor", "achieved": round(tops, 3), "peak": round(peak_int8, 1), "unit": "TOPS",
+                         "frac": round(tops / peak_int8, 4)}}
 
 
 def run_calibrate(args, dev, stream, world):
@@ -526,6 +571,7 @@ def run_calibrate(args, dev, stream, world):
     keep, stride = 32, 64
     ws = torch.empty(max(ia.calibrate_workspace_size(w.B, w.H), 1), dtype=torch.uint8, device=dev)
     call = lambda: ia.calibrate_clip(q, k, sc, w.causal, keep, stride, workspace=ws, stream=stream)
+    torch.cuda.synchronize(dev)  # inputs made on the default stream are complete before `stream` reads them
     for _ in range(max(3, args.warmup)):
         call()
     steps = max(5, min(args.steps, 20))
@@ -571,6 +617,7 @@ def run_gelu(args, dev, stream, world, peaks, peak_src):
     n = xs[0].numel()
     out = torch.empty_like(xs[0])
     steps = max(10, min(args.steps, 100))
+    torch.cuda.synchronize(dev)  # inputs made on the default stream are complete before `stream` reads them
     for i in range(max(3, args.warmup)):
         ia.gelu(xs[i % 4], s_x, s_x, spec["c"], out=out, stream=stream)
     torch.cuda.synchronize(dev)
@@ -612,6 +659,7 @@ def run_decode(args, dev, stream, world, peaks, peak_src, name):
     else:
         call = lambda: ia.decode(x.q, x.k, x.v, sc, w.Lk, w.clip_c, out=out, workspace=ws, stream=stream)
     steps = max(10, min(args.steps, 100))
+    torch.cuda.synchronize(dev)  # inputs made on the default stream are complete before `stream` reads them
     for _ in range(max(3, args.warmup)):
         call()
     torch.cuda.synchronize(dev)

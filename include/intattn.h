@@ -286,6 +286,17 @@ int intattn_forward_fp(const void *q, const void *k, const void *v, int dtype, i
                        int d, int causal, int8_t *out, float *scales_out, void *workspace,
                        size_t workspace_bytes, intattn_stream_t stream);
 
+/* intattn_forward_fp with K and V quantised with zero-points (u8 codes, the
+ * rule of intattn_quantize_zp) and Q symmetric, then the integer forward
+ * with those zero-points (the definition under intattn_scales_t.z_k / z_v).
+ * zero_points_out (optional, DEVICE int32, 4-byte aligned): receives z_k then
+ * z_v (H entries each per head, else one each).  Workspace, arguments and
+ * return codes as intattn_forward_fp. */
+int intattn_forward_fp_zp(const void *q, const void *k, const void *v, int dtype, int per_head, const float *s_o,
+                          const float *clip, float clip_c, int B, int H, int Lq, int Lk, int d, int causal,
+                          int8_t *out, float *scales_out, int32_t *zero_points_out, void *workspace,
+                          size_t workspace_bytes, intattn_stream_t stream);
+
 /* Bytes of device workspace intattn_calibrate_clip needs (0 for invalid sizes). */
 size_t intattn_calibrate_workspace_size(int B, int H);
 

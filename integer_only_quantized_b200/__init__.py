@@ -24,6 +24,7 @@ MAX_CLIPS = 8
 # every function declared in include/intattn.h
 EXPORTED = ("intattn_derive_params", "intattn_forward", "intattn_forward_variant",
             "intattn_forward_host_workspace_size", "intattn_forward_fp_workspace_size", "intattn_forward_fp",
+            "intattn_forward_fp_zp",
             "intattn_calibrate_workspace_size", "intattn_calibrate_clip",
             "intattn_forward_host", "intattn_decode_workspace_size",
             "intattn_decode", "intattn_decode_int4", "intattn_decode_static_scratch", "intattn_quantize",
@@ -126,6 +127,8 @@ def lib() -> ctypes.CDLL:
         f32p = ctypes.POINTER(ctypes.c_float)
         L.intattn_forward_fp.argtypes = [vp, vp, vp, i32, i32, f32p, f32p, f32, i32, i32, i32, i32, i32, i32,
                                          vp, vp, vp, ctypes.c_size_t, vp]
+        L.intattn_forward_fp_zp.argtypes = [vp, vp, vp, i32, i32, f32p, f32p, f32, i32, i32, i32, i32, i32, i32,
+                                            vp, vp, vp, vp, ctypes.c_size_t, vp]
         L.intattn_calibrate_workspace_size.argtypes = [i32, i32]
         L.intattn_calibrate_workspace_size.restype = ctypes.c_size_t
         L.intattn_calibrate_clip.argtypes = [vp, vp, ctypes.POINTER(_Scales), i32, i32, i32, i32, i32, i32, i32,
@@ -274,10 +277,12 @@ def forward_fp_workspace_size(B: int, H: int, Lq: int, Lk: int, d: int) -> int:
 
 
 def forward_fp(q, k, v, per_head: bool, s_o, causal: bool, clip_c: float, clip=None, out=None, scales_out=None,
-               workspace=None, stream=None):
+               workspace=None, stream=None, zero_points=False, zero_points_out=None):
     """intattn_forward_fp: fp16 / bf16 q [B,H,Lq,d], k, v [B,H,Lk,d] (CUDA)
     -> int8 out, quantising on the device.  s_o (and clip, optional): host
-    floats, H entries per head or 1."""
+    floats, H entries per head or 1.  zero_points=True: intattn_forward_fp_zp
+    (K and V quantised with zero-points; zero_points_out, optional CUDA int32
+    [2 n], receives z_k then z_v)."""
     import torch
     dt = {torch.float16: DTYPE_FP16, torch.bfloat16: DTYPE_BF16}
     for t, n in ((q, "q"), (k, "k"), (v, "v")):
@@ -298,12 +303,17 @@ def forward_fp(q, k, v, per_head: bool, s_o, causal: bool, clip_c: float, clip=N
     if workspace is None:
         workspace = torch.empty(max(need, 1), dtype=torch.uint8, device=q.device)
     f32p = ctypes.POINTER(ctypes.c_float)
-    rc = lib().intattn_forward_fp(q.data_ptr(), k.data_ptr(), v.data_ptr(), dt[q.dtype], int(bool(per_head)),
-                                  so.ctypes.data_as(f32p), None if cl is None else cl.ctypes.data_as(f32p),
-                                  float(clip_c), B, H, Lq, Lk, d, int(bool(causal)), out.data_ptr(),
-                                  None if scales_out is None else scales_out.data_ptr(), workspace.data_ptr(),
-                                  workspace.numel(), _stream_handle(stream, q.device))
-    _check(rc, "intattn_forward_fp")
+    args = (q.data_ptr(), k.data_ptr(), v.data_ptr(), dt[q.dtype], int(bool(per_head)), so.ctypes.data_as(f32p),
+            None if cl is None else cl.ctypes.data_as(f32p), float(clip_c), B, H, Lq, Lk, d, int(bool(causal)),
+            out.data_ptr(), None if scales_out is None else scales_out.data_ptr())
+    tail = (workspace.data_ptr(), workspace.numel(), _stream_handle(stream, q.device))
+    if zero_points:
+        zp = None if zero_points_out is None else zero_points_out.data_ptr()
+        rc = lib().intattn_forward_fp_zp(*args, zp, *tail)
+        _check(rc, "intattn_forward_fp_zp")
+    else:
+        rc = lib().intattn_forward_fp(*args, *tail)
+        _check(rc, "intattn_forward_fp")
     return out
 
 

@@ -187,37 +187,37 @@ int note_launch(cudaError_t e) {
 }
 
 // ------------------------------------------------------- kernel attributes
-template <int D>
+template <int D, bool ZV>
 int prefill_launch(const PrefillArgs& args, int grid, cudaStream_t stream) {
-  using C = intattn::prefill::Cfg<D>;
+  using C = intattn::prefill::Cfg<D, ZV>;
   static bool attr_set[64] = {};
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return INTATTN_ERR_CUDA;
   if (dev < 0 || dev >= 64) return INTATTN_ERR_CUDA;
   if (!attr_set[dev]) {
-    if (cudaFuncSetAttribute(intattn::prefill::prefill_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    if (cudaFuncSetAttribute(intattn::prefill::prefill_kernel<D, ZV>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              static_cast<int>(C::kSmemBytes)) != cudaSuccess)
       return INTATTN_ERR_CUDA;
     attr_set[dev] = true;
   }
-  intattn::prefill::prefill_kernel<D><<<grid, intattn::prefill::kThreads, C::kSmemBytes, stream>>>(args);
+  intattn::prefill::prefill_kernel<D, ZV><<<grid, intattn::prefill::kThreads, C::kSmemBytes, stream>>>(args);
   return note_launch(cudaGetLastError());
 }
 
-template <int D>
+template <int D, bool ZV>
 int prefill_short_launch(const PrefillArgs& args, int grid, cudaStream_t stream) {
-  using C = intattn::shortrow::Cfg<D>;
+  using C = intattn::shortrow::Cfg<D, ZV>;
   static bool attr_set[64] = {};
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return INTATTN_ERR_CUDA;
   if (dev < 0 || dev >= 64) return INTATTN_ERR_CUDA;
   if (!attr_set[dev]) {
-    if (cudaFuncSetAttribute(intattn::shortrow::prefill_short_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    if (cudaFuncSetAttribute(intattn::shortrow::prefill_short_kernel<D, ZV>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              static_cast<int>(C::kSmemBytes)) != cudaSuccess)
       return INTATTN_ERR_CUDA;
     attr_set[dev] = true;
   }
-  intattn::shortrow::prefill_short_kernel<D><<<grid, intattn::shortrow::kThreads, C::kSmemBytes, stream>>>(args);
+  intattn::shortrow::prefill_short_kernel<D, ZV><<<grid, intattn::shortrow::kThreads, C::kSmemBytes, stream>>>(args);
   return note_launch(cudaGetLastError());
 }
 
@@ -431,8 +431,13 @@ int forward_launch(const int8_t* q, const int8_t* k, const int8_t* v, PrefillArg
   const bool short_rows = variant == INTATTN_VARIANT_SHORT_ROWS ||
                           (variant == INTATTN_VARIANT_AUTO && Lk <= intattn::shortrow::kMaxKeys);
   if (short_rows)
-    return d == 64 ? prefill_short_launch<64>(args, grid, st) : prefill_short_launch<128>(args, grid, st);
-  return d == 64 ? prefill_launch<64>(args, grid, st) : prefill_launch<128>(args, grid, st);
+    return args.v_u8 ? (d == 64 ? prefill_short_launch<64, true>(args, grid, st)
+                                : prefill_short_launch<128, true>(args, grid, st))
+                     : (d == 64 ? prefill_short_launch<64, false>(args, grid, st)
+                                : prefill_short_launch<128, false>(args, grid, st));
+  // the kernel instance with the V zero-point correction only when V has zero-points
+  return args.v_u8 ? (d == 64 ? prefill_launch<64, true>(args, grid, st) : prefill_launch<128, true>(args, grid, st))
+                   : (d == 64 ? prefill_launch<64, false>(args, grid, st) : prefill_launch<128, false>(args, grid, st));
 }
 
 // Exp tables of the distinct clip thresholds of n entries (clips[i], or
@@ -462,7 +467,7 @@ size_t align256_fp(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
 // Workspace of intattn_forward_fp: int8 q, k, v; the three scale arrays; the
 // head parameters; the derivation status.
 struct FpLayout {
-  size_t q8, k8, v8, sc, hp, status, total;
+  size_t q8, k8, v8, sc, zp, hp, status, total;
 };
 
 FpLayout fp_layout(int B, int H, int Lq, int Lk, int d) {
@@ -472,7 +477,8 @@ FpLayout fp_layout(int B, int H, int Lq, int Lk, int d) {
   L.k8 = L.q8 + align256_fp(bh * Lq * d);
   L.v8 = L.k8 + align256_fp(bh * Lk * d);
   L.sc = L.v8 + align256_fp(bh * Lk * d);
-  L.hp = L.sc + 3 * align256_fp(INTATTN_MAX_HEADS * sizeof(float));
+  L.zp = L.sc + 3 * align256_fp(INTATTN_MAX_HEADS * sizeof(float));
+  L.hp = L.zp + 2 * align256_fp(INTATTN_MAX_HEADS * sizeof(int32_t));
   L.status = L.hp + align256_fp(INTATTN_MAX_HEADS * sizeof(HeadParamsDev));
   L.total = L.status + 256;
   return L;
@@ -509,10 +515,19 @@ size_t intattn_forward_fp_workspace_size(int B, int H, int Lq, int Lk, int d) {
   return fp_layout(B, H, Lq, Lk, d).total;
 }
 
-int intattn_forward_fp(const void* q, const void* k, const void* v, int dtype, int per_head, const float* s_o,
-                       const float* clip, float clip_c, int B, int H, int Lq, int Lk, int d, int causal,
-                       int8_t* out, float* scales_out, void* workspace, size_t workspace_bytes,
-                       intattn_stream_t stream) {
+}  // extern "C"
+
+namespace {
+
+int quantize_impl(const void* x, int dtype, int B, int H, int L, int d, int per_head, void* out, float* scales,
+                  int32_t* zero_points, cudaStream_t st);
+
+// intattn_forward_fp (asym_kv false) and intattn_forward_fp_zp (K and V
+// quantised with zero-points, u8 codes).
+int forward_fp_impl(const void* q, const void* k, const void* v, int dtype, int per_head, const float* s_o,
+                    const float* clip, float clip_c, int B, int H, int Lq, int Lk, int d, int causal, int8_t* out,
+                    float* scales_out, bool asym_kv, int32_t* zero_points_out, void* workspace,
+                    size_t workspace_bytes, intattn_stream_t stream) {
   if (B < 0 || H <= 0 || Lq < 0 || Lk < 1 || Lk > 65535) return INTATTN_ERR_INVALID_ARG;
   if (causal && Lq > Lk) return INTATTN_ERR_INVALID_ARG;
   if (d != 64 && d != 128) return INTATTN_ERR_UNSUPPORTED;
@@ -538,6 +553,7 @@ int intattn_forward_fp(const void* q, const void* k, const void* v, int dtype, i
   if (!q || !k || !v || !out) return INTATTN_ERR_INVALID_ARG;
   if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out)) return INTATTN_ERR_UNSUPPORTED;
   if (scales_out && (reinterpret_cast<uintptr_t>(scales_out) & 3u)) return INTATTN_ERR_UNSUPPORTED;
+  if (zero_points_out && (reinterpret_cast<uintptr_t>(zero_points_out) & 3u)) return INTATTN_ERR_UNSUPPORTED;
   const FpLayout L = fp_layout(B, H, Lq, Lk, d);
   if (!workspace || workspace_bytes < L.total || (reinterpret_cast<uintptr_t>(workspace) & 255u))
     return INTATTN_ERR_WORKSPACE;
@@ -550,17 +566,21 @@ int intattn_forward_fp(const void* q, const void* k, const void* v, int dtype, i
   float* s_q = sc;
   float* s_k = sc + sc_step;
   float* s_v = sc + 2 * sc_step;
+  const size_t zp_step = align256_fp(INTATTN_MAX_HEADS * sizeof(int32_t)) / sizeof(int32_t);
+  int32_t* z_k = asym_kv ? reinterpret_cast<int32_t*>(ws + L.zp) : nullptr;
+  int32_t* z_v = asym_kv ? z_k + zp_step : nullptr;
   HeadParamsDev* hp = reinterpret_cast<HeadParamsDev*>(ws + L.hp);
   uint32_t* status = reinterpret_cast<uint32_t*>(ws + L.status);
   // quantise on the stream (scales stay on the device)
-  if ((rc = intattn_quantize(q, dtype, B, H, Lq, d, per_head, q8, s_q, stream)) ||
-      (rc = intattn_quantize(k, dtype, B, H, Lk, d, per_head, k8, s_k, stream)) ||
-      (rc = intattn_quantize(v, dtype, B, H, Lk, d, per_head, v8, s_v, stream)))
-    return rc;
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  if ((rc = quantize_impl(q, dtype, B, H, Lq, d, per_head, q8, s_q, nullptr, st)) ||
+      (rc = quantize_impl(k, dtype, B, H, Lk, d, per_head, k8, s_k, z_k, st)) ||
+      (rc = quantize_impl(v, dtype, B, H, Lk, d, per_head, v8, s_v, z_v, st)))
+    return rc;
   da.s_q = s_q;
   da.s_k = s_k;
   da.s_v = s_v;
+  da.z_v = z_v;
   da.hp = hp;
   da.status = status;
   da.n = n;
@@ -573,10 +593,38 @@ int intattn_forward_fp(const void* q, const void* k, const void* v, int dtype, i
                                             cudaMemcpyDeviceToDevice, st))))
         return rc;
   }
+  if (zero_points_out && asym_kv) {
+    for (int t = 0; t < 2; ++t)
+      if ((rc = note_launch(cudaMemcpyAsync(zero_points_out + t * n, z_k + t * zp_step, n * sizeof(int32_t),
+                                            cudaMemcpyDeviceToDevice, st))))
+        return rc;
+  }
   args.per_head = per_head ? 1 : 0;
+  args.k_u8 = asym_kv ? 1 : 0;
+  args.v_u8 = asym_kv ? 1 : 0;
   args.hp_dev = hp;
   args.status = status;
   return forward_launch(q8, k8, v8, args, B, H, Lq, Lk, d, causal, out, INTATTN_VARIANT_AUTO, st);
+}
+
+}  // namespace
+
+extern "C" {
+
+int intattn_forward_fp(const void* q, const void* k, const void* v, int dtype, int per_head, const float* s_o,
+                       const float* clip, float clip_c, int B, int H, int Lq, int Lk, int d, int causal,
+                       int8_t* out, float* scales_out, void* workspace, size_t workspace_bytes,
+                       intattn_stream_t stream) {
+  return forward_fp_impl(q, k, v, dtype, per_head, s_o, clip, clip_c, B, H, Lq, Lk, d, causal, out, scales_out,
+                         false, nullptr, workspace, workspace_bytes, stream);
+}
+
+int intattn_forward_fp_zp(const void* q, const void* k, const void* v, int dtype, int per_head, const float* s_o,
+                          const float* clip, float clip_c, int B, int H, int Lq, int Lk, int d, int causal,
+                          int8_t* out, float* scales_out, int32_t* zero_points_out, void* workspace,
+                          size_t workspace_bytes, intattn_stream_t stream) {
+  return forward_fp_impl(q, k, v, dtype, per_head, s_o, clip, clip_c, B, H, Lq, Lk, d, causal, out, scales_out,
+                         true, zero_points_out, workspace, workspace_bytes, stream);
 }
 
 // ------------------------------------------------ forward from host buffers
@@ -840,6 +888,8 @@ int intattn_decode_static_scratch(const int8_t* q, const int8_t* k_cache, const 
   return d == 64 ? decode_launch<64>(a, st) : decode_launch<128>(a, st);
 }
 
+}  // extern "C"
+
 namespace {
 
 // intattn_quantize (zero_points == nullptr) and intattn_quantize_zp.
@@ -904,6 +954,8 @@ int quantize_impl(const void* x, int dtype, int B, int H, int L, int d, int per_
 }
 
 }  // namespace
+
+extern "C" {
 
 int intattn_quantize(const void* x, int dtype, int B, int H, int L, int d, int per_head, int8_t* out,
                      float* scales, intattn_stream_t stream) {

@@ -22,6 +22,7 @@ struct DeriveArgs {
   const float* s_q;      // device: quantisation scales, H entries (per head) or 1
   const float* s_k;
   const float* s_v;
+  const int32_t* z_v;    // device: V zero-points (asymmetric V codes), or null
   HeadParamsDev* hp;     // device out: per head (or entry 0)
   uint32_t* status;      // device out: 0, or kErrParamRange
   int32_t n;             // entries: H (per head) or 1
@@ -76,6 +77,7 @@ __global__ void derive_params_kernel(const __grid_constant__ DeriveArgs a) {
     HeadParamsDev hp{};
     const bool ok = index_params(a.s_q[i], a.s_k[i], a.d, a.clip[i], hp) && requant_params(a.s_v[i], a.s_o[i], hp);
     hp.lut = a.lut[i];
+    hp.zv = a.z_v ? a.z_v[i] : 0;
     a.hp[i] = hp;
     if (!ok) atomicOr(&bad, 1);
   }

@@ -127,7 +127,9 @@ enum Bar : int {
   kBarKvFull = 21,      // [stages], then kv_empty[stages]
 };
 
-template <int D>
+// ZV: the kernel instance that supports a V zero-point (the correction tile
+// and the sums of P); the other instance is the plain int8 kernel.
+template <int D, bool ZV = false>
 struct Cfg {
   static constexpr int kStages = (D == 64) ? 8 : 6;
   // O accumulators in TMEM: with d = 64 two fit below the P buffers, so a
@@ -148,7 +150,7 @@ struct Cfg {
   // probability table, four copies [b][33][kBM] u32 with P << 8b, so four
   // looked-up bytes pack into a word by integer adds
   static constexpr uint32_t kPtabBytes = 33 * kBM * 4;
-  static constexpr uint32_t kOffPtab = kOffCorr + 32 * D;
+  static constexpr uint32_t kOffPtab = kOffCorr + (ZV ? 32 * D : 0);
   static constexpr uint32_t kOffRed = kOffPtab + 4 * kPtabBytes;        // [2][kGroups][kBM] int32
   static constexpr uint32_t kOffLut = kOffRed + 2 * kGroups * kBM * 4;
   static constexpr uint32_t kOffHp = kOffLut + INTATTN_MAX_CLIPS * 32 * 4;  // head parameters
@@ -240,9 +242,9 @@ __device__ __forceinline__ Tile tile_of(const PrefillArgs& a, int L) {
   return t;
 }
 
-template <int D>
+template <int D, bool ZV>
 __global__ void __launch_bounds__(kThreads, 1) prefill_kernel(const __grid_constant__ PrefillArgs args) {
-  using C = Cfg<D>;
+  using C = Cfg<D, ZV>;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   // 1024-byte aligned base (swizzled TMA tiles); offsetting the __shared__
   // array keeps the compiler aware of the address space.
@@ -292,7 +294,7 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_kernel(const __grid_const
   // head parameters in shared memory: a dynamically indexed kernel argument
   // is a constant-bank load that can miss
   for (int i = tid; i < (args.per_head ? args.H : 1); i += blockDim.x) hp_s[i] = args.hp_dev ? args.hp_dev[i] : args.hp[i];
-  {
+  if constexpr (ZV) {
     // the zero-point correction tile (uniform rows: the swizzle moves bytes within a row only)
     uint32_t* corr = reinterpret_cast<uint32_t*>(smem + C::kOffCorr);
     for (int i = tid; i < 8 * D; i += blockDim.x) {
@@ -497,7 +499,7 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_kernel(const __grid_const
       all_sync(true);  // the table is complete
 
       // ---- pass C: P tiles into TMEM for the P.V MMAs ----
-      const bool corr = hp.zv != 0;  // V zero-point: sum this thread's P bytes
+      const bool corr = ZV && hp.zv != 0;  // V zero-point: sum this thread's P bytes
       uint32_t psum = 0;
       for (int j = first_j(sc); j < T.nkt; j += kTeams) {
         const uint32_t pi = pc + j;  // running P index of this tile
@@ -748,7 +750,7 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_kernel(const __grid_const
         next_slot();
       }
       if (!ok) break;
-      if (hp_s[args.per_head ? T.h : 0].zv != 0) {
+      if (ZV && hp_s[args.per_head ? T.h : 0].zv != 0) {
         // O -= z_v sum_j P_j: one correction tile per softmax team
         for (int t = 0; t < kTeams; ++t, ++pc) {
           const uint32_t pb = pc & (kPBufs - 1);

@@ -88,7 +88,9 @@ enum Bar : int {
   kBarKvFull = 21,  // [stages], then kv_empty[stages]
 };
 
-template <int D>
+// ZV: the kernel instance that supports a V zero-point (the correction tile
+// and the sums of P); the other instance is the plain int8 kernel.
+template <int D, bool ZV = false>
 struct Cfg {
   static constexpr int kStages = (D == 64) ? 8 : 6;
   static constexpr int kOBufs = (D == 64) ? 2 : 1;
@@ -106,7 +108,7 @@ struct Cfg {
   static constexpr int kCorrGroup = 8;
   // probability table, four copies [b][33][kBM] u32 holding P << 8b
   static constexpr uint32_t kPtabBytes = 33 * kBM * 4;
-  static constexpr uint32_t kOffPtab = kOffCorr + 32 * D;
+  static constexpr uint32_t kOffPtab = kOffCorr + (ZV ? 32 * D : 0);
   static constexpr uint32_t kOffRed = kOffPtab + 4 * kPtabBytes;             // [2][kColGroups][kBM] int32
   static constexpr uint32_t kOffLut = kOffRed + 2 * kColGroups * kBM * 4;
   static constexpr uint32_t kOffHp = kOffLut + INTATTN_MAX_CLIPS * 32 * 4;   // head parameters
@@ -150,9 +152,9 @@ __device__ __forceinline__ void walk_schedule(const PrefillArgs& a, BEGIN&& begi
   }
 }
 
-template <int D>
+template <int D, bool ZV>
 __global__ void __launch_bounds__(kThreads, 1) prefill_short_kernel(const __grid_constant__ PrefillArgs args) {
-  using C = Cfg<D>;
+  using C = Cfg<D, ZV>;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
   const uint32_t s_base = smem_u32(smem);
@@ -199,7 +201,7 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_short_kernel(const __grid
   // head parameters in shared memory: a dynamically indexed kernel argument
   // is a constant-bank load that can miss
   for (int i = tid; i < (args.per_head ? args.H : 1); i += blockDim.x) hp_s[i] = args.hp_dev ? args.hp_dev[i] : args.hp[i];
-  {
+  if constexpr (ZV) {
     uint32_t* corr = reinterpret_cast<uint32_t*>(smem + C::kOffCorr);
     for (int i = tid; i < 8 * D; i += blockDim.x) {
       const int key = (4 * i) / D % C::kCorrGroup;
@@ -358,7 +360,7 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_short_kernel(const __grid
       if (!quad_sync(ok)) { ok = false; break; }  // this quadrant's table rows are complete
 
       // ---- pass C: P into TMEM for the P.V MMAs; each S buffer released after its last read ----
-      const bool corr = hp.zv != 0;  // V zero-point: sum this thread's P bytes
+      const bool corr = ZV && hp.zv != 0;  // V zero-point: sum this thread's P bytes
       uint32_t psum = 0;
 #pragma unroll
       for (int j = 0; j < kMaxKeyTiles; ++j) {
@@ -579,7 +581,7 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_short_kernel(const __grid
       next_slot();
       ++pc;
       if (j == T.nkt - 1) {
-        if (hp_s[args.per_head ? T.h : 0].zv != 0) {
+        if (ZV && hp_s[args.per_head ? T.h : 0].zv != 0) {
           // O -= z_v sum_j P_j through the correction tile
           const uint32_t cb = pc & (kPBufs - 1);
           if (!mbar_wait_warp(bar(kBarPFull + cb), (pc / kPBufs) & 1, kRoleMma)) return false;

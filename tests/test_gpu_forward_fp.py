@@ -107,3 +107,39 @@ def test_forward_fp_parameter_out_of_range_is_reported_on_the_device(ia):
     ia.forward_fp(q.cuda(), k.cuda(), v.cuda(), False, [0.03], False, 8.0, out=out)
     assert ia.device_error() == ia.OK
     assert not bool((out == 0x5A).all())
+
+
+ZP_CASES = [  # B, H, Lq, Lk, d, causal, per_head, dtype, K shift, V shift
+    (2, 4, 200, 200, 64, False, True, "bf16", 2.0, -3.0),
+    (1, 3, 130, 300, 128, True, False, "fp16", -1.0, 1.5),
+    (1, 2, 700, 700, 128, True, True, "bf16", 0.5, 4.0),
+]
+
+
+@pytest.mark.parametrize("case", ZP_CASES, ids=lambda c: "B{}H{}Lq{}Lk{}d{}{}{}{}".format(
+    *c[:5], "c" if c[5] else "", "h" if c[6] else "", c[7]))
+def test_forward_fp_with_zero_points_matches_oracle(ia, oracle_mod, case):
+    """intattn_forward_fp_zp: K and V lopsided (shifted) so that their
+    zero-points are far from the middle; equal to oracle quantise (q
+    symmetric, k and v asymmetric) + the oracle forward with those
+    zero-points, and the zero-points copied out equal the oracle's."""
+    import torch
+    B, H, Lq, Lk, d, causal, per_head, dtype, ks, vs = case
+    q, k, v = _inputs((B, H, Lq, d), (B, H, Lk, d), dtype, seed=3300 + Lq + Lk)
+    k = (k.float() + ks).to(k.dtype)
+    v = (v.float() + vs).to(v.dtype)
+    n = H if per_head else 1
+    s_o = np.linspace(0.03, 0.06, n).astype(np.float32)
+    cq, sq = oq.quantize(q.float().numpy(), per_head)
+    ck, sk, zk = oq.quantize_asym(k.float().numpy(), per_head)
+    cv, sv, zv = oq.quantize_asym(v.float().numpy(), per_head)
+    want = oracle_mod.forward(cq, ck, cv, per_head, sq, sk, sv, s_o, causal, 8.0, z_k=zk, z_v=zv)
+    scales = torch.zeros(3 * n, dtype=torch.float32, device="cuda")
+    zps = torch.full((2 * n,), -7, dtype=torch.int32, device="cuda")
+    out = ia.forward_fp(q.cuda(), k.cuda(), v.cuda(), per_head, s_o, causal, 8.0, scales_out=scales,
+                        zero_points=True, zero_points_out=zps)
+    assert ia.device_error() == ia.OK
+    assert np.array_equal(scales.cpu().numpy(), np.concatenate([sq, sk, sv]))
+    assert np.array_equal(zps.cpu().numpy(), np.concatenate([zk, zv]))
+    got = out.cpu().numpy()
+    assert np.array_equal(got, want), f"{int((got != want).sum())} of {got.size} bytes differ from the oracle"
