@@ -91,8 +91,9 @@ typedef struct intattn_scales {
      * else INTATTN_ERR_INVALID_ARG.  The definition then reads
      * S_j = sum_t Q[i,t] (K[j,t] - z_k) and acc_t = sum_j P_j (V[j,t] - z_v).
      * Q stays symmetric int8.  Accepted by the forward, intattn_forward_variant,
-     * intattn_forward_host and the int8 decode; intattn_decode_int4 and
-     * intattn_calibrate_clip return INTATTN_ERR_UNSUPPORTED for them. */
+     * intattn_forward_host and both decodes (intattn_decode_int4: unsigned
+     * nibbles c in [0, 15] with zero-points 0 .. 15 instead of two's complement
+     * nibbles); intattn_calibrate_clip returns INTATTN_ERR_UNSUPPORTED. */
     const int32_t *z_k;
     const int32_t *z_v;
 } intattn_scales_t;

@@ -21,7 +21,10 @@
 // u = x + 8 of its even and of its odd channels (nibble ^ 8: one logic op
 // per 4 channels); dp4a works on u and the bias is removed exactly:
 // q.x = q.u - 8 sum(q), and sum P x = sum P u - 8 sum(P).
-// Zero-points (int8 cache only): u8 K codes need only the dp4a operand type
+// Unsigned int4 codes with zero-points: a nibble c in [0, 15] stands for
+// c - z; the kernels then skip the XOR (u = c) and remove z instead of 8
+// (for K any per-row constant cancels in the gaps, so none is removed).
+// Zero-points of the int8 cache: u8 K codes need only the dp4a operand type
 // (the per-row constant q.z_k cancels in every gap); u8 V codes with
 // zero-point z_v give sum P (v - z_v) = sum P v - z_v sum P, with sum P
 // found by decode_z in a second sweep over the scores once R is known.
@@ -45,7 +48,7 @@ struct DecodeArgs {
   uint32_t* ws_cnt;  // [BH]              arrival tickets
   int32_t* ws_mr;    // [BH, 4]           row max, reciprocal R, sum of P (V zero-point only)
   int32_t BH, H, Lk, Lmax, nsplit, chunk, per_head, ld_s;
-  int32_t k_u8, v_u8;  // int8 cache: K / V codes are u8 (they carry zero-points)
+  int32_t k_u8, v_u8;  // K / V codes are unsigned (u8, or u4 nibbles) with zero-points
   uint32_t lut[INTATTN_MAX_CLIPS][32];  // one exp table per distinct clip threshold
   HeadParamsDev hp[INTATTN_MAX_HEADS];
 };
@@ -91,13 +94,14 @@ __device__ __forceinline__ int32_t dp4a_uu(uint32_t a, uint32_t b, int32_t c) {
   return d;
 }
 
-// 8 packed int4 channels (one word) -> biased bytes u = x + 8 of the even
-// channels (lo) and of the odd channels (hi)
-__device__ __forceinline__ uint32_t nib_lo(uint32_t w) { return (w & 0x0F0F0F0Fu) ^ 0x08080808u; }
-// The high nibbles in place, biased: byte t holds 16 * (x_hi + 8).  Products
-// with it are 16 times the biased ones (one op fewer than shifting down);
-// their sums are divided by 16 exactly at the end.
-__device__ __forceinline__ uint32_t nib_hi16(uint32_t w) { return (w & 0xF0F0F0F0u) ^ 0x80808080u; }
+// 8 packed int4 channels (one word) -> unsigned bytes u of the even channels
+// (lo): u = x + 8 for two's complement nibbles (x8 = 0x08080808), u = c for
+// unsigned ones (x8 = 0).
+__device__ __forceinline__ uint32_t nib_lo(uint32_t w, uint32_t x8) { return (w & 0x0F0F0F0Fu) ^ x8; }
+// The odd channels' nibbles in place: byte t holds 16 u.  Products with it
+// are 16 times the unshifted ones (one op fewer than shifting down); their
+// sums are divided by 16 exactly at the end.
+__device__ __forceinline__ uint32_t nib_hi16(uint32_t w, uint32_t x8) { return (w & 0xF0F0F0F0u) ^ (x8 << 4); }
 
 __device__ __forceinline__ int32_t imax32(int32_t a, int32_t b) { return a > b ? a : b; }
 
@@ -448,7 +452,9 @@ __global__ void __launch_bounds__(kThreads) decode4_qk_kernel(const __grid_const
                           __byte_perm(qa.z, qa.w, 0x6420), __byte_perm(qa.z, qa.w, 0x7531),
                           __byte_perm(qb.x, qb.y, 0x6420), __byte_perm(qb.x, qb.y, 0x7531),
                           __byte_perm(qb.z, qb.w, 0x6420), __byte_perm(qb.z, qb.w, 0x7531)};
-  const int32_t qbias =
+  // unsigned codes: no bias is removed (q.z_k is the same for every key of the row)
+  const uint32_t kx8 = a.k_u8 ? 0u : 0x08080808u;
+  const int32_t qbias = a.k_u8 ? 0 :
       8 * dp4a_ss(qa.x, 0x01010101u, dp4a_ss(qa.y, 0x01010101u, dp4a_ss(qa.z, 0x01010101u, dp4a_ss(qa.w, 0x01010101u,
       dp4a_ss(qb.x, 0x01010101u, dp4a_ss(qb.y, 0x01010101u, dp4a_ss(qb.z, 0x01010101u, dp4a_ss(qb.w, 0x01010101u, 0))))))));
   const int8_t* kbase = a.k + static_cast<size_t>(bh) * a.Lmax * kRowBytes + piece * 16;
@@ -475,8 +481,8 @@ __global__ void __launch_bounds__(kThreads) decode4_qk_kernel(const __grid_const
       int32_t acc = -qbias, acc16 = 0;  // even channels; odd channels x 16
 #pragma unroll
       for (int g = 0; g < 4; ++g) {
-        acc = dp4a_su(qw[2 * g], nib_lo(w[g]), acc);
-        acc16 = dp4a_su(qw[2 * g + 1], nib_hi16(w[g]), acc16);
+        acc = dp4a_su(qw[2 * g], nib_lo(w[g], kx8), acc);
+        acc16 = dp4a_su(qw[2 * g + 1], nib_hi16(w[g], kx8), acc16);
       }
       s[i] = acc + (acc16 >> 4);  // acc16 is a multiple of 16
     }
@@ -665,6 +671,8 @@ __global__ void __launch_bounds__(kThreads, 3) decode4_pv_kernel(const __grid_co
 #pragma unroll
   for (int c = 0; c < 16; ++c) acc[c] = 0;
   int32_t psum = 0;  // sum of this thread's P: the bias correction
+  const uint32_t vx8 = a.v_u8 ? 0u : 0x08080808u;
+  const int32_t vbias = a.v_u8 ? hp.zv : 8;  // what each V code is offset by
   auto octet = [&](int r0, const uint2 (&cur)[8]) {
 #pragma unroll
     for (int hq = 0; hq < 2; ++hq) {  // the two row quads of the octet
@@ -679,10 +687,10 @@ __global__ void __launch_bounds__(kThreads, 3) decode4_pv_kernel(const __grid_co
 #pragma unroll
         for (int e = 0; e < 2; ++e) {
           // e = 1: the odd channels, 16 x biased (accumulators divided by 16 at the end)
-          const uint32_t x0 = e ? nib_hi16(y0) : nib_lo(y0);
-          const uint32_t x1 = e ? nib_hi16(y1) : nib_lo(y1);
-          const uint32_t x2 = e ? nib_hi16(y2) : nib_lo(y2);
-          const uint32_t x3 = e ? nib_hi16(y3) : nib_lo(y3);
+          const uint32_t x0 = e ? nib_hi16(y0, vx8) : nib_lo(y0, vx8);
+          const uint32_t x1 = e ? nib_hi16(y1, vx8) : nib_lo(y1, vx8);
+          const uint32_t x2 = e ? nib_hi16(y2, vx8) : nib_lo(y2, vx8);
+          const uint32_t x3 = e ? nib_hi16(y3, vx8) : nib_lo(y3, vx8);
           // bytes (row i, column c) -> word c holds the 4 rows of column c
           const uint32_t ab_lo = __byte_perm(x0, x1, 0x5140);
           const uint32_t ab_hi = __byte_perm(x0, x1, 0x7362);
@@ -709,7 +717,7 @@ __global__ void __launch_bounds__(kThreads, 3) decode4_pv_kernel(const __grid_co
 #pragma unroll
   for (int s = 0; s < 16; ++s) {
     const int g = s >> 3, e = (s >> 2) & 1, c = s & 3;
-    part[(8 * g + 2 * c + e) * kPartStride + tid] = (e ? (acc[s] >> 4) : acc[s]) - 8 * psum;  // acc >= 0
+    part[(8 * g + 2 * c + e) * kPartStride + tid] = (e ? (acc[s] >> 4) : acc[s]) - vbias * psum;  // acc >= 0
   }
   __syncthreads();
   int32_t* gpart = a.ws_part + (static_cast<size_t>(bh) * a.nsplit + sp) * D;

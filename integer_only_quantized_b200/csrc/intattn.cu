@@ -851,7 +851,14 @@ int intattn_decode(const int8_t* q, const int8_t* k_cache, const int8_t* v_cache
 int intattn_decode_int4(const int8_t* q, const uint8_t* k_cache, const uint8_t* v_cache,
                         const intattn_scales_t* scales, int B, int H, int Lk, int Lmax, int d, float clip_c,
                         int8_t* out, void* workspace, size_t workspace_bytes, intattn_stream_t stream) {
-  if (scales && (scales->z_k || scales->z_v)) return INTATTN_ERR_UNSUPPORTED;  // int4 codes: no zero-points
+  // unsigned int4 codes carry zero-points of 0 .. 15
+  if (scales) {
+    const int n = scales->per_head ? H : 1;
+    for (int i = 0; scales->z_k && i < n && H > 0; ++i)
+      if (scales->z_k[i] < 0 || scales->z_k[i] > 15) return INTATTN_ERR_INVALID_ARG;
+    for (int i = 0; scales->z_v && i < n && H > 0; ++i)
+      if (scales->z_v[i] < 0 || scales->z_v[i] > 15) return INTATTN_ERR_INVALID_ARG;
+  }
   DecodeArgs a;
   DecodeLayout L{};
   bool empty = false;

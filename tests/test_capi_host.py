@@ -160,8 +160,8 @@ def test_quantize_zp_argument_errors_need_no_device(ia):
 
 
 def test_zero_point_argument_errors_need_no_device(ia):
-    """Zero-points out of 0..255 are rejected before any launch; the int4
-    decode and the calibration take no zero-points."""
+    """Zero-points out of 0..255 (0..15 for int4 codes) are rejected before
+    any launch; the calibration takes no zero-points."""
     import numpy as np
     L = ia.lib()
     one = np.array([0.02], np.float32)
@@ -175,9 +175,11 @@ def test_zero_point_argument_errors_need_no_device(ia):
         assert rc == ia.ERR_INVALID_ARG, (zk, zv)
         rc = L.intattn_decode(16, 16, 16, ctypes.byref(sc), 1, 2, 64, 64, 64, 8.0, 16, 256, 1 << 20, None)
         assert rc == ia.ERR_INVALID_ARG, (zk, zv)
+    for zk, zv in ((16, None), (None, 16), (-1, 3)):  # unsigned int4 codes: zero-points 0 .. 15
+        sc, keep = scales(zk, zv)
+        assert L.intattn_decode_int4(16, 16, 16, ctypes.byref(sc), 1, 2, 64, 64, 64, 8.0, 16, 256, 1 << 20,
+                                     None) == ia.ERR_INVALID_ARG
     sc, keep = scales(3, 4)
-    assert L.intattn_decode_int4(16, 16, 16, ctypes.byref(sc), 1, 2, 64, 64, 64, 8.0, 16, 256, 1 << 20,
-                                 None) == ia.ERR_UNSUPPORTED
     clip = np.zeros(1, np.float32)
     assert L.intattn_calibrate_clip(16, 16, ctypes.byref(sc), 1, 2, 64, 64, 64, 0, 4, 4, 0.5, 8.0,
                                     clip.ctypes.data_as(ctypes.POINTER(ctypes.c_float)), None, 256, 1 << 20,

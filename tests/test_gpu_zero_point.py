@@ -162,3 +162,47 @@ def test_forward_host_with_zero_points(ia, oracle_mod):
     out = ia.forward_host(pin(q), pin(k), pin(v), sc, True, 8.0)
     torch.cuda.synchronize()
     assert np.array_equal(out.numpy(), want)
+
+
+def _pack_u4(c):
+    """Unsigned 4-bit codes [..., d] -> bytes [..., d/2], channel 2t in the
+    low nibble of byte t (the int4 cache layout)."""
+    c = np.asarray(c, dtype=np.uint8)
+    assert c.max(initial=0) <= 15
+    return (c[..., 0::2] | (c[..., 1::2] << np.uint8(4))).astype(np.uint8)
+
+
+INT4_CASES = [(4, 3, 1000, 1100, 128, True, "kv"), (2, 2, 4096, 4096, 64, False, "k"),
+              (3, 4, 300, 512, 128, True, "v"), (1, 2, 5000, 5000, 128, True, "kv")]
+
+
+@pytest.mark.parametrize("case", INT4_CASES, ids=lambda c: "B{}H{}Lk{}Lmax{}d{}-{}".format(*c[:5], c[6]))
+def test_decode_int4_with_zero_points_matches_oracle(ia, oracle_mod, case):
+    """Unsigned int4 codes c in [0, 15] with zero-points 0 .. 15 (lopsided
+    code distributions), K, V or both; the other tensor two's complement."""
+    from integer_only_quantized_b200 import workloads as wl
+    B, H, Lk, Lmax, d, per_head, which = case
+    rng = np.random.default_rng(Lk + d + len(which))
+    q = np.clip(np.rint(rng.standard_normal((B, H, 1, d)) * 30), -128, 127).astype(np.int8)
+    n = H if per_head else 1
+    zs = np.array([[0, 15, 7, 3][i % 4] for i in range(n)], np.int32)
+
+    def cache(asym):
+        if asym:
+            zz = zs.reshape(1, -1, 1, 1) if per_head else zs.reshape(1, 1, 1, 1)
+            c = np.clip(np.rint(rng.standard_normal((B, H, Lmax, d)) * 3) + zz, 0, 15).astype(np.uint8)
+            return c, _pack_u4(c), zs
+        x = rng.integers(-8, 8, (B, H, Lmax, d)).astype(np.int8)
+        return x, wl.pack_int4(x), None
+
+    kc, kp, zk = cache("k" in which)
+    vc, vp, zv = cache("v" in which)
+    s_q = np.full(n, 0.02, np.float32)
+    s_k = np.full(n, 0.3, np.float32)
+    s_v = np.full(n, 0.4, np.float32)
+    s_o = np.full(n, 0.02, np.float32)
+    want = oracle_mod.decode(q, kc, vc, per_head, s_q, s_k, s_v, s_o, Lk, 8.0, z_k=zk, z_v=zv)
+    sc = ia.Scales(s_q, s_k, s_v, s_o, per_head=per_head, z_k=zk, z_v=zv)
+    got = ia.decode_int4(_dev(q), _dev(kp), _dev(vp), sc, Lk, 8.0).cpu().numpy()
+    assert ia.device_error() == ia.OK
+    assert np.array_equal(got, want)
