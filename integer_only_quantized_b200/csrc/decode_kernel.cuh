@@ -556,7 +556,7 @@ struct LayoutPv4 {
 // the role of decode_z: m from the chunk maximum, Z and R from the scores it
 // reads anyway to build P.  Same arithmetic as decode_z, bit for bit.
 template <int D, bool kOwnZ>
-__global__ void __launch_bounds__(kThreads, 3) decode4_pv_kernel(const __grid_constant__ DecodeArgs a) {
+__global__ void __launch_bounds__(kThreads, 4) decode4_pv_kernel(const __grid_constant__ DecodeArgs a) {
   using Lt = LayoutPv4<D>;
   constexpr int kRowBytes = D / 2;
   const int bh = blockIdx.y;
