@@ -554,11 +554,12 @@ def run_zero_point(args, ia, dev, stream, world, peak_int8, base_ms):
 def run_calibrate(args, dev, stream, world):
     """Adaptive clip thresholds (intattn_calibrate_clip) on the LLaMA-7B
     causal prefill codes: every 64th query row of each head sampled, the gap
-    to its 32nd largest score.  Each sampled row's scores are recomputed
-    (dp4a) in each of the three radix-select sweeps, so the kernel's work is
-    3 x (sampled rows x valid keys x d) multiply-adds, its K reads served by
-    L2.  Timed with CUDA events around whole calls (the call copies the gaps
-    to the host and synchronises)."""
+    to its 32nd largest score.  Each sampled row's scores are computed once
+    (dp4a, four rows of a head per CTA sharing the K reads) into shared
+    memory, where three radix-select sweeps find the K-th largest: the
+    counted work is sampled rows x valid keys x d multiply-adds.  Timed with
+    CUDA events around whole calls (the call copies the gaps to the host and
+    synchronises)."""
     import torch
 
     import integer_only_quantized_b200 as ia
@@ -589,13 +590,14 @@ def run_calibrate(args, dev, stream, world):
     rows = list(range(stride - 1, w.Lq, stride))
     off = w.Lk - w.Lq
     keys = sum(min(w.Lk, i + off + 1) if w.causal else w.Lk for i in rows) * w.B * w.H
-    ops = 3 * keys * w.d * 2  # three sweeps of int8 multiply-adds
+    ops = keys * w.d * 2  # each sampled score once: int8 multiply-adds
     tops = ops / (ms * 1e-3) / 1e12
     # dp4a issues at half the FP32 rate: 64 per clock per SM, 8 int8 ops each
     peak = 148 * 64 * 8 * 1.965e9 / 1e12
     return {"workload": w.name + f"_keep{keep}_stride{stride}", "ms_per_call": round(ms, 5), "launches_per_call": 2,
             "sampled_rows": len(rows) * w.B * w.H, "scores_per_sweep": keys,
-            "note": "memset of the gap buffer + gap kernel; thresholds from the gaps on the host",
+            "note": "memset of the gap buffer + gap kernel (scores in shared memory, radix select there); "
+                    "thresholds from the gaps on the host",
             "value": round(aggregate_value(ops, world, ms * 1e-3) / 1e12, 3), "unit": "TOPS (dp4a int8)",
             "roofline": {"bound": "alu", "achieved": round(tops, 3), "peak": round(peak, 1), "unit": "TOPS",
                          "frac": round(tops / peak, 4), "peak_source": "148 SMs x 64 dp4a/clk x 8 ops x 1965 MHz",

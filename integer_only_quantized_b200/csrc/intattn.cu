@@ -1091,7 +1091,27 @@ int intattn_calibrate_clip(const int8_t* q, const int8_t* k, const intattn_scale
     intattn::CalibArgs a{q, k, dG, Lq, Lk, d, causal ? 1 : 0, keep, stride};
     int rc = note_launch(cudaMemsetAsync(dG, 0, static_cast<size_t>(BH) * sizeof(int32_t), st));
     if (rc) return rc;
-    intattn::calib::gap_kernel<<<dim3(rows, static_cast<unsigned>(BH)), intattn::calib::kThreads, 0, st>>>(a);
+    // scores computed once per sampled row, in shared memory, while a CTA's
+    // rows fit; else recomputed in each radix pass
+    const int per_cta = static_cast<int>(std::min<long long>(
+        intattn::calib::kRowsMax, (200ll * 1024) / (4ll * (((Lk + 3) & ~3)))));
+    if (per_cta >= 1) {
+      const size_t smem = static_cast<size_t>(per_cta) * (((Lk + 3) & ~3)) * 4;
+      static bool attr_set[64] = {};
+      int dev = 0;
+      if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return INTATTN_ERR_CUDA;
+      if (!attr_set[dev]) {
+        if ((rc = note_launch(cudaFuncSetAttribute(intattn::calib::gap_rows_kernel,
+                                                   cudaFuncAttributeMaxDynamicSharedMemorySize, 200 * 1024))))
+          return rc;
+        attr_set[dev] = true;
+      }
+      const unsigned blocks = static_cast<unsigned>((rows + per_cta - 1) / per_cta);
+      intattn::calib::gap_rows_kernel<<<dim3(blocks, static_cast<unsigned>(BH)), intattn::calib::kRowsThreads, smem,
+                                        st>>>(a, per_cta, rows);
+    } else {
+      intattn::calib::gap_kernel<<<dim3(rows, static_cast<unsigned>(BH)), intattn::calib::kThreads, 0, st>>>(a);
+    }
     if ((rc = note_launch(cudaGetLastError()))) return rc;
     if ((rc = note_launch(cudaMemcpyAsync(G.data(), dG, G.size() * sizeof(int32_t), cudaMemcpyDeviceToHost, st))))
       return rc;

@@ -35,6 +35,8 @@ CASES = [  # B, H, Lq, Lk, d, causal, per_head, keep, stride
     (2, 2, 129, 129, 64, True, False, 1, 1),
     (1, 3, 50, 50, 128, True, True, 64, 3),     # keep larger than the early causal rows
     (1, 2, 40, 40, 64, False, True, 5, 64),     # stride beyond Lq: no sampled row, c = c_min
+    (2, 3, 517, 517, 128, True, True, 20, 5),   # 103 sampled rows: shared-memory kernel, ragged last CTA
+    (1, 1, 52000, 52000, 64, True, True, 8, 5200),  # rows too long for shared memory: the recomputing kernel
 ]
 
 
