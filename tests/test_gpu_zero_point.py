@@ -206,3 +206,40 @@ def test_decode_int4_with_zero_points_matches_oracle(ia, oracle_mod, case):
     got = ia.decode_int4(_dev(q), _dev(kp), _dev(vp), sc, Lk, 8.0).cpu().numpy()
     assert ia.device_error() == ia.OK
     assert np.array_equal(got, want)
+
+
+def test_per_head_clips_with_zero_points(ia, oracle_mod):
+    """Per-head clip thresholds and per-head zero-points together: each head
+    equals the oracle run on that head alone with its threshold."""
+    B, H, L, d = 2, 4, 300, 64
+    zk, zv = _zp("mid", H, True), _zp("edges", H, True)
+    q, k, v, s_q, s_k, s_v, s_o = _inputs(21, B, H, L, L, d, True, zk, zv)
+    clips = np.array([4.0, 6.0, 9.0, 12.0], np.float32)
+    sc = ia.Scales(s_q, s_k, s_v, s_o, per_head=True, clip=clips, z_k=zk, z_v=zv)
+    for variant in (ia.VARIANT_AUTO, ia.VARIANT_THREE_PASS):
+        got = ia.forward(_dev(q), _dev(k), _dev(v), sc, True, 8.0, variant=variant).cpu().numpy()
+        for h in range(H):
+            want = oracle_mod.forward(q[:, h:h + 1], k[:, h:h + 1], v[:, h:h + 1], True, s_q[h:h + 1],
+                                      s_k[h:h + 1], s_v[h:h + 1], s_o[h:h + 1], True, float(clips[h]),
+                                      z_k=zk[h:h + 1], z_v=zv[h:h + 1])
+            assert np.array_equal(got[:, h:h + 1], want), (variant, h)
+
+
+def test_static_scratch_decode_with_zero_points(ia, oracle_mod):
+    """The allocation-free decode takes the same zero-point scales."""
+    import ctypes
+
+    import torch
+    B, H, Lk, Lmax, d = 3, 2, 900, 1024, 128
+    zk, zv = _zp("mid", H, True), _zp("edges", H, True)
+    q, kc, vc, s_q, s_k, s_v, s_o = _inputs(22, B, H, 1, Lmax, d, True, zk, zv)
+    want = oracle_mod.decode(q, kc, vc, True, s_q, s_k, s_v, s_o, Lk, 8.0, z_k=zk, z_v=zv)
+    s, keep = ia.Scales(s_q, s_k, s_v, s_o, per_head=True, z_k=zk, z_v=zv)._c()
+    qd, kd, vd = _dev(q), _dev(kc), _dev(vc)
+    out = torch.full_like(qd, 99)
+    rc = ia.lib().intattn_decode_static_scratch(qd.data_ptr(), kd.data_ptr(), vd.data_ptr(), ctypes.byref(s), B, H,
+                                                Lk, Lmax, d, 8.0, out.data_ptr(),
+                                                torch.cuda.current_stream().cuda_stream)
+    torch.cuda.synchronize()
+    assert rc == ia.OK
+    assert np.array_equal(out.cpu().numpy(), want)
