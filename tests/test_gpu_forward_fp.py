@@ -143,3 +143,38 @@ def test_forward_fp_with_zero_points_matches_oracle(ia, oracle_mod, case):
     assert np.array_equal(zps.cpu().numpy(), np.concatenate([zk, zv]))
     got = out.cpu().numpy()
     assert np.array_equal(got, want), f"{int((got != want).sum())} of {got.size} bytes differ from the oracle"
+
+
+@pytest.mark.parametrize("zero_points", [False, True], ids=["symmetric", "zero_points"])
+def test_forward_fp_full_llama_shape(ia, oracle_mod, zero_points):
+    """The headline shape from bf16 activations (B1 H32 L8192 d128, causal,
+    per head, clip 10), as the benchmark's forward_fp line runs it: every
+    output byte, the scales and the zero-points against oracle quantise +
+    the oracle forward.  With zero-points, K and V are shifted so that their
+    ranges are lopsided."""
+    import torch
+    B, H, L, d = 1, 32, 8192, 128
+    q, k, v = _inputs((B, H, L, d), (B, H, L, d), "bf16", seed=3700 + int(zero_points))
+    if zero_points:
+        k = (k.float() + torch.linspace(-3.0, 3.0, H).view(1, H, 1, 1)).to(k.dtype)
+        v = (v.float() + torch.linspace(2.0, -2.0, H).view(1, H, 1, 1)).to(v.dtype)
+    s_o = np.linspace(0.02, 0.05, H).astype(np.float32)
+    cq, sq = oq.quantize(q.float().numpy(), True)
+    if zero_points:
+        ck, sk, zk = oq.quantize_asym(k.float().numpy(), True)
+        cv, sv, zv = oq.quantize_asym(v.float().numpy(), True)
+        want = oracle_mod.forward(cq, ck, cv, True, sq, sk, sv, s_o, True, 10.0, z_k=zk, z_v=zv)
+    else:
+        ck, sk = oq.quantize(k.float().numpy(), True)
+        cv, sv = oq.quantize(v.float().numpy(), True)
+        want = oracle_mod.forward(cq, ck, cv, True, sq, sk, sv, s_o, True, 10.0)
+    scales = torch.zeros(3 * H, dtype=torch.float32, device="cuda")
+    zps = torch.full((2 * H,), -7, dtype=torch.int32, device="cuda")
+    out = ia.forward_fp(q.cuda(), k.cuda(), v.cuda(), True, s_o, True, 10.0, scales_out=scales,
+                        zero_points=zero_points, zero_points_out=zps if zero_points else None)
+    assert ia.device_error() == ia.OK
+    assert np.array_equal(scales.cpu().numpy(), np.concatenate([sq, sk, sv]))
+    if zero_points:
+        assert np.array_equal(zps.cpu().numpy(), np.concatenate([zk, zv]))
+    got = out.cpu().numpy()
+    assert np.array_equal(got, want), f"{int((got != want).sum())} of {got.size} bytes differ from the oracle"

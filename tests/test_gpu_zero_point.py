@@ -243,3 +243,26 @@ def test_static_scratch_decode_with_zero_points(ia, oracle_mod):
     torch.cuda.synchronize()
     assert rc == ia.OK
     assert np.array_equal(out.cpu().numpy(), want)
+
+
+def test_full_llama_shape_with_per_head_zero_points(ia, oracle_mod):
+    """The headline shape (B1 H32 L8192 d128, causal, per head, clip 10) with K
+    and V as u8 codes around per-head zero-points that include 0 and 255:
+    every output byte against the oracle, which computes q.(k - z_k) and
+    P.(v - z_v) literally."""
+    B, H, L, d = 1, 32, 8192, 128
+    base = [0, 255, 1, 254, 128, 127]
+    zk = np.array([base[h] if h < len(base) else (37 * h + 11) % 256 for h in range(H)], np.int32)
+    zv = np.array([base[-1 - h] if h < len(base) else (91 * h + 200) % 256 for h in range(H)], np.int32)
+    q, k, v, s_q, s_k, s_v, s_o = _inputs(777, B, H, L, L, d, True, zk, zv)
+    # a query scale ten times the small cases': over 8192 keys the rows are then
+    # peaked enough that the outputs spread over the int8 range (mean |out| ~ 18,
+    # a few saturate) instead of averaging to near 0
+    s_q = s_q * 10
+    want = oracle_mod.forward(q, k, v, True, s_q, s_k, s_v, s_o, True, 10.0, z_k=zk, z_v=zv)
+    sc = ia.Scales(s_q, s_k, s_v, s_o, per_head=True, z_k=zk, z_v=zv)
+    got = ia.forward(_dev(q), _dev(k), _dev(v), sc, True, 10.0).cpu().numpy()
+    assert ia.device_error() == ia.OK
+    if not np.array_equal(got, want):
+        bad = np.argwhere(got != want)
+        raise AssertionError(f"{len(bad)} of {got.size} bytes differ; first (b, h, i, t) {bad[0].tolist()}")
