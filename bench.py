@@ -548,7 +548,8 @@ def run_zero_point(args, ia, dev, stream, world, peak_int8, base_ms):
             "note": "u8 K and V with zero-point 128 per head: the MMA reads u8, and z_v sum P is subtracted "
                     "through one correction MMA per softmax team per query tile",
             "roofline": {"bound": "tensor", "achieved": round(tops, 3), "peak": round(peak_int8, 1), "unit": "TOPS",
-                         "frac": round(tops / peak_int8, 4)}}
+                         "frac": round(tops / peak_int8, 4),
+                         "traffic": kernel_traffic("prefill_kernel", w.name + "_u8_kv_zero_points")}}
 
 
 def run_calibrate(args, dev, stream, world):
