@@ -287,3 +287,50 @@ def test_short_rows_extreme_codes(ia, oracle_mod, d):
     for xx in cases:
         _assert_equal(_variant_forward(ia, xx, w, ia.VARIANT_SHORT_ROWS), _oracle_forward(oracle_mod, xx, w),
                       "extreme")
+
+
+# ------------------------------------------------ the largest key count (Lk = 65535)
+
+@pytest.mark.parametrize("causal", [False, True], ids=["full", "causal"])
+def test_max_key_length_all_equal_rows(ia, oracle_mod, causal):
+    """Lk = 65535, the largest the definition allows.  Head 0 has q = 0, so
+    every score is 0 and each row's sum is 32768 times its visible keys, up
+    to 32768 * 65535 = 2^31 - 32768 (the bound that limits Lk; every P is
+    then 0).  Head 1 keeps random queries at ten times the query scale, so
+    its rows are peaked enough for outputs away from 0.  Both the automatic
+    kernel and the three-pass kernel against the oracle."""
+    import dataclasses
+    w = wl.custom_workload("max_lk_equal", 1, 2, 130, 65535, 64, causal, per_head=True, index=4100 + causal)
+    x = wl.make_inputs(w)
+    q = x.q.copy()
+    q[:, 0] = 0
+    s_q = x.s_q.copy()
+    s_q[1] *= 10
+    xx = dataclasses.replace(x, q=q, s_q=s_q)
+    want = _oracle_forward(oracle_mod, xx, w)
+    for variant in (ia.VARIANT_AUTO, ia.VARIANT_THREE_PASS):
+        _assert_equal(_variant_forward(ia, xx, w, variant), want, f"Lk 65535 all-equal, variant {variant}")
+
+
+def test_max_key_length_causal_prefill(ia, oracle_mod):
+    """Lq = Lk = 65535, causal, random codes: 512 query tiles of 1..512 key
+    tiles, the last one ragged (127 rows), every output byte."""
+    w = wl.custom_workload("max_lk_causal", 1, 1, 65535, 65535, 64, True, index=4110)
+    x = wl.make_inputs(w)
+    _assert_equal(_gpu_forward(ia, x, w, guard=4096), _oracle_forward(oracle_mod, x, w), "Lq = Lk = 65535 causal")
+
+
+@pytest.mark.parametrize("bits", [8, 4])
+def test_max_key_length_decode(ia, oracle_mod, bits):
+    """One query over 65535 cached keys (128 split-K chunks for int8), int8 and int4 caches."""
+    w = wl.custom_workload("max_lk_decode", 2, 2, 1, 65535, 128, False, per_head=True, clip_c=10.0,
+                           index=4120 + bits, decode=True, Lmax=65536, kv_bits=bits)
+    x = wl.make_inputs(w)
+    sc = ia.Scales(x.s_q, x.s_k, x.s_v, x.s_o, per_head=True)
+    if bits == 8:
+        out = ia.decode(_dev(x.q), _dev(x.k), _dev(x.v), sc, w.Lk, w.clip_c)
+    else:
+        out = ia.decode_int4(_dev(x.q), _dev(wl.pack_int4(x.k)), _dev(wl.pack_int4(x.v)), sc, w.Lk, w.clip_c)
+    assert ia.device_error() == ia.OK
+    want = oracle_mod.decode(x.q, x.k, x.v, True, x.s_q, x.s_k, x.s_v, x.s_o, w.Lk, w.clip_c)
+    _assert_equal(out.cpu().numpy(), want, f"decode Lk 65535 int{bits}")
